@@ -1,0 +1,324 @@
+"""CPU oracle for the FP8 MoE expert layer -- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, the smoke check and the benchmark's CPU-baseline leg may import
+this package. The product library (fp8_grouped_gemm_fp32_b200) never does,
+and the two share no code: this package wraps the plain C in moe_oracle.c
+(see moe_oracle.h for the page citations and the readings it follows) and
+composes its steps with numpy.
+
+Parity pins for every function here are in tests/test_oracle_*.py. One part
+is "parity unpinned" beyond invariants and special cases: the end-to-end
+values of y for general inputs (the pages print no worked numeric example).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_HDR = os.path.join(_HERE, "moe_oracle.h")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+GROUP = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c with gcc (no contraction, no fast-math)."""
+    stale = (not os.path.exists(_LIB) or
+             os.path.getmtime(_LIB) < max(os.path.getmtime(_SRC), os.path.getmtime(_HDR)))
+    if force or stale:
+        tmp = _LIB + ".tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-ffp-contract=off", "-fno-fast-math",
+                               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = ctypes.CDLL(build())
+            _declare(_lib)
+    return _lib
+
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_i64 = ctypes.c_int64
+
+
+def _declare(L):
+    L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_decode.restype = ctypes.c_double
+    L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+    L.orc_e4m3_encode.restype = ctypes.c_uint8
+    L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    L.orc_bf16_to_f32.restype = ctypes.c_float
+    L.orc_f64_to_bf16.argtypes = [ctypes.c_double]
+    L.orc_f64_to_bf16.restype = ctypes.c_uint16
+    L.orc_router_logits.argtypes = [_i, _i, _i, _p, _p, _p, _p, _i]
+    L.orc_topk_softmax.argtypes = [_i, _i, _i, _p, _p, _p]
+    L.orc_route_hash.argtypes = [_i, _i, _p, _p, _p]
+    L.orc_capacity.argtypes = [_i, _i, _i, _i, _i]
+    L.orc_capacity.restype = _i64
+    L.orc_dispatch.argtypes = [_i, _i, _i, _p, _i64, _i, _i, _i, _i64, _p, _p, _p, _p, _p]
+    L.orc_dispatch.restype = _i
+    L.orc_quant_rows.argtypes = [_i64, _i, _p, _p, _p]
+    L.orc_expert_rows.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i]
+    L.orc_grouped_gemm.argtypes = [_i, _i, _i, _i, _p, _p, _p, _i, _p, _p, _i, _p, _p, _i]
+    L.orc_combine.argtypes = [_i, _i, _i, _p, _p, _p, _p]
+
+
+def _ptr(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+# ---------------------------------------------------------------- scalars
+def e4m3_decode(code: int) -> float:
+    return lib().orc_e4m3_decode(code)
+
+
+def e4m3_encode(v: float) -> int:
+    return lib().orc_e4m3_encode(v)
+
+
+def e4m3_decode_array(codes: np.ndarray) -> np.ndarray:
+    table = np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def e4m3_encode_array(v: np.ndarray) -> np.ndarray:
+    L = lib()
+    flat = np.asarray(v, dtype=np.float32).ravel()
+    return np.array([L.orc_e4m3_encode(float(x)) for x in flat], dtype=np.uint8).reshape(np.shape(v))
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    L = lib()
+    flat = np.asarray(v, dtype=np.float64).ravel()
+    return np.array([L.orc_f64_to_bf16(float(x)) for x in flat], dtype=np.uint16).reshape(np.shape(v))
+
+
+# ---------------------------------------------------------------- steps
+def router_logits(x_bf16_bits: np.ndarray, Wg: np.ndarray, bias: Optional[np.ndarray],
+                  nthreads: Optional[int] = None) -> np.ndarray:
+    x = _c(x_bf16_bits, np.uint16)
+    Wg = _c(Wg, np.float32)
+    T, H = x.shape
+    E = Wg.shape[0]
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((T, E), dtype=np.float32)
+    lib().orc_router_logits(T, H, E, _ptr(x), _ptr(Wg), _ptr(b), _ptr(out), nthreads or default_threads())
+    return out
+
+
+def topk_softmax(logits: np.ndarray, k: int):
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float32)
+    lib().orc_topk_softmax(T, E, k, _ptr(logits), _ptr(idx), _ptr(w))
+    return idx, w
+
+
+def route_hash(token_ids: np.ndarray, E: int):
+    tid = _c(token_ids, np.int32)
+    T = tid.shape[0]
+    idx = np.empty((T, 1), dtype=np.int32)
+    w = np.empty((T, 1), dtype=np.float32)
+    lib().orc_route_hash(T, E, _ptr(tid), _ptr(idx), _ptr(w))
+    return idx, w
+
+
+def capacity(T: int, k: int, E: int, cap_num: int, cap_den: int) -> int:
+    return int(lib().orc_capacity(T, k, E, cap_num, cap_den))
+
+
+def dispatch(topk_idx: np.ndarray, E: int, cap: int, layout: int, pad: int, masked_max_m: int,
+             rows_cap: int):
+    idx = _c(topk_idx, np.int32)
+    T, k = idx.shape
+    counts = np.empty(E, dtype=np.int32)
+    kept = np.empty(E, dtype=np.int32)
+    offsets = np.empty(E + 1, dtype=np.int32)
+    row_src = np.empty(rows_cap, dtype=np.int32)
+    slot_row = np.empty(T * k, dtype=np.int32)
+    overflow = lib().orc_dispatch(T, k, E, _ptr(idx), cap, layout, pad, masked_max_m, rows_cap,
+                                  _ptr(counts), _ptr(kept), _ptr(offsets), _ptr(row_src), _ptr(slot_row))
+    return dict(counts=counts, kept=kept, offsets=offsets, row_src=row_src, slot_row=slot_row,
+                overflow=bool(overflow))
+
+
+def quant_rows(v: np.ndarray):
+    v = _c(v, np.float32)
+    rows, K = v.shape
+    q = np.empty((rows, K), dtype=np.uint8)
+    s = np.empty((rows, K // GROUP), dtype=np.float32)
+    lib().orc_quant_rows(rows, K, _ptr(v), _ptr(q), _ptr(s))
+    return q, s
+
+
+def expert_rows(xq, xs, W1q, S1, W3q, S3, W2q, S2, nthreads: Optional[int] = None):
+    xq = _c(xq, np.uint8)
+    xs = _c(xs, np.float32)
+    n, H = xq.shape
+    I = W1q.shape[0]
+    args = [_c(a, t) for a, t in ((W1q, np.uint8), (S1, np.float32), (W3q, np.uint8), (S3, np.float32),
+                                  (W2q, np.uint8), (S2, np.float32))]
+    hq = np.empty((n, I), dtype=np.uint8)
+    hs = np.empty((n, I // GROUP), dtype=np.float32)
+    o = np.empty((n, H), dtype=np.uint16)
+    lib().orc_expert_rows(n, H, I, _ptr(xq), _ptr(xs), *[_ptr(a) for a in args],
+                          _ptr(hq), _ptr(hs), _ptr(o), nthreads or default_threads())
+    return hq, hs, o
+
+
+def grouped_gemm(layout: int, E: int, N: int, K: int, A, As, group_info, M_rows: int, B, Bs,
+                 epilogue: int, nthreads: Optional[int] = None):
+    """Oracle of moe_grouped_gemm_fp8. Rows outside every group are left 0."""
+    A = _c(A, np.uint8)
+    As = _c(As, np.float32)
+    gi = _c(group_info, np.int32)
+    B = _c(B, np.uint8)
+    Bs = _c(Bs, np.float32)
+    rows = A.shape[0] if layout == 0 else E * M_rows
+    if epilogue == 0:
+        D = np.zeros((rows, N), dtype=np.uint16)
+        Ds = None
+    else:
+        D = np.zeros((rows, N // 2), dtype=np.uint8)
+        G = N // 2 // GROUP
+        Ds = np.zeros((G, M_rows) if layout == 0 else (E, G, M_rows), dtype=np.float32)
+    lib().orc_grouped_gemm(layout, E, N, K, _ptr(A), _ptr(As), _ptr(gi), M_rows, _ptr(B), _ptr(Bs),
+                           epilogue, _ptr(D), _ptr(Ds), nthreads or default_threads())
+    return D, Ds
+
+
+def combine(slot_row: np.ndarray, topk_w: np.ndarray, O: np.ndarray, T: int, k: int) -> np.ndarray:
+    sr = _c(slot_row, np.int32)
+    w = _c(topk_w, np.float32)
+    O = _c(O, np.uint16)
+    H = O.shape[1]
+    y = np.empty((T, H), dtype=np.uint16)
+    lib().orc_combine(T, k, H, _ptr(sr), _ptr(w), _ptr(O), _ptr(y))
+    return y
+
+
+# ---------------------------------------------------------------- pipeline
+def route(cfg, x_bits, Wg, bias, token_ids, nthreads=None):
+    """Routing step of the layer: (topk_idx [T,k], topk_w [T,k], logits or None)."""
+    if cfg.routing == "hash":
+        idx, w = route_hash(token_ids, cfg.E)
+        return idx, w, None
+    logits = router_logits(x_bits, Wg, bias, nthreads)
+    idx, w = topk_softmax(logits, cfg.k)
+    return idx, w, logits
+
+
+def permute(cfg, x_bits, topk_idx, rows_cap: int, pad: int = GROUP):
+    """Dispatch + activation quantisation in the boundary's layout:
+    Aq [rows_cap, H] (masked: [E*Mmax, H]) and As K-block-major [H/128][ld]
+    (masked: [E][H/128][Mmax]); padding rows hold code 0 and scale 1.0."""
+    T, H = x_bits.shape
+    layout = 1 if cfg.layout == "masked" else 0
+    cap = capacity(T, topk_idx.shape[1], cfg.E, cfg.cap_num, cfg.cap_den)
+    d = dispatch(topk_idx, cfg.E, cap, layout, pad, cfg.masked_max_m, rows_cap)
+    xq, xs = quant_rows(bf16_bits_to_f32(x_bits))
+    k = topk_idx.shape[1]
+    G = H // GROUP
+    Aq = np.zeros((rows_cap, H), dtype=np.uint8)
+    src = d["row_src"]
+    valid = src >= 0
+    tok = np.where(valid, src // k, 0)
+    Aq[valid] = xq[tok[valid]]
+    if layout == 0:
+        As = np.ones((G, rows_cap), dtype=np.float32)
+        As[:, valid] = xs[tok[valid]].T
+    else:
+        M = cfg.masked_max_m
+        As = np.ones((cfg.E, G, M), dtype=np.float32)
+        rows = np.nonzero(valid)[0]
+        As[rows // M, :, rows % M] = xs[tok[rows]]
+    d.update(cap=cap, Aq=Aq, As=As, xq=xq, xs=xs)
+    return d
+
+
+def expert_outputs_for_rows(inp, rows_by_expert, xq, xs, nthreads=None):
+    """{expert: (token list)} -> {expert: o bf16 [n, H]} through orc_expert_rows."""
+    out = {}
+    for e, toks in rows_by_expert.items():
+        toks = np.asarray(toks, dtype=np.int64)
+        _, _, o = expert_rows(xq[toks], xs[toks], inp["W1q"][e], inp["S1"][e], inp["W3q"][e], inp["S3"][e],
+                              inp["W2q"][e], inp["S2"][e], nthreads)
+        out[e] = o
+    return out
+
+
+def forward(cfg, inp: dict, tokens: Optional[np.ndarray] = None, rows_cap: Optional[int] = None,
+            nthreads=None):
+    """The whole layer. `inp` holds numpy arrays: x (bf16 bits [T,H]), Wg, bias,
+    token_ids, W1q, S1, W3q, S3, W2q, S2 (natural, non-interleaved layout).
+    With `tokens`, y is evaluated only for those tokens (routing, capacity and
+    permutation still run over all T, since ranks are global); rows of y for
+    other tokens are left 0. Returns a dict of every intermediate."""
+    T = inp["x"].shape[0]
+    idx, w, logits = route(cfg, inp["x"], inp["Wg"], inp["bias"], inp["token_ids"], nthreads)
+    k = idx.shape[1]
+    if rows_cap is None:
+        rows_cap = (cfg.E * cfg.masked_max_m if cfg.layout == "masked"
+                    else -(-(T * k + cfg.E * (GROUP - 1)) // GROUP) * GROUP)
+    d = permute(cfg, inp["x"], idx, rows_cap)
+    sel = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    by_e = {}
+    for t in sel:
+        for j in range(k):
+            if d["slot_row"][t * k + j] >= 0:
+                by_e.setdefault(int(idx[t, j]), []).append(int(t))
+    outs = expert_outputs_for_rows(inp, by_e, d["xq"], d["xs"], nthreads)
+    H = inp["x"].shape[1]
+    O = np.zeros((rows_cap, H), dtype=np.uint16)
+    for e, toks in by_e.items():
+        for n, t in enumerate(toks):
+            j = int(np.nonzero(idx[t] == e)[0][0])
+            O[d["slot_row"][t * k + j]] = outs[e][n]
+    y_all = combine(d["slot_row"], w, O, T, k)
+    y = np.zeros_like(y_all)
+    y[sel] = y_all[sel]
+    d.update(topk_idx=idx, topk_w=w, logits=logits, O=O, y=y, tokens=sel)
+    return d
+
+
+def moe_inputs_to_numpy(inp) -> dict:
+    """torch MoeInputs -> numpy dict (bit-preserving views; host copies)."""
+    import torch
+    return dict(
+        x=inp.x.detach().cpu().view(torch.int16).numpy().view(np.uint16),
+        Wg=inp.Wg.detach().cpu().numpy(), bias=inp.bias.detach().cpu().numpy(),
+        token_ids=inp.token_ids.detach().cpu().numpy(),
+        W1q=inp.W1q.detach().cpu().numpy(), S1=inp.S1.detach().cpu().numpy(),
+        W3q=inp.W3q.detach().cpu().numpy(), S3=inp.S3.detach().cpu().numpy(),
+        W2q=inp.W2q.detach().cpu().numpy(), S2=inp.S2.detach().cpu().numpy())

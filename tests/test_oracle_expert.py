@@ -1,0 +1,154 @@
+"""Pins for the oracle's expert math and the whole layer:
+
+* E = 1, k = 1 reduces the layer to one dense SwiGLU FFN (weights exactly 1);
+  compared with torch float64 matmuls and torch's silu.
+* Concat(E_1(T_1), ..., E_E(T_E)) (MegaMoE page, section 2.1): the grouped
+  GEMM over the permuted buffer equals one dense float64 matmul per expert
+  over that expert's gathered rows.
+* Brute force of y = sum_{i in TopK} G(x)_i E_i(x) per token on tiny inputs,
+  sharing nothing with the grouped code path (fp64 logits, per-token loops).
+
+The torch reference below re-derives the storage points the boundary fixes
+(x and h in E4M3 with 1x128 scales, o in bf16) with torch casts.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_grouped_gemm_fp32_b200.inputs import MoeConfig, make_inputs, interleave_w13
+
+
+def _deq_w(q, s):
+    """torch: E4M3 codes * 128x128 block scales, rounded to fp32, as float64."""
+    v = torch.from_numpy(np.ascontiguousarray(q)).view(torch.float8_e4m3fn).to(torch.float32)
+    N, K = v.shape
+    sc = torch.from_numpy(np.ascontiguousarray(s)).repeat_interleave(128, 0).repeat_interleave(128, 1)
+    return (v * sc).to(torch.float64)
+
+
+def _quant_torch(v32):
+    """torch: 1x128 group quantisation (scale = amax/448 in fp32, RNE e4m3 cast)."""
+    v = v32.reshape(v32.shape[0], -1, 128)
+    amax = v.abs().amax(-1)
+    s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    q = (v / s[..., None]).to(torch.float8_e4m3fn)
+    deq = (q.to(torch.float32) * s[..., None]).reshape(v32.shape)
+    return deq.to(torch.float64)
+
+
+def _ffn_torch(x_bits, W1q, S1, W3q, S3, W2q, S2):
+    x = torch.from_numpy(oracle.bf16_bits_to_f32(x_bits))
+    xd = _quant_torch(x)
+    a = xd @ _deq_w(W1q, S1).T
+    b = xd @ _deq_w(W3q, S3).T
+    h = (torch.nn.functional.silu(a) * b).to(torch.float32)
+    o = _quant_torch(h) @ _deq_w(W2q, S2).T
+    return o
+
+
+def _close_bf16(ours_bits, ref64, frac_equal=0.999):
+    ours = oracle.bf16_bits_to_f32(ours_bits).astype(np.float64)
+    ref_b = oracle.bf16_bits_to_f32(oracle.f64_to_bf16_bits(ref64)).astype(np.float64)
+    diff = np.abs(ours - ref_b)
+    ulp = np.abs(ref_b) * 2.0 ** -7 + 1e-30
+    assert np.all(diff <= ulp * 1.01)                   # at most one bf16 step apart
+    assert np.mean(ours_bits == oracle.f64_to_bf16_bits(ref64)) >= frac_equal
+
+
+@pytest.fixture(scope="module")
+def dense_inputs():
+    cfg = MoeConfig("dense", T=64, H=256, E=1, I=256, k=1, bias="uniform", seed=123)
+    return cfg, oracle.moe_inputs_to_numpy(make_inputs(cfg))
+
+
+def test_dense_reduction_E1_k1(dense_inputs):
+    cfg, inp = dense_inputs
+    out = oracle.forward(cfg, inp)
+    assert np.all(out["topk_idx"] == 0) and np.all(out["topk_w"] == 1.0)
+    ref = _ffn_torch(inp["x"], inp["W1q"][0], inp["S1"][0], inp["W3q"][0], inp["S3"][0],
+                     inp["W2q"][0], inp["S2"][0]).numpy()
+    _close_bf16(out["y"], ref)
+
+
+def test_grouped_gemm_equals_per_expert_dense_gemms():
+    cfg = MoeConfig("g", T=96, H=256, E=4, I=128, k=2, bias="uniform", seed=5)
+    t = make_inputs(cfg)
+    inp = oracle.moe_inputs_to_numpy(t)
+    idx, w, _ = oracle.route(cfg, inp["x"], inp["Wg"], inp["bias"], inp["token_ids"])
+    rows_cap = -(-(cfg.T * cfg.k + cfg.E * 127) // 128) * 128
+    d = oracle.permute(cfg, inp["x"], idx, rows_cap)
+    off = d["offsets"]
+    # down-projection-shaped grouped GEMM (epilogue 0: bf16 out), B = W2 stacks, K = H here
+    B = np.ascontiguousarray(inp["W1q"])          # [E, I, H] used as a plain [E, N, K] operand
+    Bs = np.ascontiguousarray(inp["S1"])
+    D, _ = oracle.grouped_gemm(0, cfg.E, cfg.I, cfg.H, d["Aq"], d["As"], off, rows_cap, B, Bs, 0)
+    for e in range(cfg.E):
+        rows = slice(off[e], off[e + 1])
+        A = torch.from_numpy(d["Aq"][rows]).view(torch.float8_e4m3fn).to(torch.float32)
+        sA = torch.from_numpy(d["As"][:, rows].T.copy()).repeat_interleave(128, 1)
+        ref = ((A * sA).to(torch.float64) @ _deq_w(B[e], Bs[e]).T).numpy()
+        _close_bf16(D[rows], ref)
+    # the SwiGLU epilogue over interleaved W1|W3 equals the per-row expert function
+    W13, S13 = interleave_w13(t.W1q, t.S1, t.W3q, t.S3)
+    Dq, Ds = oracle.grouped_gemm(0, cfg.E, 2 * cfg.I, cfg.H, d["Aq"], d["As"], off, rows_cap,
+                                 W13.numpy(), S13.numpy(), 1)
+    for e in range(cfg.E):
+        r0, r1 = off[e], off[e] + d["kept"][e]
+        xs = np.ascontiguousarray(d["As"][:, r0:r1].T)
+        hq, hs, _ = oracle.expert_rows(d["Aq"][r0:r1], xs, inp["W1q"][e], inp["S1"][e], inp["W3q"][e],
+                                       inp["S3"][e], inp["W2q"][e], inp["S2"][e])
+        assert np.array_equal(Dq[r0:r1], hq) and np.array_equal(Ds[:, r0:r1].T, hs)
+
+
+def _brute_layer(cfg, inp, tokens):
+    """Per token, straight from the formulas: fp64 logits, softmax over all E, top-k
+    (ties to lower index), renormalise, y = sum_i w_i * E_i(x) with each expert
+    evaluated on this one token."""
+    x_bits = inp["x"]
+    xf = oracle.bf16_bits_to_f32(x_bits).astype(np.float64)
+    out = {}
+    for t in tokens:
+        l = xf[t] @ inp["Wg"].astype(np.float64).T + inp["bias"].astype(np.float64)
+        s = np.exp(l - l.max())
+        s /= s.sum()
+        order = np.argsort(-s, kind="stable")[:cfg.k]
+        g = s[order] / s[order].sum()
+        y = np.zeros(x_bits.shape[1])
+        for gi, e in zip(g, order):
+            o = _ffn_torch(x_bits[t:t + 1], inp["W1q"][e], inp["S1"][e], inp["W3q"][e], inp["S3"][e],
+                           inp["W2q"][e], inp["S2"][e]).numpy()[0]
+            o_bf16 = oracle.bf16_bits_to_f32(oracle.f64_to_bf16_bits(o)).astype(np.float64)
+            y += gi * o_bf16
+        out[t] = (order, y)
+    return out
+
+
+def test_brute_force_y_formula_tiny():
+    cfg = MoeConfig("bf", T=8, H=256, E=8, I=128, k=2, bias="uniform", seed=9)
+    inp = oracle.moe_inputs_to_numpy(make_inputs(cfg))
+    res = oracle.forward(cfg, inp)
+    brute = _brute_layer(cfg, inp, range(cfg.T))
+    for t, (order, y) in brute.items():
+        assert res["topk_idx"][t].tolist() == order.tolist()
+        _close_bf16(res["y"][t:t + 1], y[None], frac_equal=0.99)
+
+
+def test_sampled_forward_equals_full_forward():
+    cfg = MoeConfig("s", T=200, H=256, E=8, I=128, k=2, bias="zipf", cap_num=5, cap_den=4, seed=4)
+    inp = oracle.moe_inputs_to_numpy(make_inputs(cfg))
+    full = oracle.forward(cfg, inp)
+    toks = np.array([0, 7, 150, 199])
+    part = oracle.forward(cfg, inp, tokens=toks)
+    assert np.array_equal(part["y"][toks], full["y"][toks])
+    assert np.array_equal(part["slot_row"], full["slot_row"])
+    assert np.count_nonzero(full["slot_row"] < 0) > 0          # capacity dropped some slots
+
+
+def test_all_dropped_token_gives_zero():
+    cfg = MoeConfig("z", T=300, H=128, E=2, I=128, k=1, bias="zero", cap_num=1, cap_den=2, seed=1)
+    inp = oracle.moe_inputs_to_numpy(make_inputs(cfg))
+    out = oracle.forward(cfg, inp)
+    dropped = np.nonzero(out["slot_row"] < 0)[0]
+    assert len(dropped) > 0
+    assert np.all(out["y"][dropped] == 0)
