@@ -1,0 +1,423 @@
+"""Benchmark of the FP8 MoE expert layer on B200: tokens/s of moe_forward,
+grouped-GEMM TFLOPS and the dominant kernel's roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config page] [--impl ours|reference]
+
+A step is one moe_forward (route -> permute -> up GEMM + SwiGLU/requant ->
+down GEMM -> combine) over one batch of synthetic tokens with inputs resident
+in HBM. With N > 1 (one process per GPU under torch.distributed) every rank runs
+an independent replica of the layer on its own batch: the layer has no
+cross-GPU exchange on one GPU's path, so there is no data-path collective and
+scaling is weak. Rank 0 prints one JSON line.
+
+`--impl reference` times the CPU oracle (the plain C implementation the
+parity tests check against) on the host cores, on bounded samples of the same
+workload, and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from fp8_grouped_gemm_fp32_b200.inputs import CONFIGS, MoeConfig, interleave_w13, make_inputs  # noqa: E402
+
+METRIC = "MoE layer tokens/s; grouped FP8 GEMM TFLOPS and % of B200 roofline"
+FP8_PER_BF16 = 2.0          # nominal dense FP8 : BF16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def describe(cfg: MoeConfig) -> str:
+    s = (f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} I={cfg.I} "
+         f"{'hash k=1' if cfg.routing == 'hash' else f'top-{cfg.k} softmax'} {cfg.layout} layout")
+    if cfg.cap_num:
+        s += f" capacity ceil(T*k/E)*{cfg.cap_num}/{cfg.cap_den}"
+    return s + f" bias={cfg.bias} seed={cfg.seed}"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls NVML (SM clock, max clock, throttle reasons) on a thread while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.ok = False
+        self.samples = []
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": [],
+                    "samples": 0}
+        mhz = [s for s, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        names = sorted({n for b, n in self.REASONS.items() if bits & b})
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": float(self.max_mhz), "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ algorithmic work
+def algorithmic_work(cfg: MoeConfig, kept: np.ndarray):
+    """Minimum bytes each step must move and the FLOPs it must do (unpadded rows)."""
+    T, H, E, I, k = cfg.T, cfg.H, cfg.E, cfg.I, cfg.k
+    Rk = int(kept.sum())
+    touched = int(np.count_nonzero(kept))
+    G = lambda n: n // 128
+    w13 = touched * (2 * I * H + 4 * G(2 * I) * G(H))
+    w2 = touched * (H * I + 4 * G(H) * G(I))
+    work = {
+        "router": dict(bytes=(T * H * 2 + E * H * 4 + T * k * 8) if cfg.routing != "hash" else T * 4 + T * k * 8,
+                       flops=2.0 * T * E * H if cfg.routing != "hash" else 0.0),
+        "permute": dict(bytes=T * H * 2 + Rk * (H + 4 * G(H)) + 12 * T * k, flops=0.0),
+        "gemm_up": dict(bytes=w13 + Rk * (H + 4 * G(H)) + Rk * (I + 4 * G(I)), flops=2.0 * Rk * 2 * I * H),
+        "gemm_down": dict(bytes=w2 + Rk * (I + 4 * G(I)) + Rk * H * 2, flops=2.0 * Rk * H * I),
+        "combine": dict(bytes=Rk * H * 2 + T * H * 2 + T * k * 8, flops=0.0),
+    }
+    return work, Rk, touched
+
+
+# ------------------------------------------------------------------ our arm
+class Layer:
+    """Device buffers + the C-ABI calls of one replica of the layer."""
+
+    def __init__(self, cfg: MoeConfig, dev, seed_offset: int = 0):
+        from fp8_grouped_gemm_fp32_b200 import api
+        self.api = api
+        self.cfg = cfg
+        self.inp = make_inputs(cfg.replace(seed=cfg.seed + seed_offset), device=dev)
+        self.W13, self.S13 = interleave_w13(self.inp.W1q, self.inp.S1, self.inp.W3q, self.inp.S3)
+        self.c = api.Config.from_moe(cfg)
+        T, k, H, E, I = cfg.T, cfg.k, cfg.H, cfg.E, cfg.I
+        z = lambda *s, dt: torch.empty(*s, dtype=dt, device=dev)
+        self.y = z(T, H, dt=torch.bfloat16)
+        self.topk_idx = z(T, k, dt=torch.int32)
+        self.topk_w = z(T, k, dt=torch.float32)
+        self.counts = z(E, dt=torch.int32)
+        self.slot_row = z(T * k, dt=torch.int32)
+        self.ws = z(api.moe_workspace_size(self.c, True), dt=torch.uint8)
+        # step-wise buffers (per-kernel breakdown)
+        rows = api.moe_rows_capacity(self.c)
+        self.rows = rows
+        masked = cfg.layout == "masked"
+        self.M_rows = cfg.masked_max_m if masked else rows
+        self.Aq = z(rows, H, dt=torch.uint8)
+        self.As = z(rows * (H // 128), dt=torch.float32)
+        self.Hq = z(rows, I, dt=torch.uint8)
+        self.Hs = z(rows * (I // 128), dt=torch.float32)
+        self.O = z(rows, H, dt=torch.bfloat16)
+        self.kept = z(E, dt=torch.int32)
+        self.offsets = z(E + 1, dt=torch.int32)
+        self.row_src = z(rows, dt=torch.int32)
+        self.step_ws = z(api.moe_workspace_size(self.c, False), dt=torch.uint8)
+        self.launches_per_step = (1 if cfg.routing == "hash" else 2) + 3 + 2 + 1
+
+    def forward(self, x=None, stream=None):
+        a = self.api
+        i = self.inp
+        a.moe_forward(self.c, i.x if x is None else x, i.Wg, i.bias, i.token_ids, self.W13, self.S13, i.W2q, i.S2,
+                      self.y, self.topk_idx, self.topk_w, self.counts, self.slot_row, self.ws, stream)
+
+    def steps(self, ev):
+        """The same five steps as separate C-ABI calls, with an event after each."""
+        a, i, cfg = self.api, self.inp, self.cfg
+        masked = cfg.layout == "masked"
+        group = self.kept if masked else self.offsets
+        ev[0].record()
+        a.moe_route(self.c, i.x, i.Wg, i.bias, i.token_ids, self.topk_idx, self.topk_w, self.step_ws)
+        ev[1].record()
+        a.moe_permute(self.c, i.x, self.topk_idx, self.Aq, self.As, self.counts, self.kept, self.offsets,
+                      self.row_src, self.slot_row, self.step_ws)
+        ev[2].record()
+        a.moe_grouped_gemm_fp8(int(masked), cfg.E, 2 * cfg.I, cfg.H, self.Aq, self.As, group,
+                               self.M_rows, self.W13, self.S13, a.EPI_SWIGLU_FP8, self.Hq, self.Hs)
+        ev[3].record()
+        a.moe_grouped_gemm_fp8(int(masked), cfg.E, cfg.H, cfg.I, self.Hq, self.Hs, group, self.M_rows,
+                               i.W2q, i.S2, a.EPI_BF16, self.O)
+        ev[4].record()
+        a.moe_combine(self.c, self.O, self.slot_row, self.topk_w, self.y)
+        ev[5].record()
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif n_gpus > 1:
+        raise SystemExit("--gpus N > 1 runs under torch.distributed.run (one process per GPU)")
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(cfg: MoeConfig, target_s: float = 12.0):
+    """The oracle, as it stands, on a bounded sample of the workload's tokens."""
+    import oracle
+    threads = oracle.default_threads()
+    full = make_inputs(cfg, device="cpu", T=min(cfg.T, 256))
+    npi = oracle.moe_inputs_to_numpy(full)
+
+    def run(n):
+        sub = dict(npi)
+        sub["x"] = npi["x"][:n]
+        sub["token_ids"] = npi["token_ids"][:n]
+        c = cfg.replace(T=n, masked_max_m=(-(-n // 32) * 32 if cfg.layout == "masked" else cfg.masked_max_m))
+        t0 = time.perf_counter()
+        oracle.forward(c, sub, nthreads=threads)
+        return time.perf_counter() - t0
+
+    n = 2
+    dt = run(n)
+    n = int(max(1, min(full.cfg.T, math.floor(n * target_s / max(dt, 1e-3)))))
+    dt = run(n)
+    return {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {n} tokens of the {cfg.name} workload as one batch (routing, permutation, "
+                      f"expert math in fp64, combine), {dt:.1f} s"}
+
+
+def run_ours(args):
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = CONFIGS[args.config]
+    from fp8_grouped_gemm_fp32_b200 import api
+    api.lib()                                      # fails loudly if the native library is missing
+    layer = Layer(cfg, dev, seed_offset=rank)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        layer.forward()
+    torch.cuda.synchronize()
+    assert api.moe_get_device_status() == api.MOE_OK
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        start.record()
+        for _ in range(args.steps):
+            layer.forward()
+        end.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = start.elapsed_time(end) / args.steps
+    ms_max = max_over_ranks(ms, world)
+    st = api.moe_get_device_status()
+    assert st == api.MOE_OK, api.STATUS_NAMES.get(st)
+    value = world * cfg.T / (ms_max / 1e3)
+
+    # end to end through the public call with host buffers: H2D of x (and token ids), forward, D2H of y
+    x_host = layer.inp.x.cpu().pin_memory()
+    tid_host = layer.inp.token_ids.cpu().pin_memory()
+    y_host = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
+    x_dev = torch.empty_like(layer.inp.x)
+    tid_dev = layer.inp.token_ids
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x=x_dev)
+        y_host.copy_(layer.y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    start.record()
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        if cfg.routing == "hash":
+            tid_dev.copy_(tid_host, non_blocking=True)
+        layer.forward(x=x_dev)
+        y_host.copy_(layer.y, non_blocking=True)
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(start.elapsed_time(end) / args.steps, world)
+    h2d = x_host.numel() * 2 + (tid_host.numel() * 4 if cfg.routing == "hash" else 0)
+    d2h = y_host.numel() * 2
+
+    # per-kernel breakdown through the step-wise calls (same kernels, one event between each)
+    names = ["router", "permute", "gemm_up", "gemm_down", "combine"]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for _ in range(2):
+        layer.steps([torch.cuda.Event(enable_timing=True) for _ in range(6)])
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        layer.steps(evs[i])
+    torch.cuda.synchronize()
+    per = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+           for j, n in enumerate(names)}
+    kept = layer.kept.cpu().numpy()
+    work, Rk, touched = algorithmic_work(cfg, kept)
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    fp8_sus = FP8_PER_BF16 * float(peaks["bf16_tflops_sustained"])
+    fp8_burst = FP8_PER_BF16 * float(peaks["bf16_tflops"])
+    dom = max(per, key=per.get)
+    w = work[dom]
+    t_s = per[dom] / 1e3
+    t_tensor = w["flops"] / (fp8_sus * 1e12) if dom.startswith("gemm") else 0.0
+    t_hbm = w["bytes"] / (hbm * 1e9)
+    if dom.startswith("gemm") and t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": w["flops"] / t_s / 1e12, "peak": fp8_sus, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": w["bytes"] / t_s / 1e9, "peak": hbm, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["traffic"] = None
+    roof["peak_source"] = (f"{peak_src}: " + ("FP8 = 2 x sustained bf16 cuBLAS (nominal FP8:BF16 ratio)"
+                                              if roof["bound"] == "tensor" else "HBM copy"))
+    gemm_ms = per["gemm_up"] + per["gemm_down"]
+    gemm_flops = work["gemm_up"]["flops"] + work["gemm_down"]["flops"]
+    gemm_tflops = gemm_flops / (gemm_ms / 1e3) / 1e12
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8e4m3 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": describe(cfg), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "no flush: the FP8 weights streamed every step (%.2f GB) exceed the 126 MB L2"
+                         % ((work["gemm_up"]["bytes"] + work["gemm_down"]["bytes"]) / 1e9)},
+        "roofline": roof,
+        "gemm": {"tflops": gemm_tflops, "frac_fp8_sustained": gemm_tflops / fp8_sus,
+                 "frac_fp8_nominal_4500": gemm_tflops / 4500.0, "ms": gemm_ms, "rows_kept": Rk,
+                 "experts_touched": touched},
+        "kernels_ms": per,
+        "e2e": {"value": world * cfg.T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": layer.launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+    cfg = CONFIGS[args.config]
+    threads = oracle.default_threads()
+    inp = oracle.moe_inputs_to_numpy(make_inputs(cfg, device="cpu", T=min(cfg.T, 256)))
+
+    def step(n):
+        sub = dict(inp)
+        sub["x"] = inp["x"][:n]
+        sub["token_ids"] = inp["token_ids"][:n]
+        c = cfg.replace(T=n, masked_max_m=(-(-n // 32) * 32 if cfg.layout == "masked" else cfg.masked_max_m))
+        t0 = time.perf_counter()
+        oracle.forward(c, sub, nthreads=threads)
+        return time.perf_counter() - t0
+
+    budget = 150.0 / max(1, args.steps + args.warmup)        # whole run within a few minutes
+    dt = step(2)
+    n = int(max(1, min(256, math.floor(2 * min(budget, 10.0) / max(dt, 1e-3)))))
+    for _ in range(args.warmup):
+        step(n)
+    times = [step(n) for _ in range(args.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    value = n / (ms / 1e3)
+    sample = f"first {n} tokens of the {cfg.name} workload per step as one batch"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp64 (oracle)", "data": "synthetic",
+            "config": {"workload": describe(cfg), "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": threads,
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="page", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+"""Thin ctypes binding of include/moe_fp8.h with the same entry-point names.
+
+Argument marshalling only: every step runs in libmoe_fp8.so's kernels. Tensors
+are torch CUDA tensors (torch provides device memory and streams); their data
+pointers are passed straight through. A missing library raises at import of
+the first call; there is no fallback path."""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from .build import LIB
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED_SHAPE = 2
+MOE_ERR_UNSUPPORTED_DEVICE = 3
+MOE_ERR_WORKSPACE_TOO_SMALL = 4
+MOE_ERR_CAPACITY = 5
+MOE_ERR_CUDA = 6
+MOE_ERR_DEVICE_TIMEOUT = 7
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
+                3: "MOE_ERR_UNSUPPORTED_DEVICE", 4: "MOE_ERR_WORKSPACE_TOO_SMALL", 5: "MOE_ERR_CAPACITY",
+                6: "MOE_ERR_CUDA", 7: "MOE_ERR_DEVICE_TIMEOUT"}
+ROUTE_SOFTMAX_TOPK, ROUTE_HASH = 0, 1
+LAYOUT_CONTIGUOUS, LAYOUT_MASKED = 0, 1
+EPI_BF16, EPI_SWIGLU_FP8 = 0, 1
+EXPORTS = ("moe_rows_capacity", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_gemm_fp8",
+           "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("T", "H", "E", "I", "k", "routing", "cap_num", "cap_den",
+                                            "layout", "masked_max_m")]
+
+    @classmethod
+    def from_moe(cls, cfg) -> "Config":
+        """From an inputs.MoeConfig."""
+        return cls(cfg.T, cfg.H, cfg.E, cfg.I, cfg.k,
+                   ROUTE_HASH if cfg.routing == "hash" else ROUTE_SOFTMAX_TOPK,
+                   cfg.cap_num, cfg.cap_den,
+                   LAYOUT_MASKED if cfg.layout == "masked" else LAYOUT_CONTIGUOUS,
+                   cfg.masked_max_m)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise RuntimeError(f"native library {LIB} is missing: run fp8_grouped_gemm_fp32_b200.build.build()")
+        L = ctypes.CDLL(LIB)
+        P, I, SZ, CP = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.POINTER(Config)
+        L.moe_rows_capacity.argtypes = [CP]
+        L.moe_rows_capacity.restype = SZ
+        L.moe_workspace_size.argtypes = [CP, I]
+        L.moe_workspace_size.restype = SZ
+        L.moe_route.argtypes = [CP, P, P, P, P, P, P, P, SZ, P]
+        L.moe_permute.argtypes = [CP, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_grouped_gemm_fp8.argtypes = [I, I, I, I, P, P, P, I, P, P, I, P, P, P]
+        L.moe_combine.argtypes = [CP, P, P, P, P, P]
+        L.moe_forward.argtypes = [CP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_get_device_status.argtypes = [P]
+        L.moe_selftest_wait_timeout.argtypes = [I, P]
+        L.moe_status_string.argtypes = [I]
+        L.moe_status_string.restype = ctypes.c_char_p
+        for f in EXPORTS:
+            if f not in ("moe_rows_capacity", "moe_workspace_size", "moe_status_string"):
+                getattr(L, f).restype = I
+        _lib = L
+    return _lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        return ctypes.c_void_p(int(t))
+    if t.numel() and not t.is_cuda:
+        raise ValueError("moe_fp8 entry points take CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("moe_fp8 entry points take contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr()) if t.numel() else None
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(st: int, call: str):
+    if st != MOE_OK:
+        raise MoeError(st, call)
+
+
+def status_string(st: int) -> str:
+    return lib().moe_status_string(st).decode()
+
+
+def moe_rows_capacity(cfg: Config) -> int:
+    return int(lib().moe_rows_capacity(ctypes.byref(cfg)))
+
+
+def moe_workspace_size(cfg: Config, for_forward: bool = False) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(cfg), int(for_forward)))
+
+
+def moe_route(cfg, x, Wg, bias, token_ids, topk_idx, topk_w, ws, stream=None):
+    _check(lib().moe_route(ctypes.byref(cfg), _p(x), _p(Wg), _p(bias), _p(token_ids), _p(topk_idx), _p(topk_w),
+                           _p(ws), ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)),
+           "moe_route")
+
+
+def moe_permute(cfg, x, topk_idx, Aq, As, counts, kept, offsets, row_src, slot_row, ws, stream=None):
+    _check(lib().moe_permute(ctypes.byref(cfg), _p(x), _p(topk_idx), _p(Aq), _p(As), _p(counts), _p(kept),
+                             _p(offsets), _p(row_src), _p(slot_row), _p(ws), ws.numel() * ws.element_size(),
+                             _stream(stream)), "moe_permute")
+
+
+def moe_grouped_gemm_fp8(layout, E, N, K, A, As, group_info, M_rows, B, Bs, epilogue, D, Ds=None, stream=None):
+    _check(lib().moe_grouped_gemm_fp8(layout, E, N, K, _p(A), _p(As), _p(group_info), M_rows, _p(B), _p(Bs),
+                                      epilogue, _p(D), _p(Ds), _stream(stream)), "moe_grouped_gemm_fp8")
+
+
+def moe_combine(cfg, O, slot_row, topk_w, y, stream=None):
+    _check(lib().moe_combine(ctypes.byref(cfg), _p(O), _p(slot_row), _p(topk_w), _p(y), _stream(stream)),
+           "moe_combine")
+
+
+def moe_forward(cfg, x, Wg, bias, token_ids, W13, S13, W2, S2, y, topk_idx, topk_w, counts, slot_row, ws,
+                stream=None):
+    _check(lib().moe_forward(ctypes.byref(cfg), _p(x), _p(Wg), _p(bias), _p(token_ids), _p(W13), _p(S13), _p(W2),
+                             _p(S2), _p(y), _p(topk_idx), _p(topk_w), _p(counts), _p(slot_row), _p(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+
+
+def moe_get_device_status(stream=None) -> int:
+    return int(lib().moe_get_device_status(_stream(stream)))
+
+
+def moe_selftest_wait_timeout(limit_us: int, stream=None):
+    _check(lib().moe_selftest_wait_timeout(limit_us, _stream(stream)), "moe_selftest_wait_timeout")

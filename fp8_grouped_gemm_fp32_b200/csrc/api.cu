@@ -1,0 +1,317 @@
+// The C ABI (include/moe_fp8.h): argument validation on the host, workspace
+// carving, the per-device status word and the launch sequence of moe_forward.
+// Nothing here allocates device memory or synchronises the host, except
+// moe_get_device_status, whose job is to synchronise and read the status.
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "../../include/moe_fp8.h"
+#include "common.cuh"
+
+namespace moe {
+cudaError_t launch_router_softmax(const uint16_t* x, const float* Wg, const float* bias, float* logits, int T, int H,
+                                  int E, int k, int32_t* topk_idx, float* topk_w, int num_sms, cudaStream_t s);
+cudaError_t launch_router_hash(const int32_t* token_ids, int T, int E, int32_t* topk_idx, float* topk_w,
+                               cudaStream_t s);
+size_t permute_scratch_bytes(int T, int E);
+cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, int T, int H, int k, int E, int64_t cap,
+                           int masked_max_m, int ld_rows, uint8_t* Aq, float* As, int32_t* counts, int32_t* kept,
+                           int32_t* offsets, int32_t* row_src, int32_t* slot_row, void* scratch, int* status,
+                           int num_sms, cudaStream_t s);
+cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                                const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs, int epilogue,
+                                void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s);
+cudaError_t launch_combine(const uint16_t* O, const int32_t* slot_row, const float* topk_w, int T, int k, int H,
+                           uint16_t* y, cudaStream_t s);
+cudaError_t launch_selftest_wait(int* status, uint64_t wait_ns, cudaStream_t s);
+
+// The device status word (one per device that loads the library).
+__device__ int g_status;
+
+namespace {
+
+constexpr uint64_t kWaitNs = 4000000000ull;   // a legitimate wait never comes near 4 s
+constexpr size_t kAlign = 256;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool supported = false;
+    int num_sms = 0;
+    int* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+moe_status_t device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_CUDA;
+        d.supported = prop.major == 10 && prop.minor == 0;
+        d.num_sms = prop.multiProcessorCount;
+        if (d.supported) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return MOE_ERR_CUDA;
+            d.status = static_cast<int*>(p);
+        }
+        d.ready = true;
+    }
+    if (!d.supported) return MOE_ERR_UNSUPPORTED_DEVICE;
+    *out = &d;
+    return MOE_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+moe_status_t check_cfg(const moe_config_t* c) {
+    if (!c) return MOE_ERR_INVALID_ARG;
+    if (c->T < 0 || c->H <= 0 || c->I <= 0 || c->E <= 0 || c->k <= 0) return MOE_ERR_INVALID_ARG;
+    if (c->H % kGroup || c->I % kGroup || c->H > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->E > MOE_MAX_EXPERTS || c->k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->k > c->E) return MOE_ERR_INVALID_ARG;
+    if (c->routing != MOE_ROUTE_SOFTMAX_TOPK && c->routing != MOE_ROUTE_HASH) return MOE_ERR_INVALID_ARG;
+    if (c->routing == MOE_ROUTE_HASH && c->k != 1) return MOE_ERR_INVALID_ARG;
+    if (c->cap_num < 0 || c->cap_den < 0 || ((c->cap_num == 0) != (c->cap_den == 0))) return MOE_ERR_INVALID_ARG;
+    if (c->layout != MOE_LAYOUT_CONTIGUOUS && c->layout != MOE_LAYOUT_MASKED) return MOE_ERR_INVALID_ARG;
+    if (c->layout == MOE_LAYOUT_MASKED && (c->masked_max_m <= 0 || c->masked_max_m % 32)) return MOE_ERR_INVALID_ARG;
+    const int64_t rows = c->layout == MOE_LAYOUT_MASKED
+                             ? static_cast<int64_t>(c->E) * c->masked_max_m
+                             : static_cast<int64_t>(c->T) * c->k + static_cast<int64_t>(c->E) * (kGroup - 1);
+    if (rows >= (1ll << 31) / kGroup) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+int64_t capacity_of(const moe_config_t* c) {
+    if (c->cap_num == 0) return -1;
+    const int64_t R = static_cast<int64_t>(c->T) * c->k;
+    return (R + c->E - 1) / c->E * c->cap_num / c->cap_den;
+}
+
+size_t rows_of(const moe_config_t* c) {
+    if (c->layout == MOE_LAYOUT_MASKED) return static_cast<size_t>(c->E) * c->masked_max_m;
+    const size_t r = static_cast<size_t>(c->T) * c->k + static_cast<size_t>(c->E) * (kGroup - 1);
+    return (r + kGroup - 1) / kGroup * kGroup;
+}
+
+size_t route_scratch(const moe_config_t* c) {
+    return c->routing == MOE_ROUTE_SOFTMAX_TOPK ? align_up(sizeof(float) * static_cast<size_t>(c->T) * c->E) : 0;
+}
+
+// moe_forward's scratch, in carving order
+struct FwdWs {
+    uint8_t* Aq;
+    float* As;
+    uint8_t* Hq;
+    float* Hs;
+    uint16_t* O;
+    int32_t* kept;
+    int32_t* offsets;
+    int32_t* row_src;
+    void* step;   // route / permute scratch
+    size_t total;
+};
+
+FwdWs carve(const moe_config_t* c, void* base) {
+    FwdWs w;
+    const size_t rows = rows_of(c);
+    uint8_t* p = static_cast<uint8_t*>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* q = p ? p + off : nullptr;
+        off += align_up(bytes);
+        return q;
+    };
+    w.Aq = take(rows * c->H);
+    w.As = reinterpret_cast<float*>(take(sizeof(float) * rows * (c->H / kGroup)));
+    w.Hq = take(rows * c->I);
+    w.Hs = reinterpret_cast<float*>(take(sizeof(float) * rows * (c->I / kGroup)));
+    w.O = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * rows * c->H));
+    w.kept = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * c->E));
+    w.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (c->E + 1)));
+    w.row_src = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * rows));
+    w.step = take(std::max(route_scratch(c), align_up(moe::permute_scratch_bytes(c->T, c->E))));
+    w.total = off;
+    return w;
+}
+
+inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_rows_capacity(const moe_config_t* cfg) {
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    return rows_of(cfg);
+}
+
+size_t moe_workspace_size(const moe_config_t* cfg, int for_forward) {
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    if (for_forward) return carve(cfg, nullptr).total;
+    return std::max(route_scratch(cfg), align_up(permute_scratch_bytes(cfg->T, cfg->E)));
+}
+
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* Wg, const float* bias,
+                       const int32_t* token_ids, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                       void* stream) {
+    moe_status_t st = check_cfg(cfg);
+    if (st != MOE_OK) return st;
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    if (!ptr_ok(topk_idx) || !ptr_ok(topk_w)) return MOE_ERR_INVALID_ARG;
+    if (cfg->routing == MOE_ROUTE_HASH) {
+        if (!ptr_ok(token_ids)) return MOE_ERR_INVALID_ARG;
+    } else {
+        if (!ptr_ok(x) || !ptr_ok(Wg) || (bias && !aligned16(bias)) || !ptr_ok(ws)) return MOE_ERR_INVALID_ARG;
+        if (ws_bytes < route_scratch(cfg)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    }
+    if (cfg->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cfg->routing == MOE_ROUTE_HASH)
+        return cuda_status(launch_router_hash(token_ids, cfg->T, cfg->E, topk_idx, topk_w, s));
+    return cuda_status(launch_router_softmax(static_cast<const uint16_t*>(x), Wg, bias, static_cast<float*>(ws),
+                                             cfg->T, cfg->H, cfg->E, cfg->k, topk_idx, topk_w, dev->num_sms, s));
+}
+
+moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, uint8_t* Aq, float* As,
+                         int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_src, int32_t* slot_row,
+                         void* ws, size_t ws_bytes, void* stream) {
+    moe_status_t st = check_cfg(cfg);
+    if (st != MOE_OK) return st;
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    if (!ptr_ok(x) || !ptr_ok(topk_idx) || !ptr_ok(Aq) || !ptr_ok(As) || !ptr_ok(counts) || !ptr_ok(kept) ||
+        !ptr_ok(offsets) || !ptr_ok(row_src) || !ptr_ok(slot_row) || !ptr_ok(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < permute_scratch_bytes(cfg->T, cfg->E)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (cfg->T == 0) return MOE_OK;
+    const bool masked = cfg->layout == MOE_LAYOUT_MASKED;
+    return cuda_status(launch_permute(static_cast<const uint16_t*>(x), topk_idx, cfg->T, cfg->H, cfg->k, cfg->E,
+                                      capacity_of(cfg), masked ? cfg->masked_max_m : 0,
+                                      static_cast<int>(rows_of(cfg)), Aq, As, counts, kept, offsets, row_src,
+                                      slot_row, ws, dev->status, dev->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_gemm_fp8(int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                                  const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
+                                  int epilogue, void* D, float* Ds, void* stream) {
+    if (layout != MOE_LAYOUT_CONTIGUOUS && layout != MOE_LAYOUT_MASKED) return MOE_ERR_INVALID_ARG;
+    if (epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_SWIGLU_FP8) return MOE_ERR_INVALID_ARG;
+    if (E <= 0 || N <= 0 || K <= 0 || M_rows <= 0) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS || N % kGroup || K % kGroup) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (epilogue == MOE_EPI_SWIGLU_FP8 && N % (2 * kGroup)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (layout == MOE_LAYOUT_MASKED && M_rows % 32) return MOE_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(E) * N >= (1ll << 31) || static_cast<int64_t>(E) * M_rows >= (1ll << 31))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!ptr_ok(A) || !ptr_ok(As) || !ptr_ok(group_info) || !ptr_ok(B) || !ptr_ok(Bs) || !ptr_ok(D))
+        return MOE_ERR_INVALID_ARG;
+    if (epilogue == MOE_EPI_SWIGLU_FP8 && !ptr_ok(Ds)) return MOE_ERR_INVALID_ARG;
+    moe_status_t st;
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    return cuda_status(launch_grouped_gemm(layout, E, N, K, A, As, group_info, M_rows, B, Bs, epilogue, D, Ds,
+                                           dev->status, kWaitNs, dev->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const void* O, const int32_t* slot_row, const float* topk_w,
+                         void* y, void* stream) {
+    moe_status_t st = check_cfg(cfg);
+    if (st != MOE_OK) return st;
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    if (!ptr_ok(O) || !ptr_ok(slot_row) || !ptr_ok(topk_w) || !ptr_ok(y)) return MOE_ERR_INVALID_ARG;
+    if (cfg->T == 0) return MOE_OK;
+    return cuda_status(launch_combine(static_cast<const uint16_t*>(O), slot_row, topk_w, cfg->T, cfg->k, cfg->H,
+                                      static_cast<uint16_t*>(y), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg, const float* bias,
+                         const int32_t* token_ids, const uint8_t* W13, const float* S13, const uint8_t* W2,
+                         const float* S2, void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                         int32_t* slot_row, void* ws, size_t ws_bytes, void* stream) {
+    moe_status_t st = check_cfg(cfg);
+    if (st != MOE_OK) return st;
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    if (!ptr_ok(x) || !ptr_ok(W13) || !ptr_ok(S13) || !ptr_ok(W2) || !ptr_ok(S2) || !ptr_ok(y) || !ptr_ok(topk_idx) ||
+        !ptr_ok(topk_w) || !ptr_ok(counts) || !ptr_ok(slot_row) || !ptr_ok(ws) || (ws && (reinterpret_cast<uintptr_t>(ws) % kAlign)))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->routing == MOE_ROUTE_SOFTMAX_TOPK && (!ptr_ok(Wg) || (bias && !aligned16(bias))))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->routing == MOE_ROUTE_HASH && !ptr_ok(token_ids)) return MOE_ERR_INVALID_ARG;
+    const FwdWs w = carve(cfg, ws);
+    if (ws_bytes < w.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (cfg->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool masked = cfg->layout == MOE_LAYOUT_MASKED;
+    const int rows = static_cast<int>(rows_of(cfg));
+    const int M_rows = masked ? cfg->masked_max_m : rows;
+    const int32_t* group = masked ? w.kept : w.offsets;
+    cudaError_t e;
+    if (cfg->routing == MOE_ROUTE_HASH)
+        e = launch_router_hash(token_ids, cfg->T, cfg->E, topk_idx, topk_w, s);
+    else
+        e = launch_router_softmax(static_cast<const uint16_t*>(x), Wg, bias, static_cast<float*>(w.step), cfg->T,
+                                  cfg->H, cfg->E, cfg->k, topk_idx, topk_w, dev->num_sms, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_permute(static_cast<const uint16_t*>(x), topk_idx, cfg->T, cfg->H, cfg->k, cfg->E, capacity_of(cfg),
+                       masked ? cfg->masked_max_m : 0, rows, w.Aq, w.As, counts, w.kept, w.offsets, w.row_src,
+                       slot_row, w.step, dev->status, dev->num_sms, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_grouped_gemm(cfg->layout, cfg->E, 2 * cfg->I, cfg->H, w.Aq, w.As, group, M_rows, W13, S13,
+                            MOE_EPI_SWIGLU_FP8, w.Hq, w.Hs, dev->status, kWaitNs, dev->num_sms, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_grouped_gemm(cfg->layout, cfg->E, cfg->H, cfg->I, w.Hq, w.Hs, group, M_rows, W2, S2, MOE_EPI_BF16,
+                            w.O, nullptr, dev->status, kWaitNs, dev->num_sms, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_combine(w.O, slot_row, topk_w, cfg->T, cfg->k, cfg->H, static_cast<uint16_t*>(y), s);
+    return cuda_status(e);
+}
+
+moe_status_t moe_get_device_status(void* stream) {
+    moe_status_t st;
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpy(&v, dev->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpy(dev->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    return static_cast<moe_status_t>(v);
+}
+
+moe_status_t moe_selftest_wait_timeout(int limit_us, void* stream) {
+    if (limit_us < 0) return MOE_ERR_INVALID_ARG;
+    moe_status_t st;
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    return cuda_status(launch_selftest_wait(dev->status, static_cast<uint64_t>(limit_us) * 1000ull,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+const char* moe_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case MOE_ERR_UNSUPPORTED_DEVICE: return "FP8 not supported on this GPU (needs sm_100)";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case MOE_ERR_CAPACITY: return "a masked group had more rows than masked_max_m";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,622 @@
+// FP8 grouped GEMM on the sm_100a tensor cores (tcgen05 + tensor memory).
+//
+// Problem (MegaMoE page, sections 2.1 and 3.2): one GEMM per expert group;
+// every group has its own M (tokens), all groups share N and K; A is the
+// groups' rows concatenated, B = [E, N, K] ("nt": both K-major). FP8 E4M3
+// operands with fine-grained fp32 scales: one per 1x128 activation group and
+// one per 128x128 weight block (DeepSeek open-source week page, "Day 3").
+// FP8 tensor-core partial sums are promoted to fp32 on the CUDA cores, where
+// the scales are applied (same page: two-level accumulation), and the fp32
+// accumulator is converted to bf16 with round-to-nearest-even only at the end
+// (MegaMoE page, 3.3). The up projection fuses SwiGLU and the 1x128 FP8
+// requantisation of h into its epilogue (3.2: epilogue fusion).
+//
+// Two kernels, both persistent (one CTA per SM) and warp-specialised:
+//
+// * contiguous layout (prefill): tiles of 128 rows x 256 columns over the
+//   flattened, 128-padded M of all groups (the pages' global tile scheduler,
+//   3.2). Warp 0 issues TMA loads into a 4-stage shared-memory ring; warp 1
+//   issues tcgen05.mma (kind::f8f6f4, M=128, N=256, K=32) for each 128-wide K
+//   block into one of two tensor-memory buffers; 8 promotion warps read each
+//   finished block with tcgen05.ld and fold it into fp32 register
+//   accumulators scaled by sa[row] * sw[block], then run the epilogue. Tiles
+//   are ordered expert -> N tile -> M tile, so the CTAs working at the same
+//   time share one weight tile through L2.
+// * masked layout (decode, few tokens per expert): swap-AB. The weight block
+//   is the MMA's M=128 operand and up to 32 tokens are its N, so weights
+//   stream from HBM in 16 KB (or 2 x 16 KB) stages while the token tile is
+//   tiny; experts with no tokens produce no tiles.
+//
+// Every wait on an mbarrier is bounded; a wait that runs out records
+// MOE_ERR_DEVICE_TIMEOUT, the CTA stops issuing work, lets copies and MMAs in
+// flight land, frees its tensor memory and returns.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kBM = 128, kBN = 256, kBK = 128;
+constexpr int kStagesC = 4;
+constexpr int kABytes = kBM * kBK;            // 16 KB
+constexpr int kBBytes = kBN * kBK;            // 32 KB
+constexpr int kThreadsC = 384;                // 12 warps
+constexpr int kDrainNs = 200000;              // settle time after an abort
+
+struct SmemC {
+    uint8_t a[kStagesC][kABytes];
+    uint8_t b[kStagesC][kBBytes];
+    uint64_t full[kStagesC];
+    uint64_t empty[kStagesC];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t red_bar[2];
+    float red[2][2][kBM];
+    uint32_t tmem_base;
+    volatile int abort_flag;
+    int32_t P[kMaxE + 1];
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Largest e in [0, E) with P[e] <= q (P non-decreasing, P[0] = 0 <= q).
+__device__ __forceinline__ int find_group(const int32_t* P, int E, int q) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P[mid] <= q) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+struct TileC {
+    int e, m0, n0, width;
+};
+
+__device__ __forceinline__ TileC decode_tile_c(const int32_t* P, int E, int NT, int N, int tile) {
+    TileC t;
+    const int q = tile / NT;
+    t.e = find_group(P, E, q);
+    const int mt_e = P[t.e + 1] - P[t.e];
+    const int local = tile - NT * P[t.e];
+    const int nt = local / mt_e;
+    t.m0 = (P[t.e] + local % mt_e) * kBM;
+    t.n0 = nt * kBN;
+    t.width = min(kBN, N - t.n0);
+    return t;
+}
+
+__device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreadsC, 1)
+gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const float* __restrict__ As, const int32_t* __restrict__ offsets, int M_rows,
+                 const float* __restrict__ Bs, int E, int N, int K, void* __restrict__ D, float* __restrict__ Ds,
+                 int* status, uint64_t wait_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    SmemC& sm = *reinterpret_cast<SmemC*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KB = K / kBK;
+    const int NB = N / kBM;                 // 128-wide weight blocks along N
+    const int NT = (N + kBN - 1) / kBN;
+
+    // group prefix in M tiles: P[e] = offsets[e] / 128
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) sm.P[e] = offsets[e] / kBM;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesC; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.tfull[b], 1);
+            mbar_init(&sm.tempty[b], 8);
+            mbar_init(&sm.red_bar[b], 256);
+        }
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const int MT = sm.P[E];
+    const int total = MT * NT;
+
+    auto fail = [&]() {
+        set_status(status, kStatusTimeout);
+        sm.abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ---------------- TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tmA);
+            prefetch_tensormap(&tmB);
+            uint32_t it = 0;
+            for (int tile = blockIdx.x; tile < total && !sm.abort_flag; tile += gridDim.x) {
+                const TileC t = decode_tile_c(sm.P, E, NT, N, tile);
+                const uint32_t bytes = kABytes + (t.width == kBN ? kBBytes : kBBytes / 2);
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = it % kStagesC;
+                    const uint32_t ph = (it / kStagesC) & 1;
+                    if (!mbar_wait(&sm.empty[s], ph ^ 1, wait_ns)) { fail(); break; }
+                    mbar_arrive_expect_tx(&sm.full[s], bytes);
+                    tma_load_2d(sm.a[s], &tmA, &sm.full[s], kb * kBK, t.m0);
+                    tma_load_2d(sm.b[s], &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0);
+                    if (t.width == kBN)
+                        tma_load_2d(sm.b[s] + kBBytes / 2, &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0 + 128);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, kbt = 0;
+            for (int tile = blockIdx.x; tile < total && !sm.abort_flag; tile += gridDim.x) {
+                const TileC t = decode_tile_c(sm.P, E, NT, N, tile);
+                const uint32_t idesc = f8_idesc(kBM, t.width);
+                for (int kb = 0; kb < KB; ++kb, ++it, ++kbt) {
+                    const int s = it % kStagesC;
+                    const uint32_t ph = (it / kStagesC) & 1;
+                    const int buf = kbt & 1;
+                    const uint32_t bph = (kbt >> 1) & 1;
+                    if (!mbar_wait(&sm.full[s], ph, wait_ns)) { fail(); break; }
+                    if (!mbar_wait(&sm.tempty[buf], bph ^ 1, wait_ns)) { fail(); break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+                    const uint32_t d = tmem + buf * kBN;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 32; ++kk)
+                        umma_f8(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc, kk > 0);
+                    umma_commit(&sm.empty[s]);
+                    umma_commit(&sm.tfull[buf]);
+                }
+            }
+        }
+    } else if (warp >= 4) {
+        // ---------------- promotion + epilogue (256 threads)
+        const int q = warp & 3;                 // tensor-memory lane quadrant
+        const int half = (warp - 4) >> 2;       // which 64 columns of each 128-column half
+        const int row = q * 32 + lane;          // row within the tile
+        uint32_t kbt = 0, ep = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            if (sm.abort_flag) break;
+            const TileC t = decode_tile_c(sm.P, E, NT, N, tile);
+            const bool full = t.width == kBN;
+            float acc[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            const float* bs0 = Bs + (static_cast<int64_t>(t.e) * NB + t.n0 / kBM) * KB;
+            const float* bs1 = bs0 + KB;
+            const float* as_row = As + t.m0 + row;
+            bool ok = true;
+            for (int kb = 0; kb < KB; ++kb, ++kbt) {
+                const int buf = kbt & 1;
+                const uint32_t bph = (kbt >> 1) & 1;
+                const float sa = as_row[static_cast<int64_t>(kb) * M_rows];
+                const float f0 = sa * bs0[kb];
+                const float f1 = full ? sa * bs1[kb] : 0.0f;
+                if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
+                tc_fence_after();
+                const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kBN + half * 64;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    float v[32];
+                    tmem_ld32(taddr + c * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(v[i], f0, acc[c * 32 + i]);
+                }
+                if (full) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        float v[32];
+                        tmem_ld32(taddr + 128 + c * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) acc[64 + c * 32 + i] = fmaf(v[i], f1, acc[64 + c * 32 + i]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+            }
+            if (!ok) break;
+            const int64_t grow = t.m0 + row;
+            if constexpr (EPI == 0) {
+                uint16_t* out = static_cast<uint16_t*>(D) + grow * N + t.n0 + half * 64;
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    if (r == 1 && !full) break;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        uint32_t u[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const __nv_bfloat162 b =
+                                __floats2bfloat162_rn(acc[r * 64 + v * 8 + 2 * i], acc[r * 64 + v * 8 + 2 * i + 1]);
+                            u[i] = *reinterpret_cast<const uint32_t*>(&b);
+                        }
+                        *reinterpret_cast<uint4*>(out + r * 128 + v * 8) = make_uint4(u[0], u[1], u[2], u[3]);
+                    }
+                }
+            } else {
+                // SwiGLU on (a = acc[0..63], b = acc[64..127]) for h columns n0/2 + half*64 + [0, 64)
+                const int I = N / 2;
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    acc[i] = silu_f(acc[i]) * acc[64 + i];
+                    amax = fmaxf(amax, fabsf(acc[i]));
+                }
+                const int p = ep & 1;
+                sm.red[p][half][row] = amax;
+                mbar_arrive(&sm.red_bar[p]);
+                if (!mbar_wait(&sm.red_bar[p], (ep >> 1) & 1, wait_ns)) { fail(); break; }
+                ++ep;
+                amax = fmaxf(sm.red[p][0][row], sm.red[p][1][row]);
+                const float s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+                uint8_t* hq = static_cast<uint8_t*>(D) + grow * I + t.n0 / 2 + half * 64;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint32_t u[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = v * 16 + i * 4;
+                        const float d0 = amax == 0.0f ? acc[c] : __fdiv_rn(acc[c], s);
+                        const float d1 = amax == 0.0f ? acc[c + 1] : __fdiv_rn(acc[c + 1], s);
+                        const float d2 = amax == 0.0f ? acc[c + 2] : __fdiv_rn(acc[c + 2], s);
+                        const float d3 = amax == 0.0f ? acc[c + 3] : __fdiv_rn(acc[c + 3], s);
+                        u[i] = f32x2_to_e4m3x2(d0, d1) | (static_cast<uint32_t>(f32x2_to_e4m3x2(d2, d3)) << 16);
+                    }
+                    *reinterpret_cast<uint4*>(hq + v * 16) = make_uint4(u[0], u[1], u[2], u[3]);
+                }
+                if (half == 0) Ds[static_cast<int64_t>(t.n0 / kBN) * M_rows + grow] = s;
+            }
+        }
+    }
+
+    __syncthreads();
+    if (sm.abort_flag) {
+        // let TMA copies and MMAs that were already issued land before the memory is released
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < kDrainNs) __nanosleep(1000);
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ====================================================================== masked layout, swap-AB
+constexpr int kBT = 32;                       // tokens per tile (the MMA's N)
+constexpr int kXBytes = kBT * kBK;            // 4 KB
+constexpr int kWBlk = kBM * kBK;              // 16 KB: 128 weight rows x 128 K bytes
+constexpr int kThreadsM = 192;                // 6 warps
+
+template <int EPI>
+struct SmemM {
+    static constexpr int kW = EPI == 1 ? 2 * kWBlk : kWBlk;    // weight rows per stage: 256 (a|b) or 128
+    static constexpr int kStages = EPI == 1 ? 4 : 8;
+    static constexpr int kCols = EPI == 1 ? 2 * kBT : kBT;     // tensor-memory columns per buffer
+    uint8_t w[kStages][kW];
+    uint8_t x[kStages][kXBytes];
+    float hs[2][kBT][kBM];                                      // SwiGLU output staged for the requant
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t red_bar[2];
+    uint32_t tmem_base;
+    volatile int abort_flag;
+    int32_t P[kMaxE + 1];
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreadsM, 1)
+gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                 const float* __restrict__ As, const int32_t* __restrict__ masked_m, int Mmax,
+                 const float* __restrict__ Bs, int E, int N, int K, void* __restrict__ D, float* __restrict__ Ds,
+                 int* status, uint64_t wait_ns) {
+    using S = SmemM<EPI>;
+    extern __shared__ uint8_t smem_raw[];
+    S& sm = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KB = K / kBK;
+    const int NB = N / kBM;                          // 128-row weight blocks per expert
+    const int NBt = EPI == 1 ? NB / 2 : NB;          // weight tiles per expert
+    constexpr uint32_t kTmemCols = EPI == 1 ? 128 : 64;
+
+    if (warp == 0) {
+        // tile prefix over experts: tiles_e = NBt * ceil(m_e / 32)
+        int32_t carry = 0;
+        if (lane == 0) sm.P[0] = 0;
+        for (int b = 0; b < E; b += 32) {
+            const int e = b + lane;
+            int32_t v = e < E ? NBt * ((masked_m[e] + kBT - 1) / kBT) : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            if (e < E) sm.P[e + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < S::kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.tfull[b], 1);
+            mbar_init(&sm.tempty[b], 4);
+            mbar_init(&sm.red_bar[b], 128);
+        }
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const int total = sm.P[E];
+
+    auto fail = [&]() {
+        set_status(status, kStatusTimeout);
+        sm.abort_flag = 1;
+    };
+    auto decode = [&](int tile, int& e, int& nb, int& tt, int& m_e) {
+        e = find_group(sm.P, E, tile);
+        m_e = masked_m[e];
+        const int ntt = (m_e + kBT - 1) / kBT;
+        const int local = tile - sm.P[e];
+        nb = local / ntt;
+        tt = local % ntt;
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&tmX);
+            prefetch_tensormap(&tmW);
+            uint32_t it = 0;
+            for (int tile = blockIdx.x; tile < total && !sm.abort_flag; tile += gridDim.x) {
+                int e, nb, tt, m_e;
+                decode(tile, e, nb, tt, m_e);
+                const int wrow = e * N + nb * (EPI == 1 ? 2 * kBM : kBM);
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = it % S::kStages;
+                    const uint32_t ph = (it / S::kStages) & 1;
+                    if (!mbar_wait(&sm.empty[s], ph ^ 1, wait_ns)) { fail(); break; }
+                    mbar_arrive_expect_tx(&sm.full[s], S::kW + kXBytes);
+                    tma_load_2d(sm.w[s], &tmW, &sm.full[s], kb * kBK, wrow);
+                    if (EPI == 1) tma_load_2d(sm.w[s] + kWBlk, &tmW, &sm.full[s], kb * kBK, wrow + kBM);
+                    tma_load_2d(sm.x[s], &tmX, &sm.full[s], kb * kBK, e * Mmax + tt * kBT);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = f8_idesc(kBM, kBT);
+            uint32_t it = 0, kbt = 0;
+            for (int tile = blockIdx.x; tile < total && !sm.abort_flag; tile += gridDim.x) {
+                for (int kb = 0; kb < KB; ++kb, ++it, ++kbt) {
+                    const int s = it % S::kStages;
+                    const uint32_t ph = (it / S::kStages) & 1;
+                    const int buf = kbt & 1;
+                    const uint32_t bph = (kbt >> 1) & 1;
+                    if (!mbar_wait(&sm.full[s], ph, wait_ns)) { fail(); break; }
+                    if (!mbar_wait(&sm.tempty[buf], bph ^ 1, wait_ns)) { fail(); break; }
+                    tc_fence_after();
+                    const uint32_t w0 = smem_u32(sm.w[s]), x0 = smem_u32(sm.x[s]);
+                    const uint32_t d = tmem + buf * S::kCols;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 32; ++kk) {
+                        const uint64_t xd = sw128_kmajor_desc(x0 + kk * 32);
+                        umma_f8(d, sw128_kmajor_desc(w0 + kk * 32), xd, idesc, kk > 0);
+                        if (EPI == 1) umma_f8(d + kBT, sw128_kmajor_desc(w0 + kWBlk + kk * 32), xd, idesc, kk > 0);
+                    }
+                    umma_commit(&sm.empty[s]);
+                    umma_commit(&sm.tfull[buf]);
+                }
+            }
+        }
+    } else {
+        // promotion + epilogue: 4 warps, thread = tensor-memory lane = weight row
+        const int q = warp & 3;
+        const int pw = warp - 2;                 // 0..3
+        const int r = q * 32 + lane;
+        uint32_t kbt = 0, ep = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            if (sm.abort_flag) break;
+            int e, nb, tt, m_e;
+            decode(tile, e, nb, tt, m_e);
+            float acc[EPI == 1 ? 2 * kBT : kBT];
+#pragma unroll
+            for (int i = 0; i < (EPI == 1 ? 2 * kBT : kBT); ++i) acc[i] = 0.0f;
+            const int blk_a = EPI == 1 ? 2 * nb : nb;
+            const float* bsa = Bs + (static_cast<int64_t>(e) * NB + blk_a) * KB;
+            const float* bsb = bsa + KB;
+            bool ok = true;
+            for (int kb = 0; kb < KB; ++kb, ++kbt) {
+                const int buf = kbt & 1;
+                const uint32_t bph = (kbt >> 1) & 1;
+                const float4* sa4 =
+                    reinterpret_cast<const float4*>(As + (static_cast<int64_t>(e) * KB + kb) * Mmax + tt * kBT);
+                float sa[kBT];
+#pragma unroll
+                for (int i = 0; i < kBT / 4; ++i) {
+                    const float4 v = sa4[i];
+                    sa[4 * i] = v.x; sa[4 * i + 1] = v.y; sa[4 * i + 2] = v.z; sa[4 * i + 3] = v.w;
+                }
+                const float swa = bsa[kb];
+                const float swb = EPI == 1 ? bsb[kb] : 0.0f;
+                if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
+                tc_fence_after();
+                const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * S::kCols;
+                {
+                    float v[32];
+                    tmem_ld32(taddr, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < kBT; ++c) acc[c] = fmaf(v[c], sa[c] * swa, acc[c]);
+                }
+                if (EPI == 1) {
+                    float v[32];
+                    tmem_ld32(taddr + kBT, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < kBT; ++c) acc[kBT + c] = fmaf(v[c], sa[c] * swb, acc[kBT + c]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+            }
+            if (!ok) break;
+            const int nv = min(kBT, m_e - tt * kBT);       // valid tokens in this tile
+            const int64_t row0 = static_cast<int64_t>(e) * Mmax + tt * kBT;
+            if constexpr (EPI == 0) {
+                uint16_t* out = static_cast<uint16_t*>(D) + row0 * N + nb * kBM + r;
+#pragma unroll
+                for (int c = 0; c < kBT; ++c)
+                    if (c < nv) out[static_cast<int64_t>(c) * N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[c]));
+            } else {
+                const int I = N / 2;
+                const int p = ep & 1;
+#pragma unroll
+                for (int c = 0; c < kBT; ++c) sm.hs[p][c][r] = silu_f(acc[c]) * acc[kBT + c];
+                mbar_arrive(&sm.red_bar[p]);
+                if (!mbar_wait(&sm.red_bar[p], (ep >> 1) & 1, wait_ns)) { fail(); break; }
+                ++ep;
+                for (int i = 0; i < kBT / 4; ++i) {
+                    const int c = pw * (kBT / 4) + i;
+                    if (c >= nv) break;
+                    const float4 h4 = *reinterpret_cast<const float4*>(&sm.hs[p][c][lane * 4]);
+                    const float amax = warp_max(fmaxf(fmaxf(fabsf(h4.x), fabsf(h4.y)), fmaxf(fabsf(h4.z), fabsf(h4.w))));
+                    uint32_t packed;
+                    float s = 1.0f;
+                    if (amax == 0.0f) {
+                        packed = f32x2_to_e4m3x2(h4.x, h4.y) | (static_cast<uint32_t>(f32x2_to_e4m3x2(h4.z, h4.w)) << 16);
+                    } else {
+                        s = __fdiv_rn(amax, 448.0f);
+                        packed = f32x2_to_e4m3x2(__fdiv_rn(h4.x, s), __fdiv_rn(h4.y, s)) |
+                                 (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(h4.z, s), __fdiv_rn(h4.w, s))) << 16);
+                    }
+                    uint8_t* hq = static_cast<uint8_t*>(D) + (row0 + c) * I + nb * kBM + lane * 4;
+                    *reinterpret_cast<uint32_t*>(hq) = packed;
+                    if (lane == 0) Ds[(static_cast<int64_t>(e) * (I / kBM) + nb) * Mmax + tt * kBT + c] = s;
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (sm.abort_flag) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < kDrainNs) __nanosleep(1000);
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ====================================================================== host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D map over a row-major byte matrix [rows, cols] read in boxes of 128 bytes x box_rows, 128-byte swizzle.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename Kern>
+static cudaError_t set_smem(Kern k, size_t bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                                const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs, int epilogue,
+                                void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s) {
+    CUtensorMap mapA, mapB;
+    if (layout == 0) {
+        if (!make_map(&mapA, A, K, static_cast<uint64_t>(M_rows), kBM)) return cudaErrorInvalidValue;
+        if (!make_map(&mapB, B, K, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
+        const size_t smem = sizeof(SmemC) + 1024;
+        if (epilogue == 0) {
+            cudaError_t err = set_smem(gg_contig_kernel<0>, smem);
+            if (err != cudaSuccess) return err;
+            gg_contig_kernel<0><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
+                                                                  Ds, status, wait_ns);
+        } else {
+            cudaError_t err = set_smem(gg_contig_kernel<1>, smem);
+            if (err != cudaSuccess) return err;
+            gg_contig_kernel<1><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
+                                                                  Ds, status, wait_ns);
+        }
+    } else {
+        if (!make_map(&mapA, A, K, static_cast<uint64_t>(E) * M_rows, kBT)) return cudaErrorInvalidValue;
+        if (!make_map(&mapB, B, K, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
+        if (epilogue == 0) {
+            const size_t smem = sizeof(SmemM<0>) + 1024;
+            cudaError_t err = set_smem(gg_masked_kernel<0>, smem);
+            if (err != cudaSuccess) return err;
+            gg_masked_kernel<0><<<num_sms, kThreadsM, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
+                                                                  Ds, status, wait_ns);
+        } else {
+            const size_t smem = sizeof(SmemM<1>) + 1024;
+            cudaError_t err = set_smem(gg_masked_kernel<1>, smem);
+            if (err != cudaSuccess) return err;
+            gg_masked_kernel<1><<<num_sms, kThreadsM, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
+                                                                  Ds, status, wait_ns);
+        }
+    }
+    return cudaGetLastError();
+}
+
+// One block waits on a barrier nothing completes; the bounded wait must give up and record a timeout.
+__global__ void selftest_wait_kernel(int* status, uint64_t wait_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        if (!mbar_wait(&bar, 0, wait_ns)) set_status(status, kStatusTimeout);
+    }
+}
+
+cudaError_t launch_selftest_wait(int* status, uint64_t wait_ns, cudaStream_t s) {
+    selftest_wait_kernel<<<1, 32, 0, s>>>(status, wait_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

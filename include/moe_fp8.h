@@ -1,0 +1,211 @@
+/*
+ * moe_fp8.h -- C ABI of a single-GPU FP8 Mixture-of-Experts expert layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (MegaMoE/DeepGEMM page, "2.1 From standard MoE to MegaMoE"):
+ *     y = sum_{i in TopK} G(x)_i * E_i(x),   E_i(x) = W2_i (silu(W1_i x) * W3_i x)
+ * computed as five steps, each an entry point below:
+ *   moe_route            router scores s = softmax(W_g x + b) in fp32, top-k
+ *                        (or hash routing), renormalised weights
+ *   moe_permute          per-expert counts, optional capacity drop, expert-
+ *                        contiguous (or masked per-expert) rows, and the 1x128
+ *                        FP8 quantisation of x written into those rows
+ *   moe_grouped_gemm_fp8 FP8 grouped GEMM: every group has its own M, all groups
+ *                        share N and K; fine-grained fp32 block scales applied
+ *                        in fp32 promotion; epilogue bf16 or SwiGLU + FP8 requant
+ *   moe_combine          weighted un-permute y = sum_j w_j * o_j
+ *   moe_forward          all of the above on one stream, no host sync
+ *
+ * Conventions (every entry point):
+ *  - Every array argument is a DEVICE pointer owned by the caller, except the
+ *    moe_config_t, which is read on the host during the call. The library
+ *    allocates no memory; scratch comes from the caller's `ws` buffer.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream) and never synchronise the host.
+ *  - Argument and shape errors are returned before anything is launched;
+ *    launch failures return MOE_ERR_CUDA. Device-side conditions (a masked
+ *    group overflowing its rows, a bounded wait that ran out) set a status
+ *    word that moe_get_device_status() reports.
+ *  - Device pointers must be 16-byte aligned. H and I must be multiples of 128,
+ *    H at most 16384; the masked layout needs masked_max_m a multiple of 32.
+ *  - bf16 arrays are raw 16-bit words (torch.bfloat16 layout); FP8 arrays are
+ *    E4M3FN codes (torch.float8_e4m3fn layout), one byte each.
+ *  - The group padding (tile M) is fixed at 128 rows.
+ */
+#ifndef MOE_FP8_H
+#define MOE_FP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,        /* null/misaligned pointer, bad enum, k > E, ... */
+    MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* H or I not a multiple of 128, E or k above the limits */
+    MOE_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100 ("FP8 not supported on this GPU",
+                                       MegaMoE page, section 5.1, problem three) */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 4,
+    MOE_ERR_CAPACITY = 5,           /* device status: a masked group had more rows than masked_max_m */
+    MOE_ERR_CUDA = 6,               /* a CUDA runtime call or launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = 7      /* device status: a bounded wait inside a kernel ran out */
+} moe_status_t;
+
+typedef enum { MOE_ROUTE_SOFTMAX_TOPK = 0, MOE_ROUTE_HASH = 1 } moe_routing_t;
+typedef enum { MOE_LAYOUT_CONTIGUOUS = 0, MOE_LAYOUT_MASKED = 1 } moe_layout_t;
+typedef enum { MOE_EPI_BF16 = 0, MOE_EPI_SWIGLU_FP8 = 1 } moe_epilogue_t;
+
+/* Limits checked by every entry point. */
+#define MOE_MAX_EXPERTS 512
+#define MOE_MAX_TOPK 32
+#define MOE_TILE_M 128
+
+typedef struct {
+    int T;              /* tokens (0 allowed: nothing is launched) */
+    int H;              /* hidden size, multiple of 128 */
+    int E;              /* experts, 1..MOE_MAX_EXPERTS */
+    int I;              /* expert intermediate size, multiple of 128 */
+    int k;              /* experts per token (1..min(E, MOE_MAX_TOPK)); hash routing needs k = 1 */
+    int routing;        /* moe_routing_t */
+    int cap_num;        /* capacity factor alpha = cap_num / cap_den; 0 / 0 = dropless */
+    int cap_den;
+    int layout;         /* moe_layout_t */
+    int masked_max_m;   /* rows per expert in the masked layout (ignored when contiguous) */
+} moe_config_t;
+
+/* Rows of the permuted buffers (Aq, As, Hq, Hs, O, row_src) for `cfg`:
+ * contiguous: roundup(T*k + E*127, 128) (every kept slot plus at most 127
+ * padding rows per expert); masked: E * masked_max_m. 0 on a bad config. */
+size_t moe_rows_capacity(const moe_config_t* cfg);
+
+/* Scratch bytes moe_route and moe_permute need (ws_bytes >= this) and, with
+ * for_forward != 0, the bytes moe_forward needs. 0 on a bad config. */
+size_t moe_workspace_size(const moe_config_t* cfg, int for_forward);
+
+/*
+ * Router. Source: s_i = softmax(W_g x + b_i) (MegaMoE page, section 2.2),
+ * softmax in fp32 even for bf16 activations (DeepSeek-V4 lecture page,
+ * section 2.3), top-k of the scores renormalised over the k selected experts
+ * (DeepSeek MoE architecture page, chapter 1 pseudo-code; TP-MoE page,
+ * section 3.1 names renormalisation as one of its two options).
+ *   x         [T, H] bf16, row-major
+ *   Wg        [E, H] fp32, row-major (softmax routing)
+ *   bias      [E] fp32, nullable (no bias)
+ *   token_ids [T] int32 (hash routing only; else ignored, nullable)
+ *   topk_idx  [T, k] int32 out: experts in descending score, ties to the lower index
+ *   topk_w    [T, k] fp32 out: w_j = exp(l_j - m) / sum_{top-k} exp(l_i - m)
+ *   ws        scratch of at least moe_workspace_size(cfg, 0) bytes (holds the T x E logits)
+ * Logits are fp32 with one fixed summation order: 32 interleaved fused
+ * multiply-add chains over h = j, j+32, ..., halved pairwise (j with j+16,
+ * then j+8, 4, 2, 1), then + b. Hash routing (DeepSeek-V4 lecture page,
+ * section 2.2, hash(token_id) % num_experts): expert =
+ * (uint32)(token_id * 2654435761) % E, k = 1, weight 1.
+ */
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* Wg, const float* bias,
+                       const int32_t* token_ids, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
+ * Permutation and activation quantisation. Sources: Concat(E_1(T_1), ...,
+ * E_E(T_E)) as one grouped GEMM (MegaMoE page, section 2.1); a global tile
+ * scheduler over the flattened M of all groups (section 3.2); capacity
+ * ceil(top-k * N / E) * alpha with overflow dropped silently in token order
+ * (DeepSeek MoE page, section 2.5); x_fp8 = clamp(round(x / scale), -448, 448)
+ * (MegaMoE page, section 3.3) with one scale per 1x128 group.
+ *   x          [T, H] bf16
+ *   topk_idx   [T, k] int32 (from moe_route)
+ *   Aq         [rows, H] u8 out (rows = moe_rows_capacity); masked: [E, masked_max_m, H]
+ *   As         [H/128][rows] fp32 out, K-block-major; masked: [E][H/128][masked_max_m]
+ *   counts     [E] int32 out: slots routed to each expert
+ *   kept       [E] int32 out: min(counts, capacity, masked_max_m)
+ *   offsets    [E+1] int32 out: first row of each group; contiguous groups are
+ *              padded to 128 rows, masked offsets[e] = e * masked_max_m
+ *   row_src    [rows] int32 out: slot t*k+j that a row holds, -1 for padding
+ *              (written for rows < offsets[E] in the contiguous layout and for
+ *              the first kept[e] rows of each masked group)
+ *   slot_row   [T*k] int32 out: row of slot t*k+j, or -1 if dropped
+ * Within a group, rows follow token index. Padding rows get code 0 and
+ * scale 1.0. Scale = max|x| / 448 in fp32 (1.0 for an all-zero group);
+ * code = E4M3 round-to-nearest-even, saturating, of the fp32 quotient x / scale.
+ * A masked group with more kept slots than masked_max_m keeps the first
+ * masked_max_m and sets the device status MOE_ERR_CAPACITY.
+ */
+moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                         uint8_t* Aq, float* As, int32_t* counts, int32_t* kept, int32_t* offsets,
+                         int32_t* row_src, int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * FP8 grouped GEMM, D_g = A_g * B_g^T per group g. Sources: every group has
+ * its own M, all share N and K (MegaMoE page, sections 2.1 and 3.2); the
+ * "nt" FP8 x FP8 -> bf16 grouped call with per-group sizes (section 3.2);
+ * fp32 accumulation converted to bf16 with round-to-nearest-even only at the
+ * end (section 3.3); FP8 partial sums promoted to fp32 on the CUDA cores with
+ * fine-grained scales (DeepSeek open-source week page, "Day 3"); bias,
+ * activation and quantisation fused into the epilogue (MegaMoE page, 3.2).
+ *   layout      MOE_LAYOUT_CONTIGUOUS: group_info = offsets [E+1] (multiples of
+ *               128, offsets[E] <= M_rows), rows [offsets[e], offsets[e+1]) use
+ *               expert e; A is [M_rows, K]. MOE_LAYOUT_MASKED: group_info =
+ *               masked_m [E], A is [E, M_rows, K] and rows [0, masked_m[e])
+ *               of block e use expert e.
+ *   A           u8 E4M3 codes, K-major
+ *   As          fp32 1x128 scales, [K/128][M_rows] (masked: [E][K/128][M_rows])
+ *   B           [E, N, K] u8 E4M3 codes, K-major ("nt")
+ *   Bs          [E, N/128, K/128] fp32, one scale per 128x128 block
+ *   epilogue    MOE_EPI_BF16: D = bf16 [rows, N] (RNE); Ds unused.
+ *               MOE_EPI_SWIGLU_FP8: N = 2I and B's 128-row blocks alternate
+ *               W1 block j, W3 block j; h = silu(a) * b in fp32 is quantised
+ *               per 1x128 group: D = u8 [rows, I], Ds = fp32 [I/128][M_rows]
+ *               (masked: [E][I/128][M_rows]), the A/As layout of the next GEMM.
+ * N and K must be multiples of 128 (256 for N with the SwiGLU epilogue).
+ * Contiguous rows outside [0, offsets[E]) and masked rows at or past
+ * masked_m[e] are neither read into any stored result nor written.
+ */
+moe_status_t moe_grouped_gemm_fp8(int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                                  const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
+                                  int epilogue, void* D, float* Ds, void* stream);
+
+/*
+ * Combine. Source: y = sum_{i in TopK} G(x)_i * E_i(x) (MegaMoE page,
+ * section 2.1); bf16 output rounded to nearest even (section 3.3).
+ *   O         [rows, H] bf16 expert outputs (row = slot_row[t*k+j])
+ *   slot_row  [T*k] int32; -1 = dropped slot (contributes nothing; the
+ *             other weights are not renormalised; all dropped -> y = 0)
+ *   topk_w    [T, k] fp32
+ *   y         [T, H] bf16 out: fp32 sum over j = 0..k-1 in order, then RNE
+ */
+moe_status_t moe_combine(const moe_config_t* cfg, const void* O, const int32_t* slot_row,
+                         const float* topk_w, void* y, void* stream);
+
+/*
+ * The whole layer on one stream: route -> permute -> grouped GEMM with W13
+ * (SwiGLU + FP8 requant epilogue) -> grouped GEMM with W2 (bf16) -> combine.
+ *   W13 [E, 2I, H] u8 with 128-row blocks alternating W1 block j, W3 block j
+ *   S13 [E, 2I/128, H/128] fp32 in the same block order
+ *   W2  [E, H, I] u8, S2 [E, H/128, I/128] fp32
+ *   y [T, H] bf16 out; topk_idx, topk_w, counts, slot_row as in the calls above
+ *   ws  scratch of at least moe_workspace_size(cfg, 1) bytes, 256-byte aligned
+ */
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg, const float* bias,
+                         const int32_t* token_ids, const uint8_t* W13, const float* S13,
+                         const uint8_t* W2, const float* S2, void* y, int32_t* topk_idx, float* topk_w,
+                         int32_t* counts, int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: MOE_OK, MOE_ERR_CAPACITY or MOE_ERR_DEVICE_TIMEOUT. */
+moe_status_t moe_get_device_status(void* stream);
+
+/* Test hook for the bounded-wait machinery every kernel uses: launches one
+ * block that waits, for at most `limit_us` microseconds, on a shared-memory
+ * barrier that nothing completes; the wait gives up, records
+ * MOE_ERR_DEVICE_TIMEOUT in the device status word and the kernel returns. */
+moe_status_t moe_selftest_wait_timeout(int limit_us, void* stream);
+
+const char* moe_status_string(moe_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_FP8_H */

@@ -1,0 +1,85 @@
+"""CPU checks of the C-ABI library: it builds for sm_100a, loads, exports every
+entry point include/moe_fp8.h declares, and rejects bad configurations on the
+host before touching a device. Also checks that the product path and the
+oracle share no code."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_grouped_gemm_fp32_b200 import api
+from fp8_grouped_gemm_fp32_b200.build import build
+from fp8_grouped_gemm_fp32_b200.inputs import CONFIGS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_fp8.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return api.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(api.EXPORTS)
+
+
+def test_status_strings(L):
+    for code in range(8):
+        assert api.status_string(code)
+    assert "sm_100" in api.status_string(api.MOE_ERR_UNSUPPORTED_DEVICE)
+
+
+def test_rows_and_workspace_sizes(L):
+    c = api.Config.from_moe(CONFIGS["prefill"])
+    assert api.moe_rows_capacity(c) == -(-(8192 * 8 + 256 * 127) // 128) * 128
+    assert api.moe_rows_capacity(api.Config.from_moe(CONFIGS["decode"])) == 256 * 128
+    assert api.moe_workspace_size(c, True) > api.moe_workspace_size(c, False) > 0
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("H", 100, api.MOE_ERR_UNSUPPORTED_SHAPE), ("I", 200, api.MOE_ERR_UNSUPPORTED_SHAPE),
+    ("E", 513, api.MOE_ERR_UNSUPPORTED_SHAPE), ("k", 9, api.MOE_ERR_INVALID_ARG),
+    ("k", 0, api.MOE_ERR_INVALID_ARG), ("T", -1, api.MOE_ERR_INVALID_ARG),
+    ("routing", 5, api.MOE_ERR_INVALID_ARG), ("cap_num", 3, api.MOE_ERR_INVALID_ARG),
+    ("layout", 2, api.MOE_ERR_INVALID_ARG), ("H", 16512, api.MOE_ERR_UNSUPPORTED_SHAPE)])
+def test_bad_config_rejected_before_any_device_work(L, field, value, code):
+    c = api.Config.from_moe(CONFIGS["tiny"])
+    setattr(c, field, value)
+    assert api.moe_workspace_size(c) == 0
+    st = L.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, 0, None)
+    assert st == code
+
+
+def test_hash_routing_needs_k1_and_masked_needs_rows(L):
+    c = api.Config.from_moe(CONFIGS["decode_hash"])
+    c.k = 2
+    assert api.moe_workspace_size(c) == 0
+    c = api.Config.from_moe(CONFIGS["decode"])
+    c.masked_max_m = 100                       # not a multiple of 32
+    assert api.moe_workspace_size(c) == 0
+
+
+def test_product_and_oracle_share_no_code():
+    pkg = os.path.join(ROOT, "fp8_grouped_gemm_fp32_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), f
+                assert "moe_oracle" not in src, f
+    osrc = open(os.path.join(ROOT, "oracle", "__init__.py")).read()
+    assert not re.search(r"^\s*(import|from)\s+fp8_grouped_gemm_fp32_b200\b", osrc, re.M)
+    assert "moe_fp8.h" not in open(os.path.join(ROOT, "oracle", "moe_oracle.c")).read()

@@ -1,0 +1,267 @@
+"""GPU parity of each C-ABI step against the oracle on identical inputs:
+
+* moe_route: indices bit-exact (including ties), weights to 1e-6, on every
+  workload at full size;
+* moe_permute (fed the oracle's routing): counts, kept, offsets, row_src,
+  slot_row and the quantised rows Aq / scales As bit-exact, padding included;
+* moe_grouped_gemm_fp8: both layouts x both epilogues on ragged groups
+  (empty groups, 1 row, tiles plus a ragged tail, a half-width N tile);
+* moe_combine (fed the oracle's expert outputs), with dropped slots.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_grouped_gemm_fp32_b200 import api
+from fp8_grouped_gemm_fp32_b200.inputs import CONFIGS, MoeConfig, capacity_rows_bound
+from gpu_helpers import (W_RTOL, assert_close_bf16, ensure_lib, gpu_inputs, oracle_inputs, rel_errors,
+                         to_np)
+
+pytestmark = pytest.mark.gpu
+
+
+def _route(cfg, inp):
+    c = api.Config.from_moe(cfg)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(api.moe_workspace_size(c), 16), dtype=torch.uint8, device="cuda")
+    api.moe_route(c, inp.x, inp.Wg, inp.bias, inp.token_ids, idx, w, ws)
+    torch.cuda.synchronize()
+    return to_np(idx), to_np(w)
+
+
+@pytest.mark.parametrize("name", ["tiny", "page", "prefill", "decode", "decode_hash", "skewed"])
+def test_route_full_size(name):
+    ensure_lib()
+    cfg = CONFIGS[name]
+    inp = gpu_inputs(cfg, on_device=name not in ("tiny",))
+    idx, w = _route(cfg, inp)
+    ref_idx, ref_w, _ = oracle.route(cfg, to_np(inp.x), to_np(inp.Wg), to_np(inp.bias), to_np(inp.token_ids))
+    assert np.array_equal(idx, ref_idx)
+    assert np.allclose(w, ref_w, rtol=W_RTOL, atol=0)
+    assert np.allclose(w.sum(1), 1.0, atol=1e-5)
+
+
+def test_route_ties_and_ragged_shapes():
+    # E not a multiple of the kernel's expert tile, T not a multiple of its token tile,
+    # and rows of x equal to each other so whole tokens tie (identical logits per expert
+    # pair from duplicated W_g rows): the lower expert index must win every tie.
+    ensure_lib()
+    cfg = MoeConfig("ties", T=77, H=384, E=13, I=128, k=3, bias="zero", seed=21)
+    inp = gpu_inputs(cfg)
+    inp.Wg[5] = inp.Wg[2]
+    inp.Wg[11] = inp.Wg[2]
+    inp.Wg[7] = inp.Wg[0]
+    inp.x[10] = inp.x[3]
+    idx, w = _route(cfg, inp)
+    ref_idx, ref_w, logits = oracle.route(cfg, to_np(inp.x), to_np(inp.Wg), to_np(inp.bias), None)
+    assert np.array_equal(idx, ref_idx)
+    assert np.allclose(w, ref_w, rtol=W_RTOL, atol=0)
+    assert np.any(logits[:, 2] == logits[:, 5])
+
+
+def _permute(cfg, inp, topk_idx):
+    c = api.Config.from_moe(cfg)
+    rows = api.moe_rows_capacity(c)
+    H, E = cfg.H, cfg.E
+    masked = cfg.layout == "masked"
+    dev = "cuda"
+    Aq = torch.full((rows, H), 0xAB, dtype=torch.uint8, device=dev)       # poison: every byte must be written
+    if masked:
+        As = torch.full((E, H // 128, cfg.masked_max_m), -7.0, dtype=torch.float32, device=dev)
+    else:
+        As = torch.full((H // 128, rows), -7.0, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    kept = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_src = torch.full((rows,), -99, dtype=torch.int32, device=dev)
+    slot_row = torch.empty(cfg.T * topk_idx.shape[1], dtype=torch.int32, device=dev)
+    ws = torch.empty(api.moe_workspace_size(c), dtype=torch.uint8, device=dev)
+    api.moe_permute(c, inp.x, torch.from_numpy(topk_idx).to(dev), Aq, As, counts, kept, offsets, row_src,
+                    slot_row, ws)
+    torch.cuda.synchronize()
+    return dict(Aq=to_np(Aq), As=to_np(As), counts=to_np(counts), kept=to_np(kept), offsets=to_np(offsets),
+                row_src=to_np(row_src), slot_row=to_np(slot_row)), rows
+
+
+@pytest.mark.parametrize("name,T", [("tiny", None), ("skewed", 4096), ("prefill", 512), ("decode", None),
+                                    ("decode_hash", None), ("page", 1000)])
+def test_permute_bit_exact(name, T):
+    ensure_lib()
+    cfg = CONFIGS[name]
+    inp = gpu_inputs(cfg, T=T, on_device=cfg.H > 1024)
+    cfg = inp.cfg
+    ref_idx, _, _ = oracle.route(cfg, to_np(inp.x), to_np(inp.Wg), to_np(inp.bias), to_np(inp.token_ids))
+    got, rows = _permute(cfg, inp, ref_idx)
+    ref = oracle.permute(cfg, to_np(inp.x), ref_idx, rows)
+    for key in ("counts", "kept", "offsets", "slot_row"):
+        assert np.array_equal(got[key], ref[key]), key
+    if cfg.layout == "masked":
+        M = cfg.masked_max_m
+        for e in range(cfg.E):
+            r0, r1 = e * M, e * M + ref["kept"][e]
+            assert np.array_equal(got["row_src"][r0:r1], ref["row_src"][r0:r1])
+            assert np.array_equal(got["Aq"][r0:r1], ref["Aq"][r0:r1])
+            assert np.array_equal(got["As"][e, :, :ref["kept"][e]], ref["As"][e, :, :ref["kept"][e]])
+    else:
+        used = ref["offsets"][-1]
+        assert np.array_equal(got["row_src"][:used], ref["row_src"][:used])
+        assert np.array_equal(got["Aq"][:used], ref["Aq"][:used])          # padding rows are 0 too
+        assert np.array_equal(got["As"][:, :used], ref["As"][:, :used])    # padding scales are 1
+    if cfg.cap_num:
+        assert np.count_nonzero(ref["slot_row"] < 0) > 0
+
+
+def _rand_codes(rng, shape):
+    c = rng.integers(0, 256, size=shape, dtype=np.uint8)
+    c[(c & 0x7F) == 0x7F] = 0x3C                              # no NaN codes
+    return c
+
+
+def _gemm_case(layout, epilogue, E, N, K, groups, M_rows=None, seed=0):
+    rng = np.random.default_rng(seed)
+    G = K // 128
+    if layout == 0:
+        offs = [0]
+        for g in groups:
+            offs.append(offs[-1] + -(-g // 128) * 128)
+        rows = offs[-1] + 256                                 # some rows past the last group
+        A = _rand_codes(rng, (rows, K))
+        As = rng.uniform(0.002, 0.02, (G, rows)).astype(np.float32)
+        gi = np.array(offs, np.int32)
+        M = rows
+    else:
+        M = M_rows
+        A = _rand_codes(rng, (E * M, K))
+        As = rng.uniform(0.002, 0.02, (E, G, M)).astype(np.float32)
+        gi = np.array(groups, np.int32)
+    B = _rand_codes(rng, (E, N, K))
+    Bs = rng.uniform(1e-4, 1e-3, (E, N // 128, G)).astype(np.float32)
+    return A, As, gi, M, B, Bs
+
+
+def _gemm_gpu(layout, epilogue, E, N, K, A, As, gi, M, B, Bs):
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    rows = A.shape[0]
+    if epilogue == 0:
+        D = torch.zeros(rows, N, dtype=torch.bfloat16, device="cuda")
+        Ds = None
+    else:
+        D = torch.zeros(rows, N // 2, dtype=torch.uint8, device="cuda")
+        G = N // 256
+        Ds = torch.zeros((G, M) if layout == 0 else (E, G, M), dtype=torch.float32, device="cuda")
+    api.moe_grouped_gemm_fp8(layout, E, N, K, d(A), d(As), d(gi), M, d(B), d(Bs), epilogue, D, Ds)
+    torch.cuda.synchronize()
+    assert api.moe_get_device_status() == api.MOE_OK
+    return to_np(D), (None if Ds is None else to_np(Ds))
+
+
+def _valid_rows(layout, gi, M, E):
+    if layout == 0:
+        return np.arange(gi[-1])
+    return np.concatenate([e * M + np.arange(gi[e]) for e in range(E)]).astype(np.int64)
+
+
+GEMM_CASES = [
+    # layout, epilogue, E, N, K, groups, M_rows
+    (0, 0, 5, 640, 384, [0, 1, 130, 255, 40], None),      # half-width last N tile (640 = 2*256 + 128)
+    (0, 1, 5, 512, 384, [0, 1, 130, 255, 40], None),
+    (0, 0, 3, 256, 1024, [300, 0, 129], None),
+    (1, 0, 4, 384, 256, [0, 5, 33, 64], 64),
+    (1, 1, 4, 512, 256, [0, 5, 33, 64], 64),
+    (1, 1, 3, 256, 512, [32, 1, 0], 96),
+]
+
+
+@pytest.mark.parametrize("case", GEMM_CASES)
+def test_grouped_gemm(case):
+    ensure_lib()
+    layout, epi, E, N, K, groups, Mr = case
+    A, As, gi, M, B, Bs = _gemm_case(layout, epi, E, N, K, groups, Mr, seed=sum(groups) + N)
+    D, Ds = _gemm_gpu(layout, epi, E, N, K, A, As, gi, M, B, Bs)
+    Dr, Dsr = oracle.grouped_gemm(layout, E, N, K, A, As, gi, M, B, Bs, epi)
+    rows = _valid_rows(layout, gi, M, E)
+    if epi == 0:
+        assert_close_bf16(D[rows], Dr[rows], "D")
+        assert np.mean(D[rows] == Dr[rows]) > 0.95
+    else:
+        same = D[rows] == Dr[rows]
+        assert same.mean() > 0.999, same.mean()
+        diff = np.abs(D[rows].astype(np.int32) - Dr[rows].astype(np.int32))
+        assert np.all(diff[~same] == 1)                     # at worst one E4M3 step apart
+        if layout == 0:
+            s, sr = Ds[:, rows], Dsr[:, rows]
+        else:
+            s = np.concatenate([Ds[e, :, :gi[e]] for e in range(E)], axis=1)
+            sr = np.concatenate([Dsr[e, :, :gi[e]] for e in range(E)], axis=1)
+        assert np.allclose(s, sr, rtol=1e-5, atol=0)
+
+
+def test_combine_with_drops():
+    ensure_lib()
+    cfg = MoeConfig("comb", T=300, H=384, E=4, I=128, k=3, bias="uniform", cap_num=1, cap_den=2, seed=31)
+    inp = gpu_inputs(cfg)
+    ref_idx, ref_w, _ = oracle.route(cfg, to_np(inp.x), to_np(inp.Wg), to_np(inp.bias), None)
+    rows = capacity_rows_bound(cfg)
+    d = oracle.dispatch(ref_idx, cfg.E, oracle.capacity(cfg.T, cfg.k, cfg.E, 1, 2), 0, 128, 0, rows)
+    rng = np.random.default_rng(3)
+    O = torch.randn(rows, cfg.H).to(torch.bfloat16)
+    O_bits = O.view(torch.int16).numpy().view(np.uint16)
+    y_ref = oracle.combine(d["slot_row"], ref_w, O_bits, cfg.T, cfg.k)
+    y = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    api.moe_combine(api.Config.from_moe(cfg), O.cuda(), torch.from_numpy(d["slot_row"]).cuda(),
+                    torch.from_numpy(ref_w).cuda(), y)
+    torch.cuda.synchronize()
+    assert np.count_nonzero(d["slot_row"] < 0) > 0
+    all_dropped = np.nonzero((d["slot_row"].reshape(cfg.T, cfg.k) < 0).all(1))[0]
+    assert len(all_dropped) > 0 and np.all(to_np(y)[all_dropped] == 0)
+    assert_close_bf16(to_np(y), y_ref)
+    assert np.mean(to_np(y) == y_ref) > 0.99
+
+
+def test_empty_batch_is_a_no_op():
+    ensure_lib()
+    cfg = MoeConfig("empty", T=0, H=256, E=4, I=128, k=2, seed=0)
+    c = api.Config.from_moe(cfg)
+    ws = torch.empty(max(api.moe_workspace_size(c, True), 256), dtype=torch.uint8, device="cuda")
+    z = lambda *s, dt=torch.int32: torch.empty(*s, dtype=dt, device="cuda")
+    inp = gpu_inputs(cfg.replace(T=4))
+    from fp8_grouped_gemm_fp32_b200.inputs import interleave_w13
+    W13, S13 = interleave_w13(inp.W1q, inp.S1, inp.W3q, inp.S3)
+    # zero tokens: every buffer may be empty; pass small dummies where the ABI wants a pointer
+    dummy = z(64)
+    api.moe_forward(c, dummy, inp.Wg, inp.bias, None, W13, S13, inp.W2q, inp.S2, dummy, dummy, dummy,
+                    z(cfg.E), dummy, ws)
+    torch.cuda.synchronize()
+    assert api.moe_get_device_status() == api.MOE_OK
+
+
+def test_device_timeout_is_reported_and_context_survives():
+    ensure_lib()
+    assert api.moe_get_device_status() == api.MOE_OK
+    api.moe_selftest_wait_timeout(2000)                  # a 2 ms wait on a barrier nothing completes
+    assert api.moe_get_device_status() == api.MOE_ERR_DEVICE_TIMEOUT
+    assert api.moe_get_device_status() == api.MOE_OK     # read-and-clear
+    test_combine_with_drops()                             # the context still works
+
+
+def test_host_side_errors_on_device():
+    ensure_lib()
+    cfg = CONFIGS["tiny"]
+    inp = gpu_inputs(cfg)
+    c = api.Config.from_moe(cfg)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(api.MoeError) as ei:
+        api.moe_route(c, inp.x, inp.Wg, inp.bias, None, idx, w, small)
+    assert ei.value.status == api.MOE_ERR_WORKSPACE_TOO_SMALL
+    ws = torch.empty(api.moe_workspace_size(c), dtype=torch.uint8, device="cuda")
+    mis = torch.empty(cfg.T * cfg.k * 4 + 4, dtype=torch.uint8, device="cuda")[4:].view(torch.int32)
+    with pytest.raises(api.MoeError) as ei:
+        api.moe_route(c, inp.x, inp.Wg, inp.bias, None, mis, w, ws)
+    assert ei.value.status == api.MOE_ERR_INVALID_ARG          # misaligned pointer
+    with pytest.raises(api.MoeError) as ei:
+        api.moe_grouped_gemm_fp8(0, 4, 200, 256, inp.x, w, idx, 128, inp.x, w, 0, idx)
+    assert ei.value.status == api.MOE_ERR_UNSUPPORTED_SHAPE    # N not a multiple of 128
