@@ -221,29 +221,48 @@ def max_over_ranks(v: float, world: int) -> float:
     return float(t.item())
 
 
-def cpu_baseline(cfg: MoeConfig, target_s: float = 12.0):
+class _HostExperts:
+    """Expert-indexed host view of a device weight tensor (one expert copied per access)."""
+
+    def __init__(self, t):
+        self.t = t
+
+    def __getitem__(self, e):
+        return self.t[e].cpu().numpy()
+
+
+def _oracle_view(inp):
+    """numpy view of a MoeInputs for the oracle; weights stay put until an expert is used."""
+    return dict(x=inp.x.cpu().view(torch.int16).numpy().view(np.uint16), Wg=inp.Wg.cpu().numpy(),
+                bias=inp.bias.cpu().numpy(), token_ids=inp.token_ids.cpu().numpy(),
+                W1q=_HostExperts(inp.W1q), S1=_HostExperts(inp.S1), W3q=_HostExperts(inp.W3q),
+                S3=_HostExperts(inp.S3), W2q=_HostExperts(inp.W2q), S2=_HostExperts(inp.S2))
+
+
+def _oracle_step(cfg, view, n, threads):
+    """One oracle pass over the first n tokens of the workload as one batch; returns seconds."""
+    import oracle
+    sub = dict(view)
+    sub["x"] = view["x"][:n]
+    sub["token_ids"] = view["token_ids"][:n]
+    c = cfg.replace(T=n, masked_max_m=(-(-n // 32) * 32 if cfg.layout == "masked" else cfg.masked_max_m))
+    t0 = time.perf_counter()
+    oracle.forward(c, sub, nthreads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg: MoeConfig, inp, target_s: float = 12.0):
     """The oracle, as it stands, on a bounded sample of the workload's tokens."""
     import oracle
     threads = oracle.default_threads()
-    full = make_inputs(cfg, device="cpu", T=min(cfg.T, 256))
-    npi = oracle.moe_inputs_to_numpy(full)
-
-    def run(n):
-        sub = dict(npi)
-        sub["x"] = npi["x"][:n]
-        sub["token_ids"] = npi["token_ids"][:n]
-        c = cfg.replace(T=n, masked_max_m=(-(-n // 32) * 32 if cfg.layout == "masked" else cfg.masked_max_m))
-        t0 = time.perf_counter()
-        oracle.forward(c, sub, nthreads=threads)
-        return time.perf_counter() - t0
-
+    view = _oracle_view(inp)
     n = 2
-    dt = run(n)
-    n = int(max(1, min(full.cfg.T, math.floor(n * target_s / max(dt, 1e-3)))))
-    dt = run(n)
+    dt = _oracle_step(cfg, view, n, threads)
+    n = int(max(1, min(cfg.T, math.floor(n * target_s / max(dt, 1e-3)))))
+    dt = _oracle_step(cfg, view, n, threads)
     return {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"first {n} tokens of the {cfg.name} workload as one batch (routing, permutation, "
-                      f"expert math in fp64, combine), {dt:.1f} s"}
+                      f"expert math in fp64 split over {threads} threads, combine), {dt:.1f} s"}
 
 
 def run_ours(args):
@@ -356,7 +375,7 @@ def run_ours(args):
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg)
+        line["cpu_baseline"] = cpu_baseline(cfg, layer.inp)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -372,26 +391,17 @@ def run_reference(args):
     import oracle
     cfg = CONFIGS[args.config]
     threads = oracle.default_threads()
-    inp = oracle.moe_inputs_to_numpy(make_inputs(cfg, device="cpu", T=min(cfg.T, 256)))
-
-    def step(n):
-        sub = dict(inp)
-        sub["x"] = inp["x"][:n]
-        sub["token_ids"] = inp["token_ids"][:n]
-        c = cfg.replace(T=n, masked_max_m=(-(-n // 32) * 32 if cfg.layout == "masked" else cfg.masked_max_m))
-        t0 = time.perf_counter()
-        oracle.forward(c, sub, nthreads=threads)
-        return time.perf_counter() - t0
-
+    dev = "cuda" if torch.cuda.is_available() else "cpu"     # where the seeded workload is drawn
+    view = _oracle_view(make_inputs(cfg, device=dev, T=min(cfg.T, 512)))
     budget = 150.0 / max(1, args.steps + args.warmup)        # whole run within a few minutes
-    dt = step(2)
-    n = int(max(1, min(256, math.floor(2 * min(budget, 10.0) / max(dt, 1e-3)))))
+    dt = _oracle_step(cfg, view, 2, threads)
+    n = int(max(1, min(512, math.floor(2 * min(budget, 10.0) / max(dt, 1e-3)))))
     for _ in range(args.warmup):
-        step(n)
-    times = [step(n) for _ in range(args.steps)]
+        _oracle_step(cfg, view, n, threads)
+    times = [_oracle_step(cfg, view, n, threads) for _ in range(args.steps)]
     ms = 1e3 * sum(times) / len(times)
     value = n / (ms / 1e3)
-    sample = f"first {n} tokens of the {cfg.name} workload per step as one batch"
+    sample = f"first {n} tokens of the {cfg.name} workload per step as one batch, {threads} threads"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp64 (oracle)", "data": "synthetic",

@@ -132,7 +132,11 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         sm.abort_flag = 1;
     };
 
-    if (warp == 0) {
+    // Register split (launch: 384 threads x 168 = 64512): the TMA/MMA warpgroup gives up
+    // registers to the two promotion warpgroups, 128 x 56 + 256 x 224 = 64512.
+    if (warp < 4) {
+      setmaxnreg_dec<56>();
+      if (warp == 0) {
         // ---------------- TMA producer
         if (lane == 0) {
             prefetch_tensormap(&tmA);
@@ -153,7 +157,7 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
             }
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
             uint32_t it = 0, kbt = 0;
@@ -178,7 +182,9 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
             }
         }
-    } else if (warp >= 4) {
+      }
+    } else {
+        setmaxnreg_inc<224>();
         // ---------------- promotion + epilogue (256 threads)
         const int q = warp & 3;                 // tensor-memory lane quadrant
         const int half = (warp - 4) >> 2;       // which 64 columns of each 128-column half
@@ -192,36 +198,51 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
             const float* bs0 = Bs + (static_cast<int64_t>(t.e) * NB + t.n0 / kBM) * KB;
-            const float* bs1 = bs0 + KB;
+            const float* bs1 = full ? bs0 + KB : bs0;
             const float* as_row = As + t.m0 + row;
+            // scales run two K blocks ahead of their use, so their L2 latency overlaps the MMAs
+            float sa_0 = as_row[0], w0_0 = bs0[0], w1_0 = bs1[0];
+            float sa_1 = 0.f, w0_1 = 0.f, w1_1 = 0.f;
+            if (KB > 1) { sa_1 = as_row[M_rows]; w0_1 = bs0[1]; w1_1 = bs1[1]; }
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb, ++kbt) {
                 const int buf = kbt & 1;
                 const uint32_t bph = (kbt >> 1) & 1;
-                const float sa = as_row[static_cast<int64_t>(kb) * M_rows];
-                const float f0 = sa * bs0[kb];
-                const float f1 = full ? sa * bs1[kb] : 0.0f;
+                float sa_2 = 0.f, w0_2 = 0.f, w1_2 = 0.f;
+                if (kb + 2 < KB) {
+                    sa_2 = as_row[static_cast<int64_t>(kb + 2) * M_rows];
+                    w0_2 = bs0[kb + 2];
+                    w1_2 = bs1[kb + 2];
+                }
+                const float f0 = sa_0 * w0_0;
+                const float f1 = sa_0 * w1_0;
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kBN + half * 64;
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    float v[32];
-                    tmem_ld32(taddr + c * 32, v);
+                {
+                    float v0[32], v1[32];
+                    tmem_ld32(taddr, v0);
+                    tmem_ld32(taddr + 32, v1);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(v[i], f0, acc[c * 32 + i]);
-                }
-                if (full) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float v[32];
-                        tmem_ld32(taddr + 128 + c * 32, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) acc[64 + c * 32 + i] = fmaf(v[i], f1, acc[64 + c * 32 + i]);
+                    for (int i = 0; i < 32; ++i) {
+                        acc[i] = fmaf(v0[i], f0, acc[i]);
+                        acc[32 + i] = fmaf(v1[i], f0, acc[32 + i]);
                     }
                 }
+                if (full) {
+                    float v0[32], v1[32];
+                    tmem_ld32(taddr + 128, v0);
+                    tmem_ld32(taddr + 160, v1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        acc[64 + i] = fmaf(v0[i], f1, acc[64 + i]);
+                        acc[96 + i] = fmaf(v1[i], f1, acc[96 + i]);
+                    }
+                }
+                sa_0 = sa_1; w0_0 = w0_1; w1_0 = w1_1;
+                sa_1 = sa_2; w0_1 = w0_2; w1_1 = w1_2;
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.tempty[buf]);

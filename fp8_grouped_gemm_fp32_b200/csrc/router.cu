@@ -13,32 +13,39 @@
 // shared memory feeds TR x ER register accumulators per lane (CUDA cores: the
 // fixed order rules out the tensor cores); logits go to scratch, and a
 // warp-per-token kernel selects the top-k and computes the weights in fp64.
+// W_g (7.3 MB at the largest size) stays L2-resident across token tiles.
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int kRouterHS = 128;     // h values per pipeline stage
-constexpr int kRouterStages = 3;
+constexpr int kRouterHS = 128;     // h values per stage
+constexpr int kPlaneRows = kRouterHS;
+constexpr int kPlaneBytes = kPlaneRows * 16;   // one plane: 128 rows x 16 bytes
+
+// Operands are staged h-major in "planes" of 16 bytes per h: 8 tokens (bf16) or 4
+// experts (fp32) per plane, so a lane fetches all the tokens (experts) it needs for
+// its h with one 16-byte load per plane. Rows are XOR-swizzled within each 8-row
+// group, and W planes are padded by 32 bytes, so both the transposing stores and the
+// 16-byte loads are free of bank conflicts.
+__device__ __forceinline__ int swz_row(int row) { return row ^ ((row >> 3) & 7); }
 
 template <int TR, int ER, int WT, int WE>
 struct RouterTile {
-    static constexpr int TT = TR * WT;       // tokens per CTA
-    static constexpr int EC = ER * WE;       // experts per CTA
+    static constexpr int TT = TR * WT;               // tokens per CTA
+    static constexpr int EC = ER * WE;               // experts per CTA
     static constexpr int kThreads = 32 * WT * WE;
-    static constexpr int kXBytes = TT * kRouterHS * 2;
-    static constexpr int kWBytes = EC * kRouterHS * 4;
-    static constexpr int kStageBytes = kXBytes + kWBytes;
-    static constexpr int kSmem = kRouterStages * kStageBytes;
+    static constexpr int kXPlanes = TT / 8;
+    static constexpr int kWPlanes = EC / 4;
+    static constexpr int kWPlaneStride = kPlaneBytes + 32;
+    static constexpr int kXBytes = kXPlanes * kPlaneBytes;
+    static constexpr int kStageBytes = kXBytes + kWPlanes * kWPlaneStride;
+    static constexpr int kSmem = 2 * kStageBytes;
+    // global -> register chunks per thread per stage (16 bytes each)
+    static constexpr int kXChunks = TT * (kRouterHS / 8) / kThreads;     // 8 h of one token
+    static constexpr int kWChunks = EC * (kRouterHS / 4) / kThreads;     // 4 h of one expert
+    static_assert(TR % 8 == 0 && ER % 4 == 0, "register tile must cover whole planes");
+    static_assert(TT * (kRouterHS / 8) % kThreads == 0 && EC * (kRouterHS / 4) % kThreads == 0, "chunking");
 };
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
-    const uint32_t s = smem_u32(smem);
-    const int bytes = valid ? 16 : 0;   // 0 source bytes -> the 16 bytes are zero-filled
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int TR, int ER, int WT, int WE>
 __global__ void __launch_bounds__(RouterTile<TR, ER, WT, WE>::kThreads, 1)
@@ -48,28 +55,68 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
     extern __shared__ __align__(128) uint8_t smem[];
     const int t_base = blockIdx.x * Tile::TT;
     const int e_base = blockIdx.y * Tile::EC;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
     const int wt = warp / WE, we = warp % WE;
     const int nst = H / kRouterHS;
 
-    auto issue_stage = [&](int st) {
-        uint8_t* sx = smem + (st % kRouterStages) * Tile::kStageBytes;
-        uint8_t* sw = sx + Tile::kXBytes;
+    // Chunk c of a stage: x chunks are (token, 8-h piece) with 4 pieces of one token per
+    // 4 consecutive threads and 8 tokens per warp; W chunks are (expert, 4-h piece) alike.
+    uint4 xr[Tile::kXChunks], wr[Tile::kWChunks];
+    auto load_stage = [&](int st) {
         const int h0 = st * kRouterHS;
-        // x tile: TT rows x 256 bytes = TT*16 chunks; W tile: EC rows x 512 bytes = EC*32 chunks
-        for (int c = threadIdx.x; c < Tile::TT * 16; c += Tile::kThreads) {
-            const int r = c >> 4, q = c & 15;
-            const int t = t_base + r;
-            const bool ok = t < T;
-            const uint16_t* src = x + static_cast<int64_t>(ok ? t : 0) * H + h0 + q * 8;
-            cp_async16(sx + r * 256 + q * 16, src, ok);
+#pragma unroll
+        for (int i = 0; i < Tile::kXChunks; ++i) {
+            const int c = tid + i * Tile::kThreads;          // 0 .. TT*16
+            const int grp = c >> 5, l = c & 31;               // 32 chunks: 8 tokens x 4 pieces
+            const int tok = (grp % (Tile::TT / 8)) * 8 + (l >> 2);
+            const int piece = (grp / (Tile::TT / 8)) * 4 + (l & 3);
+            const int t = t_base + tok;
+            xr[i] = t < T ? *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H + h0 + piece * 8)
+                          : make_uint4(0, 0, 0, 0);
         }
-        for (int c = threadIdx.x; c < Tile::EC * 32; c += Tile::kThreads) {
-            const int r = c >> 5, q = c & 31;
-            const int e = e_base + r;
-            const bool ok = e < E;
-            const float* src = Wg + static_cast<int64_t>(ok ? e : 0) * H + h0 + q * 4;
-            cp_async16(sw + r * 512 + q * 16, src, ok);
+#pragma unroll
+        for (int i = 0; i < Tile::kWChunks; ++i) {
+            const int c = tid + i * Tile::kThreads;          // 0 .. EC*32
+            const int grp = c >> 5, l = c & 31;               // 32 chunks: 8 experts x 4 pieces
+            const int ex = (grp % (Tile::EC / 8)) * 8 + (l >> 2);
+            const int piece = (grp / (Tile::EC / 8)) * 4 + (l & 3);
+            const int e = e_base + ex;
+            wr[i] = e < E ? *reinterpret_cast<const uint4*>(Wg + static_cast<int64_t>(e) * H + h0 + piece * 4)
+                          : make_uint4(0, 0, 0, 0);
+        }
+    };
+    auto store_stage = [&](int buf) {
+        uint8_t* sx = smem + buf * Tile::kStageBytes;
+        uint8_t* sw = sx + Tile::kXBytes;
+#pragma unroll
+        for (int i = 0; i < Tile::kXChunks; ++i) {
+            const int c = tid + i * Tile::kThreads;
+            const int grp = c >> 5, l = c & 31;
+            const int tok = (grp % (Tile::TT / 8)) * 8 + (l >> 2);
+            const int piece = (grp / (Tile::TT / 8)) * 4 + (l & 3);
+            uint8_t* plane = sx + (tok >> 3) * kPlaneBytes + (tok & 7) * 2;
+            const uint32_t u[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int row = piece * 8 + r;
+                *reinterpret_cast<uint16_t*>(plane + swz_row(row) * 16) =
+                    static_cast<uint16_t>(r & 1 ? u[r >> 1] >> 16 : u[r >> 1] & 0xffffu);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < Tile::kWChunks; ++i) {
+            const int c = tid + i * Tile::kThreads;
+            const int grp = c >> 5, l = c & 31;
+            const int ex = (grp % (Tile::EC / 8)) * 8 + (l >> 2);
+            const int piece = (grp / (Tile::EC / 8)) * 4 + (l & 3);
+            uint8_t* plane = sw + (ex >> 2) * Tile::kWPlaneStride + (ex & 3) * 4;
+            const uint32_t u[4] = {wr[i].x, wr[i].y, wr[i].z, wr[i].w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int row = piece * 4 + r;
+                *reinterpret_cast<uint32_t*>(plane + swz_row(row) * 16) = u[r];
+            }
         }
     };
 
@@ -79,34 +126,45 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
 #pragma unroll
         for (int q = 0; q < ER; ++q) acc[i][q] = 0.0f;
 
-#pragma unroll
-    for (int st = 0; st < kRouterStages - 1; ++st) {
-        if (st < nst) issue_stage(st);
-        cp_async_commit();
-    }
+    load_stage(0);
+    store_stage(0);
+    if (nst > 1) load_stage(1);
+    __syncthreads();
     for (int st = 0; st < nst; ++st) {
-        cp_async_wait<kRouterStages - 2>();
-        __syncthreads();
-        if (st + kRouterStages - 1 < nst) issue_stage(st + kRouterStages - 1);
-        cp_async_commit();
-        const uint8_t* sx = smem + (st % kRouterStages) * Tile::kStageBytes;
-        const uint16_t* xs = reinterpret_cast<const uint16_t*>(sx) + (wt * TR) * kRouterHS;
-        const float* ws = reinterpret_cast<const float*>(sx + Tile::kXBytes) + (we * ER) * kRouterHS;
+        const uint8_t* sx = smem + (st & 1) * Tile::kStageBytes;
+        const uint8_t* sxw = sx + (wt * (TR / 8)) * kPlaneBytes;
+        const uint8_t* sww = sx + Tile::kXBytes + (we * (ER / 4)) * Tile::kWPlaneStride;
 #pragma unroll
         for (int s = 0; s < kRouterHS / 32; ++s) {
-            const int h = s * 32 + lane;
+            const int row16 = swz_row(s * 32 + lane) * 16;
             float xv[TR], wv[ER];
 #pragma unroll
-            for (int i = 0; i < TR; ++i) xv[i] = bf16_bits_to_f32(xs[i * kRouterHS + h]);
+            for (int p = 0; p < TR / 8; ++p) {
+                const uint4 v = *reinterpret_cast<const uint4*>(sxw + p * kPlaneBytes + row16);
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int q = 0; q < ER; ++q) wv[q] = ws[q * kRouterHS + h];
+                for (int i = 0; i < 4; ++i) {
+                    xv[p * 8 + 2 * i] = __uint_as_float(u[i] << 16);
+                    xv[p * 8 + 2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < ER / 4; ++p) {
+                const float4 v = *reinterpret_cast<const float4*>(sww + p * Tile::kWPlaneStride + row16);
+                wv[p * 4] = v.x; wv[p * 4 + 1] = v.y; wv[p * 4 + 2] = v.z; wv[p * 4 + 3] = v.w;
+            }
+            // lane j runs the chains for h = j (mod 32), ascending h
 #pragma unroll
             for (int i = 0; i < TR; ++i)
 #pragma unroll
                 for (int q = 0; q < ER; ++q) acc[i][q] = fmaf(xv[i], wv[q], acc[i][q]);
         }
+        if (st + 1 < nst) {
+            store_stage((st + 1) & 1);       // the buffer read at st - 1; every warp passed the barrier since
+            if (st + 2 < nst) load_stage(st + 2);
+        }
+        __syncthreads();
     }
-    cp_async_wait<0>();
 
 #pragma unroll
     for (int i = 0; i < TR; ++i) {
@@ -206,12 +264,15 @@ static cudaError_t launch_logits(const uint16_t* x, const float* Wg, const float
 cudaError_t launch_router_softmax(const uint16_t* x, const float* Wg, const float* bias, float* logits, int T, int H,
                                   int E, int k, int32_t* topk_idx, float* topk_w, int num_sms, cudaStream_t s) {
     cudaError_t err;
-    // large token x expert tiles when they still give a couple of waves, small ones otherwise
-    const long big_ctas = static_cast<long>((T + 31) / 32) * ((E + 31) / 32);
-    if (big_ctas >= 2L * num_sms)
-        err = launch_logits<8, 16, 4, 2>(x, Wg, bias, logits, T, H, E, s);
+    // the largest register tile whose CTAs still cover the GPU at least once
+    const long ctas_big = static_cast<long>((T + 31) / 32) * ((E + 31) / 32);
+    const long ctas_mid = static_cast<long>((T + 15) / 16) * ((E + 15) / 16);
+    if (ctas_big >= num_sms)
+        err = launch_logits<16, 8, 2, 4>(x, Wg, bias, logits, T, H, E, s);      // 32 tokens x 32 experts
+    else if (ctas_mid >= num_sms)
+        err = launch_logits<8, 4, 2, 4>(x, Wg, bias, logits, T, H, E, s);       // 16 tokens x 16 experts
     else
-        err = launch_logits<2, 4, 4, 2>(x, Wg, bias, logits, T, H, E, s);
+        err = launch_logits<8, 4, 1, 4>(x, Wg, bias, logits, T, H, E, s);       // 8 tokens x 16 experts
     if (err != cudaSuccess) return err;
     const int blocks = (T + 7) / 8;
     if (E <= 64)

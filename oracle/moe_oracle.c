@@ -291,37 +291,49 @@ typedef struct {
     const uint8_t *xq; const float* xs;
     const uint8_t *W1q, *W3q, *W2q; const float *S1, *S3, *S2;
     uint8_t* hq; float* hs; uint16_t* o;
+    float* h;          /* [n, I] fp32 h before its quantisation */
 } expert_ctx;
 
-static void expert_range(void* vctx, int64_t b, int64_t e) {
+/* Work items are (row, output column); the split is over items only, so
+ * every output is the same sum in the same order whatever the thread count. */
+static void expert_up_range(void* vctx, int64_t b, int64_t e) {
     expert_ctx* c = (expert_ctx*)vctx;
-    int H = c->H, I = c->I, n;
-    float* h = (float*)malloc(sizeof(float) * (size_t)I);
-    int64_t r;
-    for (r = b; r < e; ++r) {
+    int H = c->H, I = c->I;
+    int64_t it;
+    for (it = b; it < e; ++it) {
+        int64_t r = it / I;
+        int n = (int)(it % I);
         const uint8_t* xr = c->xq + r * H;
         const float* xsr = c->xs + r * (H / GROUP);
-        for (n = 0; n < I; ++n) {
-            double a = dot_row(H, xr, xsr, c->W1q + (int64_t)n * H, c->S1 + (int64_t)(n / GROUP) * (H / GROUP));
-            double bb = dot_row(H, xr, xsr, c->W3q + (int64_t)n * H, c->S3 + (int64_t)(n / GROUP) * (H / GROUP));
-            h[n] = (float)(silu(a) * bb);
-        }
-        orc_quant_rows(1, I, h, c->hq + r * I, c->hs + r * (I / GROUP));
-        for (n = 0; n < H; ++n) {
-            double o = dot_row(I, c->hq + r * I, c->hs + r * (I / GROUP),
-                               c->W2q + (int64_t)n * I, c->S2 + (int64_t)(n / GROUP) * (I / GROUP));
-            c->o[r * H + n] = orc_f64_to_bf16(o);
-        }
+        double a = dot_row(H, xr, xsr, c->W1q + (int64_t)n * H, c->S1 + (int64_t)(n / GROUP) * (H / GROUP));
+        double bb = dot_row(H, xr, xsr, c->W3q + (int64_t)n * H, c->S3 + (int64_t)(n / GROUP) * (H / GROUP));
+        c->h[r * I + n] = (float)(silu(a) * bb);
     }
-    free(h);
+}
+
+static void expert_down_range(void* vctx, int64_t b, int64_t e) {
+    expert_ctx* c = (expert_ctx*)vctx;
+    int H = c->H, I = c->I;
+    int64_t it;
+    for (it = b; it < e; ++it) {
+        int64_t r = it / H;
+        int n = (int)(it % H);
+        double o = dot_row(I, c->hq + r * I, c->hs + r * (I / GROUP),
+                           c->W2q + (int64_t)n * I, c->S2 + (int64_t)(n / GROUP) * (I / GROUP));
+        c->o[r * H + n] = orc_f64_to_bf16(o);
+    }
 }
 
 void orc_expert_rows(int n, int H, int I, const uint8_t* xq, const float* xs,
                      const uint8_t* W1q, const float* S1, const uint8_t* W3q, const float* S3,
                      const uint8_t* W2q, const float* S2,
                      uint8_t* hq, float* hs, uint16_t* o, int nthreads) {
-    expert_ctx c = {H, I, xq, xs, W1q, W3q, W2q, S1, S3, S2, hq, hs, o};
-    parallel_for(n, nthreads, expert_range, &c);
+    expert_ctx c = {H, I, xq, xs, W1q, W3q, W2q, S1, S3, S2, hq, hs, o, NULL};
+    c.h = (float*)malloc(sizeof(float) * (size_t)n * (size_t)I);
+    parallel_for((int64_t)n * I, nthreads, expert_up_range, &c);     /* a, b, h = silu(a) * b */
+    orc_quant_rows(n, I, c.h, hq, hs);                                /* h -> E4M3 + 1x128 scales */
+    parallel_for((int64_t)n * H, nthreads, expert_down_range, &c);    /* o = W2 h, -> bf16 */
+    free(c.h);
 }
 
 /* ------------------------------------------------------------------ */
