@@ -39,6 +39,9 @@ constexpr int kStagesC = 4;
 constexpr int kABytes = kBM * kBK;            // 16 KB
 constexpr int kBBytes = kBN * kBK;            // 32 KB
 constexpr int kThreadsC = 384;                // 12 warps
+// setmaxnreg split: 4 warps give registers up, 8 promotion warps take them.
+constexpr int kRegsLow = 56, kRegsHigh = 224;
+constexpr int kRegsSplit = 128 * kRegsLow + 256 * kRegsHigh;   // must fit the launch allocation
 constexpr int kDrainNs = 200000;              // settle time after an abort
 
 struct SmemC {
@@ -135,7 +138,7 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // Register split (launch: 384 threads x 168 = 64512): the TMA/MMA warpgroup gives up
     // registers to the two promotion warpgroups, 128 x 56 + 256 x 224 = 64512.
     if (warp < 4) {
-      setmaxnreg_dec<56>();
+      setmaxnreg_dec<kRegsLow>();
       if (warp == 0) {
         // ---------------- TMA producer
         if (lane == 0) {
@@ -184,7 +187,7 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
       }
     } else {
-        setmaxnreg_inc<224>();
+        setmaxnreg_inc<kRegsHigh>();
         // ---------------- promotion + epilogue (256 threads)
         const int q = warp & 3;                 // tensor-memory lane quadrant
         const int half = (warp - 4) >> 2;       // which 64 columns of each 128-column half
@@ -194,9 +197,11 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (sm.abort_flag) break;
             const TileC t = decode_tile_c(sm.P, E, NT, N, tile);
             const bool full = t.width == kBN;
-            float acc[128];
+            // acc2[i] holds columns (2i, 2i+1) of this thread's 128 (64 from each 128-column half)
+            float2 acc2[64];
 #pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
+            float* acc = reinterpret_cast<float*>(acc2);
             const float* bs0 = Bs + (static_cast<int64_t>(t.e) * NB + t.n0 / kBM) * KB;
             const float* bs1 = full ? bs0 + KB : bs0;
             const float* as_row = As + t.m0 + row;
@@ -224,10 +229,11 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     tmem_ld32(taddr, v0);
                     tmem_ld32(taddr + 32, v1);
                     tmem_ld_wait();
+                    const float2 f = make_float2(f0, f0);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        acc[i] = fmaf(v0[i], f0, acc[i]);
-                        acc[32 + i] = fmaf(v1[i], f0, acc[32 + i]);
+                    for (int i = 0; i < 16; ++i) {
+                        acc2[i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), f, acc2[i]);
+                        acc2[16 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), f, acc2[16 + i]);
                     }
                 }
                 if (full) {
@@ -235,10 +241,11 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     tmem_ld32(taddr + 128, v0);
                     tmem_ld32(taddr + 160, v1);
                     tmem_ld_wait();
+                    const float2 f = make_float2(f1, f1);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        acc[64 + i] = fmaf(v0[i], f1, acc[64 + i]);
-                        acc[96 + i] = fmaf(v1[i], f1, acc[96 + i]);
+                    for (int i = 0; i < 16; ++i) {
+                        acc2[32 + i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), f, acc2[32 + i]);
+                        acc2[48 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), f, acc2[48 + i]);
                     }
                 }
                 sa_0 = sa_1; w0_0 = w0_1; w1_0 = w1_1;
@@ -586,6 +593,17 @@ static cudaError_t set_smem(Kern k, size_t bytes) {
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
+// A setmaxnreg.inc can only draw on the registers the block was launched with; if the
+// compiled kernel's launch allocation were smaller than the split, the increase would
+// never be granted. Refuse to launch such a build instead of starting it.
+template <typename Kern>
+static cudaError_t check_reg_split(Kern k) {
+    cudaFuncAttributes a;
+    cudaError_t err = cudaFuncGetAttributes(&a, k);
+    if (err != cudaSuccess) return err;
+    return a.numRegs * kThreadsC >= kRegsSplit ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                                 const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs, int epilogue,
                                 void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s) {
@@ -596,11 +614,13 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
         const size_t smem = sizeof(SmemC) + 1024;
         if (epilogue == 0) {
             cudaError_t err = set_smem(gg_contig_kernel<0>, smem);
+            if (err == cudaSuccess) err = check_reg_split(gg_contig_kernel<0>);
             if (err != cudaSuccess) return err;
             gg_contig_kernel<0><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
                                                                   Ds, status, wait_ns);
         } else {
             cudaError_t err = set_smem(gg_contig_kernel<1>, smem);
+            if (err == cudaSuccess) err = check_reg_split(gg_contig_kernel<1>);
             if (err != cudaSuccess) return err;
             gg_contig_kernel<1><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
                                                                   Ds, status, wait_ns);

@@ -120,11 +120,13 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
         }
     };
 
-    float acc[TR][ER];
+    // acc[i][q] holds tokens (2i, 2i+1) of the warp's tile for expert q; the packed
+    // fused multiply-add rounds each half exactly like a scalar fmaf.
+    float2 acc[TR / 2][ER];
 #pragma unroll
-    for (int i = 0; i < TR; ++i)
+    for (int i = 0; i < TR / 2; ++i)
 #pragma unroll
-        for (int q = 0; q < ER; ++q) acc[i][q] = 0.0f;
+        for (int q = 0; q < ER; ++q) acc[i][q] = make_float2(0.0f, 0.0f);
 
     load_stage(0);
     store_stage(0);
@@ -137,16 +139,15 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
 #pragma unroll
         for (int s = 0; s < kRouterHS / 32; ++s) {
             const int row16 = swz_row(s * 32 + lane) * 16;
-            float xv[TR], wv[ER];
+            float2 xv[TR / 2];
+            float wv[ER];
 #pragma unroll
             for (int p = 0; p < TR / 8; ++p) {
                 const uint4 v = *reinterpret_cast<const uint4*>(sxw + p * kPlaneBytes + row16);
                 const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    xv[p * 8 + 2 * i] = __uint_as_float(u[i] << 16);
-                    xv[p * 8 + 2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
-                }
+                for (int i = 0; i < 4; ++i)
+                    xv[p * 4 + i] = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
             }
 #pragma unroll
             for (int p = 0; p < ER / 4; ++p) {
@@ -155,9 +156,11 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
             }
             // lane j runs the chains for h = j (mod 32), ascending h
 #pragma unroll
-            for (int i = 0; i < TR; ++i)
+            for (int q = 0; q < ER; ++q) {
+                const float2 w2 = make_float2(wv[q], wv[q]);
 #pragma unroll
-                for (int q = 0; q < ER; ++q) acc[i][q] = fmaf(xv[i], wv[q], acc[i][q]);
+                for (int i = 0; i < TR / 2; ++i) acc[i][q] = __ffma2_rn(xv[i], w2, acc[i][q]);
+            }
         }
         if (st + 1 < nst) {
             store_stage((st + 1) & 1);       // the buffer read at st - 1; every warp passed the barrier since
@@ -170,7 +173,7 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
     for (int i = 0; i < TR; ++i) {
 #pragma unroll
         for (int q = 0; q < ER; ++q) {
-            float v = acc[i][q];
+            float v = (i & 1) ? acc[i >> 1][q].y : acc[i >> 1][q].x;
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
             const int t = t_base + wt * TR + i, e = e_base + we * ER + q;
