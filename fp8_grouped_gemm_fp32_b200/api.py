@@ -29,7 +29,8 @@ ROUTE_SOFTMAX_TOPK, ROUTE_HASH = 0, 1
 LAYOUT_CONTIGUOUS, LAYOUT_MASKED = 0, 1
 EPI_BF16, EPI_SWIGLU_FP8 = 0, 1
 EXPORTS = ("moe_rows_capacity", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_gemm_fp8",
-           "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string")
+           "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string",
+           "moe_permute_noalloc")
 
 
 class MoeError(RuntimeError):
@@ -68,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_size.restype = SZ
         L.moe_route.argtypes = [CP, P, P, P, P, P, P, P, SZ, P]
         L.moe_permute.argtypes = [CP, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_permute_noalloc.argtypes = [CP, P, P, P, P, P, P, P, P, P, P]
         L.moe_grouped_gemm_fp8.argtypes = [I, I, I, I, P, P, P, I, P, P, I, P, P, P]
         L.moe_combine.argtypes = [CP, P, P, P, P, P]
         L.moe_forward.argtypes = [CP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -127,6 +129,13 @@ def moe_permute(cfg, x, topk_idx, Aq, As, counts, kept, offsets, row_src, slot_r
     _check(lib().moe_permute(ctypes.byref(cfg), _p(x), _p(topk_idx), _p(Aq), _p(As), _p(counts), _p(kept),
                              _p(offsets), _p(row_src), _p(slot_row), _p(ws), ws.numel() * ws.element_size(),
                              _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(cfg, x, topk_idx, Aq, As, counts, kept, offsets, row_src, slot_row, stream=None):
+    """moe_permute without a workspace: for callers that may not allocate device memory.
+    Uses the library's fixed device scratch; calls that overlap on the GPU race."""
+    _check(lib().moe_permute_noalloc(ctypes.byref(cfg), _p(x), _p(topk_idx), _p(Aq), _p(As), _p(counts), _p(kept),
+                                     _p(offsets), _p(row_src), _p(slot_row), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_grouped_gemm_fp8(layout, E, N, K, A, As, group_info, M_rows, B, Bs, epilogue, D, Ds=None, stream=None):

@@ -145,6 +145,13 @@ FwdWs carve(const moe_config_t* c, void* base) {
 inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 }  // namespace
+
+// The current device's status word (for moe_permute_noalloc in its own file); nullptr if unavailable.
+int* device_status_word() {
+    DeviceInfo* dev;
+    return device_info(&dev) == MOE_OK ? dev->status : nullptr;
+}
+
 }  // namespace moe
 
 using namespace moe;

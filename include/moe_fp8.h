@@ -193,6 +193,29 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
                          const uint8_t* W2, const float* S2, void* y, int32_t* topk_idx, float* topk_w,
                          int32_t* counts, int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Permutation without a workspace, for callers that may not allocate device
+ * memory (code running during CUDA graph capture, servers that fix their
+ * memory budget up front and forbid cudaMalloc on the request path, plugin
+ * hosts whose memory belongs to another allocator). The source pages have no
+ * counterpart: it computes exactly what moe_permute computes, with the same
+ * kernels and the same arguments minus ws / ws_bytes.
+ * Its scratch is a fixed array of MOE_PERMUTE_NOALLOC_MAX_SCRATCH_BYTES in the
+ * library's own device memory, which every GPU that loads the library holds
+ * until the process exits. The call needs 8 * ceil(T / 32) * E bytes of it
+ * (e.g. T = 16384 with E = 512, or T = 32768 with E = 256) and returns
+ * MOE_ERR_UNSUPPORTED_SHAPE, launching nothing, when that exceeds the array.
+ * The first call on each device looks the array's device address up (a
+ * runtime call), so make that first call before any stream capture. Every
+ * call shares the one array: calls whose kernels overlap on the GPU (other
+ * streams, other host threads) race and corrupt each other's results; order
+ * them on one stream. It allocates nothing and calls no allocating routine.
+ */
+#define MOE_PERMUTE_NOALLOC_MAX_SCRATCH_BYTES (2u * 1024u * 1024u)
+moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                                 uint8_t* Aq, float* As, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                 int32_t* row_src, int32_t* slot_row, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: MOE_OK, MOE_ERR_CAPACITY or MOE_ERR_DEVICE_TIMEOUT. */
 moe_status_t moe_get_device_status(void* stream);
