@@ -262,15 +262,15 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 for (int r = 0; r < 2; ++r) {
                     if (r == 1 && !full) break;
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        uint32_t u[4];
+                    for (int v = 0; v < 4; ++v) {
+                        uint32_t u[8];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
+                        for (int i = 0; i < 8; ++i) {
                             const __nv_bfloat162 b =
-                                __floats2bfloat162_rn(acc[r * 64 + v * 8 + 2 * i], acc[r * 64 + v * 8 + 2 * i + 1]);
+                                __floats2bfloat162_rn(acc[r * 64 + v * 16 + 2 * i], acc[r * 64 + v * 16 + 2 * i + 1]);
                             u[i] = *reinterpret_cast<const uint32_t*>(&b);
                         }
-                        *reinterpret_cast<uint4*>(out + r * 128 + v * 8) = make_uint4(u[0], u[1], u[2], u[3]);
+                        st_global_v8(out + r * 128 + v * 16, u);   // one full 32-byte sector per thread
                     }
                 }
             } else {
@@ -289,20 +289,20 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 ++ep;
                 amax = fmaxf(sm.red[p][0][row], sm.red[p][1][row]);
                 const float s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+                // h / s as h * (1 / s): the correctly rounded reciprocal keeps the quotient within one
+                // ulp of the division, below the resolution of the E4M3 code it is rounded to
+                const float rs = amax == 0.0f ? 1.0f : __frcp_rn(s);
                 uint8_t* hq = static_cast<uint8_t*>(D) + grow * I + t.n0 / 2 + half * 64;
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    uint32_t u[4];
+                for (int v = 0; v < 2; ++v) {
+                    uint32_t u[8];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int c = v * 16 + i * 4;
-                        const float d0 = amax == 0.0f ? acc[c] : __fdiv_rn(acc[c], s);
-                        const float d1 = amax == 0.0f ? acc[c + 1] : __fdiv_rn(acc[c + 1], s);
-                        const float d2 = amax == 0.0f ? acc[c + 2] : __fdiv_rn(acc[c + 2], s);
-                        const float d3 = amax == 0.0f ? acc[c + 3] : __fdiv_rn(acc[c + 3], s);
-                        u[i] = f32x2_to_e4m3x2(d0, d1) | (static_cast<uint32_t>(f32x2_to_e4m3x2(d2, d3)) << 16);
+                    for (int i = 0; i < 8; ++i) {
+                        const int c = v * 32 + i * 4;
+                        u[i] = f32x2_to_e4m3x2(acc[c] * rs, acc[c + 1] * rs) |
+                               (static_cast<uint32_t>(f32x2_to_e4m3x2(acc[c + 2] * rs, acc[c + 3] * rs)) << 16);
                     }
-                    *reinterpret_cast<uint4*>(hq + v * 16) = make_uint4(u[0], u[1], u[2], u[3]);
+                    st_global_v8(hq + v * 32, u);
                 }
                 if (half == 0) Ds[static_cast<int64_t>(t.n0 / kBN) * M_rows + grow] = s;
             }
