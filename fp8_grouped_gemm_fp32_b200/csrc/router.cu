@@ -120,13 +120,11 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
         }
     };
 
-    // acc[i][q] holds tokens (2i, 2i+1) of the warp's tile for expert q; the packed
-    // fused multiply-add rounds each half exactly like a scalar fmaf.
-    float2 acc[TR / 2][ER];
+    float acc[TR][ER];
 #pragma unroll
-    for (int i = 0; i < TR / 2; ++i)
+    for (int i = 0; i < TR; ++i)
 #pragma unroll
-        for (int q = 0; q < ER; ++q) acc[i][q] = make_float2(0.0f, 0.0f);
+        for (int q = 0; q < ER; ++q) acc[i][q] = 0.0f;
 
     load_stage(0);
     store_stage(0);
@@ -156,11 +154,12 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
             }
             // lane j runs the chains for h = j (mod 32), ascending h
 #pragma unroll
-            for (int q = 0; q < ER; ++q) {
-                const float2 w2 = make_float2(wv[q], wv[q]);
+            for (int i = 0; i < TR / 2; ++i)
 #pragma unroll
-                for (int i = 0; i < TR / 2; ++i) acc[i][q] = __ffma2_rn(xv[i], w2, acc[i][q]);
-            }
+                for (int q = 0; q < ER; ++q) {
+                    acc[2 * i][q] = fmaf(xv[i].x, wv[q], acc[2 * i][q]);
+                    acc[2 * i + 1][q] = fmaf(xv[i].y, wv[q], acc[2 * i + 1][q]);
+                }
         }
         if (st + 1 < nst) {
             store_stage((st + 1) & 1);       // the buffer read at st - 1; every warp passed the barrier since
@@ -173,7 +172,7 @@ router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W
     for (int i = 0; i < TR; ++i) {
 #pragma unroll
         for (int q = 0; q < ER; ++q) {
-            float v = (i & 1) ? acc[i >> 1][q].y : acc[i >> 1][q].x;
+            float v = acc[i][q];
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
             const int t = t_base + wt * TR + i, e = e_base + we * ER + q;
