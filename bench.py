@@ -47,6 +47,32 @@ def describe(cfg: MoeConfig) -> str:
     return s + f" bias={cfg.bias} seed={cfg.seed}"
 
 
+KERNEL_SOURCES = {"gemm_up": "grouped_gemm.cu", "gemm_down": "grouped_gemm.cu", "router": "router.cu",
+                  "permute": "permute.cu", "combine": "combine.cu"}
+
+
+def source_hash(step: str) -> str:
+    import hashlib
+    path = os.path.join(ROOT, "fp8_grouped_gemm_fp32_b200", "csrc", KERNEL_SOURCES[step])
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(step: str, workload: str):
+    """DRAM bytes per launch (read + write) of a step's kernel from profiles/dram_traffic.txt,
+    a summary of one ncu capture; only valid while the kernel's source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = source_hash(step)
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and not line.startswith("#") and parts[0] == step and parts[1] == workload:
+                return float(parts[3]) if parts[2] == want else None
+    return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -350,7 +376,8 @@ def run_ours(args):
         roof = {"bound": "hbm", "achieved": w["bytes"] / t_s / 1e9, "peak": hbm, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = dom
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(dom, cfg.name)
+    roof["algorithmic_bytes"] = w["bytes"]
     roof["peak_source"] = (f"{peak_src}: " + ("FP8 = 2 x sustained bf16 cuBLAS (nominal FP8:BF16 ratio)"
                                               if roof["bound"] == "tensor" else "HBM copy"))
     gemm_ms = per["gemm_up"] + per["gemm_down"]

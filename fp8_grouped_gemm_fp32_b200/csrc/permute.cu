@@ -195,35 +195,62 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
     }
     __syncthreads();
 
-    // quantise (token r of the chunk, group g): one warp per item, 4 values per lane
-    const int items = kChunk * (g1 - g0);
-    for (int it = warp; it < items; it += 8) {
-        const int r = it / (g1 - g0), g = g0 + it % (g1 - g0);
-        const int t = c * kChunk + r;
-        if (t >= T) continue;
-        const uint2 raw = *reinterpret_cast<const uint2*>(x + static_cast<int64_t>(t) * H + g * kGroup + lane * 4);
-        const float v0 = __uint_as_float(raw.x << 16), v1 = __uint_as_float(raw.x & 0xffff0000u);
-        const float v2 = __uint_as_float(raw.y << 16), v3 = __uint_as_float(raw.y & 0xffff0000u);
-        const float amax = warp_max(fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
-        float s = 1.0f;
-        uint32_t packed;
-        if (amax == 0.0f) {
-            packed = f32x2_to_e4m3x2(v0, v1) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v2, v3)) << 16);
-        } else {
-            s = __fdiv_rn(amax, 448.0f);
-            packed = f32x2_to_e4m3x2(__fdiv_rn(v0, s), __fdiv_rn(v1, s)) |
-                     (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(v2, s), __fdiv_rn(v3, s))) << 16);
+    // quantise (token r of the chunk, group g): a warp takes 4 items at a time so their loads and
+    // reductions overlap; 4 values per lane per item
+    constexpr int U = 4;
+    const int gs = g1 - g0;
+    const int items = kChunk * gs;
+    for (int base = warp * U; base < items; base += 8 * U) {
+        uint2 raw[U];
+        int tok_r[U], grp[U];
+        bool live[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int it = base + u;
+            tok_r[u] = it / gs;
+            grp[u] = g0 + it % gs;
+            const int t = c * kChunk + tok_r[u];
+            live[u] = it < items && t < T;
+            raw[u] = live[u] ? *reinterpret_cast<const uint2*>(x + static_cast<int64_t>(t) * H + grp[u] * kGroup + lane * 4)
+                             : make_uint2(0, 0);
         }
-        for (int j = 0; j < k; ++j) {
-            const int32_t row = dest[r * k + j];
-            if (row < 0) continue;
-            *reinterpret_cast<uint32_t*>(Aq + static_cast<int64_t>(row) * H + g * kGroup + lane * 4) = packed;
-            if (lane == 0) {
-                if (masked) {
-                    const int e = row / masked_max_m, rr = row - e * masked_max_m;
-                    As[(static_cast<int64_t>(e) * G + g) * masked_max_m + rr] = s;
-                } else {
-                    As[static_cast<int64_t>(g) * ld_rows + row] = s;
+        float v[U][4], amax[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            v[u][0] = __uint_as_float(raw[u].x << 16);
+            v[u][1] = __uint_as_float(raw[u].x & 0xffff0000u);
+            v[u][2] = __uint_as_float(raw[u].y << 16);
+            v[u][3] = __uint_as_float(raw[u].y & 0xffff0000u);
+            amax[u] = fmaxf(fmaxf(fabsf(v[u][0]), fabsf(v[u][1])), fmaxf(fabsf(v[u][2]), fabsf(v[u][3])));
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < U; ++u) amax[u] = fmaxf(amax[u], __shfl_xor_sync(0xffffffffu, amax[u], o));
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (!live[u]) continue;
+            float sc = 1.0f;
+            uint32_t packed;
+            if (amax[u] == 0.0f) {
+                packed = f32x2_to_e4m3x2(v[u][0], v[u][1]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[u][2], v[u][3])) << 16);
+            } else {
+                sc = __fdiv_rn(amax[u], 448.0f);
+                packed = f32x2_to_e4m3x2(__fdiv_rn(v[u][0], sc), __fdiv_rn(v[u][1], sc)) |
+                         (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(v[u][2], sc), __fdiv_rn(v[u][3], sc))) << 16);
+            }
+            const int r = tok_r[u], g = grp[u];
+            for (int j = 0; j < k; ++j) {
+                const int32_t row = dest[r * k + j];
+                if (row < 0) continue;
+                *reinterpret_cast<uint32_t*>(Aq + static_cast<int64_t>(row) * H + g * kGroup + lane * 4) = packed;
+                if (lane == 0) {
+                    if (masked) {
+                        const int e = row / masked_max_m, rr = row - e * masked_max_m;
+                        As[(static_cast<int64_t>(e) * G + g) * masked_max_m + rr] = sc;
+                    } else {
+                        As[static_cast<int64_t>(g) * ld_rows + row] = sc;
+                    }
                 }
             }
         }
