@@ -332,13 +332,14 @@ struct SmemM {
     static constexpr int kW = EPI == 1 ? 2 * kWBlk : kWBlk;    // weight rows per stage: 256 (a|b) or 128
     static constexpr int kStages = EPI == 1 ? 4 : 8;
     static constexpr int kCols = EPI == 1 ? 2 * kBT : kBT;     // tensor-memory columns per buffer
+    static constexpr int kBufs = 4;                            // MMA runs up to 3 K blocks ahead of promotion
     uint8_t w[kStages][kW];
     uint8_t x[kStages][kXBytes];
     float hs[2][kBT][kBM];                                      // SwiGLU output staged for the requant
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t tfull[kBufs];
+    uint64_t tempty[kBufs];
     uint64_t red_bar[2];
     uint32_t tmem_base;
     volatile int abort_flag;
@@ -358,7 +359,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     const int KB = K / kBK;
     const int NB = N / kBM;                          // 128-row weight blocks per expert
     const int NBt = EPI == 1 ? NB / 2 : NB;          // weight tiles per expert
-    constexpr uint32_t kTmemCols = EPI == 1 ? 128 : 64;
+    constexpr uint32_t kTmemCols = S::kBufs * S::kCols;        // 256 (SwiGLU) or 128 columns
 
     if (warp == 0) {
         // tile prefix over experts: tiles_e = NBt * ceil(m_e / 32)
@@ -381,11 +382,11 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < S::kBufs; ++b) {
             mbar_init(&sm.tfull[b], 1);
             mbar_init(&sm.tempty[b], 4);
-            mbar_init(&sm.red_bar[b], 128);
         }
+        for (int b = 0; b < 2; ++b) mbar_init(&sm.red_bar[b], 128);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -440,8 +441,8 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 for (int kb = 0; kb < KB; ++kb, ++it, ++kbt) {
                     const int s = it % S::kStages;
                     const uint32_t ph = (it / S::kStages) & 1;
-                    const int buf = kbt & 1;
-                    const uint32_t bph = (kbt >> 1) & 1;
+                    const int buf = kbt % S::kBufs;
+                    const uint32_t bph = (kbt / S::kBufs) & 1;
                     if (!mbar_wait(&sm.full[s], ph, wait_ns)) { fail(); break; }
                     if (!mbar_wait(&sm.tempty[buf], bph ^ 1, wait_ns)) { fail(); break; }
                     tc_fence_after();
@@ -475,19 +476,28 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const float* bsa = Bs + (static_cast<int64_t>(e) * NB + blk_a) * KB;
             const float* bsb = bsa + KB;
             bool ok = true;
+            // the token tile's scales for K block kb + 1 load while block kb is promoted
+            const float4* sa_base = reinterpret_cast<const float4*>(As + static_cast<int64_t>(e) * KB * Mmax + tt * kBT);
+            float4 nxt[kBT / 4];
+#pragma unroll
+            for (int i = 0; i < kBT / 4; ++i) nxt[i] = sa_base[i];
+            float nxt_wa = bsa[0], nxt_wb = EPI == 1 ? bsb[0] : 0.0f;
             for (int kb = 0; kb < KB; ++kb, ++kbt) {
-                const int buf = kbt & 1;
-                const uint32_t bph = (kbt >> 1) & 1;
-                const float4* sa4 =
-                    reinterpret_cast<const float4*>(As + (static_cast<int64_t>(e) * KB + kb) * Mmax + tt * kBT);
+                const int buf = kbt % S::kBufs;
+                const uint32_t bph = (kbt / S::kBufs) & 1;
                 float sa[kBT];
 #pragma unroll
                 for (int i = 0; i < kBT / 4; ++i) {
-                    const float4 v = sa4[i];
-                    sa[4 * i] = v.x; sa[4 * i + 1] = v.y; sa[4 * i + 2] = v.z; sa[4 * i + 3] = v.w;
+                    sa[4 * i] = nxt[i].x; sa[4 * i + 1] = nxt[i].y; sa[4 * i + 2] = nxt[i].z; sa[4 * i + 3] = nxt[i].w;
                 }
-                const float swa = bsa[kb];
-                const float swb = EPI == 1 ? bsb[kb] : 0.0f;
+                const float swa = nxt_wa, swb = nxt_wb;
+                if (kb + 1 < KB) {
+                    const float4* p4 = sa_base + static_cast<int64_t>(kb + 1) * (Mmax / 4);
+#pragma unroll
+                    for (int i = 0; i < kBT / 4; ++i) nxt[i] = p4[i];
+                    nxt_wa = bsa[kb + 1];
+                    if (EPI == 1) nxt_wb = bsb[kb + 1];
+                }
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * S::kCols;
