@@ -218,7 +218,9 @@ moe_status_t moe_grouped_gemm_fp8(int layout, int E, int N, int K, const uint8_t
     if (E <= 0 || N <= 0 || K <= 0 || M_rows <= 0) return MOE_ERR_INVALID_ARG;
     if (E > MOE_MAX_EXPERTS || N % kGroup || K % kGroup) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (epilogue == MOE_EPI_SWIGLU_FP8 && N % (2 * kGroup)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (K > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (layout == MOE_LAYOUT_MASKED && M_rows % 32) return MOE_ERR_INVALID_ARG;
+    if (layout == MOE_LAYOUT_CONTIGUOUS && M_rows % 4) return MOE_ERR_INVALID_ARG;
     if (static_cast<int64_t>(E) * N >= (1ll << 31) || static_cast<int64_t>(E) * M_rows >= (1ll << 31))
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!ptr_ok(A) || !ptr_ok(As) || !ptr_ok(group_info) || !ptr_ok(B) || !ptr_ok(Bs) || !ptr_ok(D))

@@ -36,6 +36,8 @@ namespace moe {
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;
 constexpr int kStagesC = 4;
+constexpr int kSaSlots = 8;                   // ring of per-K-block activation scales (128 rows each)
+constexpr int kMaxKB = 128;                   // K <= 16384: weight scales of a tile fit 4 registers per lane
 constexpr int kABytes = kBM * kBK;            // 16 KB
 constexpr int kBBytes = kBN * kBK;            // 32 KB
 constexpr int kThreadsC = 384;                // 12 warps
@@ -47,8 +49,11 @@ constexpr int kDrainNs = 200000;              // settle time after an abort
 struct SmemC {
     uint8_t a[kStagesC][kABytes];
     uint8_t b[kStagesC][kBBytes];
+    float sa[kSaSlots][kBM];    // activation scales of one K block for the tile's 128 rows
     uint64_t full[kStagesC];
     uint64_t empty[kStagesC];
+    uint64_t sfull[kSaSlots];
+    uint64_t sempty[kSaSlots];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t red_bar[2];
@@ -111,6 +116,10 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
+        for (int j = 0; j < kSaSlots; ++j) {
+            mbar_init(&sm.sfull[j], 1);
+            mbar_init(&sm.sempty[j], 8);
+        }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.tfull[b], 1);
             mbar_init(&sm.tempty[b], 8);
@@ -157,6 +166,12 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     tma_load_2d(sm.b[s], &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0);
                     if (t.width == kBN)
                         tma_load_2d(sm.b[s] + kBBytes / 2, &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0 + 128);
+                    // the 128 activation scales of this K block, into the scale ring
+                    const int j = it % kSaSlots;
+                    if (!mbar_wait(&sm.sempty[j], ((it / kSaSlots) & 1) ^ 1, wait_ns)) { fail(); break; }
+                    mbar_arrive_expect_tx(&sm.sfull[j], kBM * sizeof(float));
+                    bulk_load(sm.sa[j], As + static_cast<int64_t>(kb) * M_rows + t.m0, kBM * sizeof(float),
+                              &sm.sfull[j]);
                 }
             }
         }
@@ -193,6 +208,22 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int half = (warp - 4) >> 2;       // which 64 columns of each 128-column half
         const int row = q * 32 + lane;          // row within the tile
         uint32_t kbt = 0, ep = 0;
+        // lane l holds the weight-block scales of K blocks l, l + 32, l + 64, l + 96 of the tile's
+        // (up to) two 128-row weight blocks; loaded one tile ahead, so their latency hides behind a tile
+        float wb0[4], wb1[4];
+        auto load_wb = [&](int tile) {
+            if (tile >= total) return;
+            const TileC u = decode_tile_c(sm.P, E, NT, N, tile);
+            const float* b0 = Bs + (static_cast<int64_t>(u.e) * NB + u.n0 / kBM) * KB;
+            const float* b1 = u.width == kBN ? b0 + KB : b0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int kb = lane + 32 * i;
+                wb0[i] = kb < KB ? b0[kb] : 0.0f;
+                wb1[i] = kb < KB ? b1[kb] : 0.0f;
+            }
+        };
+        load_wb(blockIdx.x);
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             if (sm.abort_flag) break;
             const TileC t = decode_tile_c(sm.P, E, NT, N, tile);
@@ -202,25 +233,24 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
             float* acc = reinterpret_cast<float*>(acc2);
-            const float* bs0 = Bs + (static_cast<int64_t>(t.e) * NB + t.n0 / kBM) * KB;
-            const float* bs1 = full ? bs0 + KB : bs0;
-            const float* as_row = As + t.m0 + row;
-            // scales run two K blocks ahead of their use, so their L2 latency overlaps the MMAs
-            float sa_0 = as_row[0], w0_0 = bs0[0], w1_0 = bs1[0];
-            float sa_1 = 0.f, w0_1 = 0.f, w1_1 = 0.f;
-            if (KB > 1) { sa_1 = as_row[M_rows]; w0_1 = bs0[1]; w1_1 = bs1[1]; }
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb, ++kbt) {
                 const int buf = kbt & 1;
                 const uint32_t bph = (kbt >> 1) & 1;
-                float sa_2 = 0.f, w0_2 = 0.f, w1_2 = 0.f;
-                if (kb + 2 < KB) {
-                    sa_2 = as_row[static_cast<int64_t>(kb + 2) * M_rows];
-                    w0_2 = bs0[kb + 2];
-                    w1_2 = bs1[kb + 2];
-                }
-                const float f0 = sa_0 * w0_0;
-                const float f1 = sa_0 * w1_0;
+                // scales: sa from the ring (the producer copied it several K blocks ago), the weight
+                // block scales from the registers of the lane that holds them
+                const int j = kbt % kSaSlots;
+                if (!mbar_wait(&sm.sfull[j], (kbt / kSaSlots) & 1, wait_ns)) { fail(); ok = false; break; }
+                const float sa = sm.sa[j][row];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.sempty[j]);
+                const int wi = kb >> 5;
+                const float w0 = __shfl_sync(0xffffffffu, wi == 0 ? wb0[0] : wi == 1 ? wb0[1] : wi == 2 ? wb0[2] : wb0[3],
+                                             kb & 31);
+                const float w1 = __shfl_sync(0xffffffffu, wi == 0 ? wb1[0] : wi == 1 ? wb1[1] : wi == 2 ? wb1[2] : wb1[3],
+                                             kb & 31);
+                const float f0 = sa * w0;
+                const float f1 = sa * w1;
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kBN + half * 64;
@@ -248,13 +278,12 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         acc2[48 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), f, acc2[48 + i]);
                     }
                 }
-                sa_0 = sa_1; w0_0 = w0_1; w1_0 = w1_1;
-                sa_1 = sa_2; w0_1 = w0_2; w1_1 = w1_2;
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.tempty[buf]);
             }
             if (!ok) break;
+            load_wb(tile + gridDim.x);
             const int64_t grow = t.m0 + row;
             if constexpr (EPI == 0) {
                 uint16_t* out = static_cast<uint16_t*>(D) + grow * N + t.n0 + half * 64;

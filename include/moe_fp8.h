@@ -159,7 +159,10 @@ moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* 
  *               W1 block j, W3 block j; h = silu(a) * b in fp32 is quantised
  *               per 1x128 group: D = u8 [rows, I], Ds = fp32 [I/128][M_rows]
  *               (masked: [E][I/128][M_rows]), the A/As layout of the next GEMM.
- * N and K must be multiples of 128 (256 for N with the SwiGLU epilogue).
+ * N and K must be multiples of 128 (256 for N with the SwiGLU epilogue) and
+ * K at most 16384 (MOE_ERR_UNSUPPORTED_SHAPE otherwise). Contiguous layout:
+ * M_rows must be a multiple of 4, so that each K block's row of As starts on
+ * a 16-byte boundary (MOE_ERR_INVALID_ARG otherwise).
  * Contiguous rows outside [0, offsets[E]) and masked rows at or past
  * masked_m[e] are neither read into any stored result nor written.
  */

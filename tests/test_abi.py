@@ -63,6 +63,20 @@ def test_bad_config_rejected_before_any_device_work(L, field, value, code):
     assert st == code
 
 
+@pytest.mark.parametrize("layout,N,K,M_rows,epi,code", [
+    (0, 200, 256, 128, 0, api.MOE_ERR_UNSUPPORTED_SHAPE),      # N not a multiple of 128
+    (0, 384, 256, 128, 1, api.MOE_ERR_UNSUPPORTED_SHAPE),      # SwiGLU needs N a multiple of 256
+    (0, 256, 16512, 128, 0, api.MOE_ERR_UNSUPPORTED_SHAPE),    # K above 16384
+    (0, 256, 256, 130, 0, api.MOE_ERR_INVALID_ARG),            # contiguous M_rows not a multiple of 4
+    (1, 256, 256, 48, 0, api.MOE_ERR_INVALID_ARG),             # masked M_rows not a multiple of 32
+    (2, 256, 256, 128, 0, api.MOE_ERR_INVALID_ARG),            # unknown layout
+])
+def test_bad_gemm_shape_rejected_before_any_device_work(L, layout, N, K, M_rows, epi, code):
+    p = ctypes.c_void_p(4096)                  # aligned, never dereferenced: the call returns first
+    st = L.moe_grouped_gemm_fp8(layout, 4, N, K, p, p, p, M_rows, p, p, epi, p, p, None)
+    assert st == code
+
+
 def test_hash_routing_needs_k1_and_masked_needs_rows(L):
     c = api.Config.from_moe(CONFIGS["decode_hash"])
     c.k = 2

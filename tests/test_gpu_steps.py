@@ -168,6 +168,8 @@ GEMM_CASES = [
     (0, 0, 5, 640, 384, [0, 1, 130, 255, 40], None),      # half-width last N tile (640 = 2*256 + 128)
     (0, 1, 5, 512, 384, [0, 1, 130, 255, 40], None),
     (0, 0, 3, 256, 1024, [300, 0, 129], None),
+    (0, 1, 3, 768, 640, [257, 384, 0], None),             # 3 M tiles per expert, 5 K blocks
+    (0, 0, 6, 384, 128, [1, 128, 129, 0, 513, 2], None),  # a single K block
     (1, 0, 4, 384, 256, [0, 5, 33, 64], 64),
     (1, 1, 4, 512, 256, [0, 5, 33, 64], 64),
     (1, 1, 3, 256, 512, [32, 1, 0], 96),
