@@ -35,23 +35,31 @@
 namespace moe {
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;
-constexpr int kStagesC = 4;
 constexpr int kSaSlots = 8;                   // ring of per-K-block activation scales (128 rows each)
-constexpr int kMaxKB = 128;                   // K <= 16384: weight scales of a tile fit 4 registers per lane
 constexpr int kABytes = kBM * kBK;            // 16 KB
 constexpr int kBBytes = kBN * kBK;            // 32 KB
 constexpr int kThreadsC = 384;                // 12 warps
 // setmaxnreg split: 4 warps give registers up, 8 promotion warps take them.
-constexpr int kRegsLow = 56, kRegsHigh = 224;
+constexpr int kRegsLow = 40, kRegsHigh = 232;
 constexpr int kRegsSplit = 128 * kRegsLow + 256 * kRegsHigh;   // must fit the launch allocation
 constexpr int kDrainNs = 200000;              // settle time after an abort
 
+// bf16 output (EPI 0) leaves through shared memory and TMA stores: each promotion warp stages
+// its 32 rows x 128 columns as four 32 x 32 boxes (64-byte rows, 64-byte swizzle); one fewer
+// operand stage makes room for them.
+constexpr int kOutBox = 32;
+constexpr int kOutBoxBytes = kOutBox * kOutBox * 2;            // 2 KB
+constexpr int kOutStageBytes = 8 * 4 * kOutBoxBytes;           // 64 KB
+
+template <int EPI>
 struct SmemC {
-    uint8_t a[kStagesC][kABytes];
-    uint8_t b[kStagesC][kBBytes];
+    static constexpr int kStages = EPI == 0 ? 3 : 4;
+    uint8_t a[kStages][kABytes];
+    uint8_t b[kStages][kBBytes];
+    uint8_t out[EPI == 0 ? kOutStageBytes : 16];
     float sa[kSaSlots][kBM];    // activation scales of one K block for the tile's 128 rows
-    uint64_t full[kStagesC];
-    uint64_t empty[kStagesC];
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
     uint64_t sfull[kSaSlots];
     uint64_t sempty[kSaSlots];
     uint64_t tfull[2];
@@ -99,11 +107,13 @@ __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + _
 template <int EPI>
 __global__ void __launch_bounds__(kThreadsC, 1)
 gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const float* __restrict__ As, const int32_t* __restrict__ offsets, int M_rows,
+                 const __grid_constant__ CUtensorMap tmD, const float* __restrict__ As, const int32_t* __restrict__ offsets, int M_rows,
                  const float* __restrict__ Bs, int E, int N, int K, void* __restrict__ D, float* __restrict__ Ds,
                  int* status, uint64_t wait_ns) {
     extern __shared__ uint8_t smem_raw[];
-    SmemC& sm = *reinterpret_cast<SmemC*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    using SC = SmemC<EPI>;
+    constexpr int kStagesC = SC::kStages;
+    SC& sm = *reinterpret_cast<SC*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = K / kBK;
     const int NB = N / kBM;                 // 128-wide weight blocks along N
@@ -145,7 +155,7 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     };
 
     // Register split (launch: 384 threads x 168 = 64512): the TMA/MMA warpgroup gives up
-    // registers to the two promotion warpgroups, 128 x 56 + 256 x 224 = 64512.
+    // registers to the two promotion warpgroups, 128 x 40 + 256 x 232 = 64512.
     if (warp < 4) {
       setmaxnreg_dec<kRegsLow>();
       if (warp == 0) {
@@ -254,53 +264,78 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kBN + half * 64;
-                {
-                    float v0[32], v1[32];
-                    tmem_ld32(taddr, v0);
-                    tmem_ld32(taddr + 32, v1);
-                    tmem_ld_wait();
-                    const float2 f = make_float2(f0, f0);
+                // The buffer is handed back to the MMA warp as soon as the last of its columns is in
+                // registers; the multiply-adds of the second weight block run after the release.
+                auto release = [&]() {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+                };
+                auto fold = [&](float2* dst, const float (&v)[32], float f) {
+                    const float2 ff = make_float2(f, f);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        acc2[i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), f, acc2[i]);
-                        acc2[16 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), f, acc2[16 + i]);
-                    }
-                }
+                    for (int i = 0; i < 16; ++i) dst[i] = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), ff, dst[i]);
+                };
+                float va[32], vb[32];
+                tmem_ld32(taddr, va);
+                tmem_ld32(taddr + 32, vb);
+                tmem_ld_wait();
                 if (full) {
-                    float v0[32], v1[32];
-                    tmem_ld32(taddr + 128, v0);
-                    tmem_ld32(taddr + 160, v1);
+                    fold(acc2, va, f0);
+                    tmem_ld32(taddr + 128, va);
+                    fold(acc2 + 16, vb, f0);
+                    tmem_ld32(taddr + 160, vb);
                     tmem_ld_wait();
-                    const float2 f = make_float2(f1, f1);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        acc2[32 + i] = __ffma2_rn(make_float2(v0[2 * i], v0[2 * i + 1]), f, acc2[32 + i]);
-                        acc2[48 + i] = __ffma2_rn(make_float2(v1[2 * i], v1[2 * i + 1]), f, acc2[48 + i]);
-                    }
+                    release();
+                    fold(acc2 + 32, va, f1);
+                    fold(acc2 + 48, vb, f1);
+                } else {
+                    release();
+                    fold(acc2, va, f0);
+                    fold(acc2 + 16, vb, f0);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.tempty[buf]);
             }
             if (!ok) break;
             load_wb(tile + gridDim.x);
             const int64_t grow = t.m0 + row;
             if constexpr (EPI == 0) {
-                uint16_t* out = static_cast<uint16_t*>(D) + grow * N + t.n0 + half * 64;
+                // this warp's 32 rows x 128 columns as four 32 x 32 boxes: box (r, c) holds columns
+                // n0 + r * 128 + half * 64 + c * 32 + [0, 32); 16-byte pieces are placed with the
+                // 64-byte swizzle (piece p of row l at p ^ ((l >> 1) & 3)), which the store undoes
+                const uint32_t stage = smem_u32(sm.out) + (warp - 4) * 4 * kOutBoxBytes;
+                if (lane == 0) bulk_wait_read_all();          // the previous tile's stores have read it
+                __syncwarp();
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
                     if (r == 1 && !full) break;
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint32_t u[8];
+                    for (int c = 0; c < 2; ++c) {
+                        const uint32_t box = stage + (r * 2 + c) * kOutBoxBytes + lane * 64;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const __nv_bfloat162 b =
-                                __floats2bfloat162_rn(acc[r * 64 + v * 16 + 2 * i], acc[r * 64 + v * 16 + 2 * i + 1]);
-                            u[i] = *reinterpret_cast<const uint32_t*>(&b);
+                        for (int p = 0; p < 4; ++p) {
+                            uint32_t u[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int col = r * 64 + c * 32 + p * 8 + 2 * i;
+                                const __nv_bfloat162 b = __floats2bfloat162_rn(acc[col], acc[col + 1]);
+                                u[i] = *reinterpret_cast<const uint32_t*>(&b);
+                            }
+                            st_shared_v4(box + ((p ^ ((lane >> 1) & 3)) << 4), u[0], u[1], u[2], u[3]);
                         }
-                        st_global_v8(out + r * 128 + v * 16, u);   // one full 32-byte sector per thread
                     }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        if (r == 1 && !full) break;
+#pragma unroll
+                        for (int c = 0; c < 2; ++c)
+                            tma_store_2d(&tmD, sm.out + (warp - 4) * 4 * kOutBoxBytes + (r * 2 + c) * kOutBoxBytes,
+                                         t.n0 + r * 128 + half * 64 + c * 32, t.m0 + q * 32);
+                    }
+                    bulk_commit();
                 }
             } else {
                 // SwiGLU on (a = acc[0..63], b = acc[64..127]) for h columns n0/2 + half*64 + [0, 64)
@@ -338,6 +373,7 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
     }
 
+    if (EPI == 0 && warp >= 4 && lane == 0) bulk_wait_all();   // the output stores have completed
     __syncthreads();
     if (sm.abort_flag) {
         // let TMA copies and MMAs that were already issued land before the memory is released
@@ -627,6 +663,19 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over a row-major bf16 matrix [rows, cols] written in 32 x 32 boxes (64-byte rows), 64-byte swizzle.
+static bool make_out_map(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kOutBox), static_cast<cuuint32_t>(kOutBox)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 template <typename Kern>
 static cudaError_t set_smem(Kern k, size_t bytes) {
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
@@ -646,23 +695,25 @@ static cudaError_t check_reg_split(Kern k) {
 cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                                 const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs, int epilogue,
                                 void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s) {
-    CUtensorMap mapA, mapB;
+    CUtensorMap mapA, mapB, mapD;
     if (layout == 0) {
         if (!make_map(&mapA, A, K, static_cast<uint64_t>(M_rows), kBM)) return cudaErrorInvalidValue;
         if (!make_map(&mapB, B, K, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
-        const size_t smem = sizeof(SmemC) + 1024;
         if (epilogue == 0) {
+            if (!make_out_map(&mapD, D, N, static_cast<uint64_t>(M_rows))) return cudaErrorInvalidValue;
+            const size_t smem = sizeof(SmemC<0>) + 1024;
             cudaError_t err = set_smem(gg_contig_kernel<0>, smem);
             if (err == cudaSuccess) err = check_reg_split(gg_contig_kernel<0>);
             if (err != cudaSuccess) return err;
-            gg_contig_kernel<0><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
-                                                                  Ds, status, wait_ns);
+            gg_contig_kernel<0><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K,
+                                                                  D, Ds, status, wait_ns);
         } else {
+            const size_t smem = sizeof(SmemC<1>) + 1024;
             cudaError_t err = set_smem(gg_contig_kernel<1>, smem);
             if (err == cudaSuccess) err = check_reg_split(gg_contig_kernel<1>);
             if (err != cudaSuccess) return err;
-            gg_contig_kernel<1><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
-                                                                  Ds, status, wait_ns);
+            gg_contig_kernel<1><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, mapA, As, group_info, M_rows, Bs, E, N, K,
+                                                                  D, Ds, status, wait_ns);
         }
     } else {
         if (!make_map(&mapA, A, K, static_cast<uint64_t>(E) * M_rows, kBT)) return cudaErrorInvalidValue;

@@ -124,6 +124,34 @@ __device__ void group_offsets(const int32_t* __restrict__ kept, int E, int maske
     __syncthreads();
 }
 
+// v[i] <- v[i] / s correctly rounded to fp32 (s > 0), without a division per element:
+// Markstein's correction step (P. Markstein, "Computation of elementary functions on the
+// IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with r = 1/s correctly
+// rounded, q0 = v * r rounded, the remainder v - q0 * s is exact in one fused multiply-add
+// and q0 + remainder * r, rounded once, is the correctly rounded quotient, as long as no
+// intermediate leaves the normal range. Zeros keep their sign; lanes whose values are
+// tiny (|v| < 2^-96 or |v / s| < 2^-100) take the correctly rounded division instead.
+__device__ __forceinline__ void quotients_rn(float (&v)[8], float s) {
+    const float r = __frcp_rn(s);
+    float q[8];
+    bool normal = true;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float q0 = v[i] * r;
+        const float rem = fmaf(-q0, s, v[i]);
+        q[i] = fmaf(rem, r, q0);
+        if (v[i] == 0.0f) q[i] = v[i];
+        else normal = normal && fabsf(v[i]) >= 0x1p-96f && fabsf(q[i]) >= 0x1p-100f;
+    }
+    if (normal) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = q[i];
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(v[i], s);
+    }
+}
+
 // blockIdx.x < nchunks: scatter one 32-token chunk (slot maps + quantised rows);
 // blockIdx.x >= nchunks (contiguous layout only): fill expert (x - nchunks)'s padding rows.
 // blockIdx.y selects a slice of the H/128 quantisation groups.
@@ -195,61 +223,75 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
     }
     __syncthreads();
 
-    // quantise (token r of the chunk, group g): a warp takes 4 items at a time so their loads and
-    // reductions overlap; 4 values per lane per item
+    // quantise: warp w takes the (token, group) items of tokens w, w + 8, w + 16, w + 24 of the chunk,
+    // 2U per pass: a half-warp per item, 8 values (16 bytes) per lane. Each phase runs over all
+    // U items of a lane before the next, so the loads, the max butterflies, the divisions and
+    // the stores of different items overlap.
     constexpr int U = 4;
+    const int hl = lane & 15, hw = lane >> 4;
     const int gs = g1 - g0;
-    const int items = kChunk * gs;
-    for (int base = warp * U; base < items; base += 8 * U) {
-        uint2 raw[U];
-        int tok_r[U], grp[U];
+    const int ntok = min(kChunk, T - c * kChunk);
+    const int my_tok = ntok > warp ? (ntok - warp + 7) / 8 : 0;
+    const int my_items = my_tok * gs;
+    const uint32_t inv_gs = (65536u + gs - 1) / gs;          // it / gs == (it * inv_gs) >> 16 for it < 2^16 / 64
+    for (int p0 = 0; p0 < my_items; p0 += 2 * U) {
+        uint4 raw[U];
+        int row_r[U], grp[U];
         bool live[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int it = base + u;
-            tok_r[u] = it / gs;
-            grp[u] = g0 + it % gs;
-            const int t = c * kChunk + tok_r[u];
-            live[u] = it < items && t < T;
-            raw[u] = live[u] ? *reinterpret_cast<const uint2*>(x + static_cast<int64_t>(t) * H + grp[u] * kGroup + lane * 4)
-                             : make_uint2(0, 0);
+            const int it = p0 + 2 * u + hw;
+            const int q = static_cast<int>((static_cast<uint32_t>(it) * inv_gs) >> 16);
+            live[u] = it < my_items;
+            row_r[u] = warp + 8 * q;
+            grp[u] = g0 + it - q * gs;
+            raw[u] = live[u] ? *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(c * kChunk + row_r[u]) * H +
+                                                               grp[u] * kGroup + hl * 8)
+                             : make_uint4(0, 0, 0, 0);
         }
-        float v[U][4], amax[U];
+        float amax[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            v[u][0] = __uint_as_float(raw[u].x << 16);
-            v[u][1] = __uint_as_float(raw[u].x & 0xffff0000u);
-            v[u][2] = __uint_as_float(raw[u].y << 16);
-            v[u][3] = __uint_as_float(raw[u].y & 0xffff0000u);
-            amax[u] = fmaxf(fmaxf(fabsf(v[u][0]), fabsf(v[u][1])), fmaxf(fabsf(v[u][2]), fabsf(v[u][3])));
+            const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+            float m = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xffff0000u))));
+            amax[u] = m;
         }
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1)
+        for (int o = 8; o >= 1; o >>= 1)
 #pragma unroll
             for (int u = 0; u < U; ++u) amax[u] = fmaxf(amax[u], __shfl_xor_sync(0xffffffffu, amax[u], o));
+        float sc[U];
+        uint2 code[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            sc[u] = amax[u] == 0.0f ? 1.0f : __fdiv_rn(amax[u], 448.0f);
+            const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                v[2 * i] = __uint_as_float(w[i] << 16);
+                v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+            }
+            quotients_rn(v, sc[u]);
+            code[u].x = f32x2_to_e4m3x2(v[0], v[1]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[2], v[3])) << 16);
+            code[u].y = f32x2_to_e4m3x2(v[4], v[5]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[6], v[7])) << 16);
+        }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (!live[u]) continue;
-            float sc = 1.0f;
-            uint32_t packed;
-            if (amax[u] == 0.0f) {
-                packed = f32x2_to_e4m3x2(v[u][0], v[u][1]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[u][2], v[u][3])) << 16);
-            } else {
-                sc = __fdiv_rn(amax[u], 448.0f);
-                packed = f32x2_to_e4m3x2(__fdiv_rn(v[u][0], sc), __fdiv_rn(v[u][1], sc)) |
-                         (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(v[u][2], sc), __fdiv_rn(v[u][3], sc))) << 16);
-            }
-            const int r = tok_r[u], g = grp[u];
             for (int j = 0; j < k; ++j) {
-                const int32_t row = dest[r * k + j];
+                const int32_t row = dest[row_r[u] * k + j];
                 if (row < 0) continue;
-                *reinterpret_cast<uint32_t*>(Aq + static_cast<int64_t>(row) * H + g * kGroup + lane * 4) = packed;
-                if (lane == 0) {
+                *reinterpret_cast<uint2*>(Aq + static_cast<int64_t>(row) * H + grp[u] * kGroup + hl * 8) = code[u];
+                if (hl == 0) {
                     if (masked) {
                         const int e = row / masked_max_m, rr = row - e * masked_max_m;
-                        As[(static_cast<int64_t>(e) * G + g) * masked_max_m + rr] = sc;
+                        As[(static_cast<int64_t>(e) * G + grp[u]) * masked_max_m + rr] = sc[u];
                     } else {
-                        As[static_cast<int64_t>(g) * ld_rows + row] = sc;
+                        As[static_cast<int64_t>(grp[u]) * ld_rows + row] = sc[u];
                     }
                 }
             }
@@ -273,10 +315,15 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, int T, in
     permute_scan_kernel<<<E, 256, 0, s>>>(cnt, nchunks, cap, masked_max_m, base, counts, kept, status);
     const int G = H / kGroup;
     const int gx = nchunks + (masked_max_m > 0 ? 0 : E);
-    int gy = (4 * num_sms + gx - 1) / gx;
+    const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1 + kChunk * k);
+    // as many group slices per chunk as keep every block resident at once (one wave)
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_scatter_kernel, 256, smem) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    int gy = per_sm * num_sms / gx;
     gy = gy < 1 ? 1 : (gy > G ? G : gy);
     gy = (G + (G + gy - 1) / gy - 1) / ((G + gy - 1) / gy);   // no empty group slices
-    const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1 + kChunk * k);
     permute_scatter_kernel<<<dim3(gx, gy), 256, smem, s>>>(x, topk_idx, T, H, k, E, nchunks, masked_max_m, ld_rows,
                                                            base, kept, Aq, As, offsets, row_src, slot_row);
     return cudaGetLastError();
