@@ -44,9 +44,9 @@ constexpr int kRegsLow = 40, kRegsHigh = 232;
 constexpr int kRegsSplit = 128 * kRegsLow + 256 * kRegsHigh;   // must fit the launch allocation
 constexpr int kDrainNs = 200000;              // settle time after an abort
 
-// bf16 output (EPI 0) leaves through shared memory and TMA stores: each promotion warp stages
-// its 32 rows x 128 columns as four 32 x 32 boxes (64-byte rows, 64-byte swizzle); one fewer
-// operand stage makes room for them.
+// Outputs leave through shared memory and TMA stores in boxes of 32 rows x 64 bytes (64-byte
+// swizzle): bf16 (EPI 0) as four 32 x 32 boxes per promotion warp (its 32 rows x 128 columns;
+// one fewer operand stage makes room for them), FP8 h (EPI 1) as one 32 x 64 box per warp.
 constexpr int kOutBox = 32;
 constexpr int kOutBoxBytes = kOutBox * kOutBox * 2;            // 2 KB
 constexpr int kOutStageBytes = 8 * 4 * kOutBoxBytes;           // 64 KB
@@ -56,7 +56,7 @@ struct SmemC {
     static constexpr int kStages = EPI == 0 ? 3 : 4;
     uint8_t a[kStages][kABytes];
     uint8_t b[kStages][kBBytes];
-    uint8_t out[EPI == 0 ? kOutStageBytes : 16];
+    uint8_t out[EPI == 0 ? kOutStageBytes : 8 * kOutBoxBytes];
     float sa[kSaSlots][kBM];    // activation scales of one K block for the tile's 128 rows
     uint64_t full[kStages];
     uint64_t empty[kStages];
@@ -356,24 +356,34 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 // h / s as h * (1 / s): the correctly rounded reciprocal keeps the quotient within one
                 // ulp of the division, below the resolution of the E4M3 code it is rounded to
                 const float rs = amax == 0.0f ? 1.0f : __frcp_rn(s);
-                uint8_t* hq = static_cast<uint8_t*>(D) + grow * I + t.n0 / 2 + half * 64;
+                // this warp's 32 rows x 64 codes leave as one 32 x 64-byte box through shared memory
+                // (64-byte swizzle: 16-byte piece p of row l at p ^ ((l >> 1) & 3))
+                const uint32_t box = smem_u32(sm.out) + (warp - 4) * kOutBoxBytes;
+                if (lane == 0) bulk_wait_read_all();          // the previous tile's store has read it
+                __syncwarp();
 #pragma unroll
-                for (int v = 0; v < 2; ++v) {
-                    uint32_t u[8];
+                for (int p = 0; p < 4; ++p) {
+                    uint32_t u[4];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int c = v * 32 + i * 4;
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = p * 16 + i * 4;
                         u[i] = f32x2_to_e4m3x2(acc[c] * rs, acc[c + 1] * rs) |
                                (static_cast<uint32_t>(f32x2_to_e4m3x2(acc[c + 2] * rs, acc[c + 3] * rs)) << 16);
                     }
-                    st_global_v8(hq + v * 32, u);
+                    st_shared_v4(box + lane * 64 + ((p ^ ((lane >> 1) & 3)) << 4), u[0], u[1], u[2], u[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmD, sm.out + (warp - 4) * kOutBoxBytes, t.n0 / 2 + half * 64, t.m0 + q * 32);
+                    bulk_commit();
                 }
                 if (half == 0) Ds[static_cast<int64_t>(t.n0 / kBN) * M_rows + grow] = s;
             }
         }
     }
 
-    if (EPI == 0 && warp >= 4 && lane == 0) bulk_wait_all();   // the output stores have completed
+    if (warp >= 4 && lane == 0) bulk_wait_all();   // the output stores have completed
     __syncthreads();
     if (sm.abort_flag) {
         // let TMA copies and MMAs that were already issued land before the memory is released
@@ -395,20 +405,24 @@ constexpr int kThreadsM = 192;                // 6 warps
 template <int EPI>
 struct SmemM {
     static constexpr int kW = EPI == 1 ? 2 * kWBlk : kWBlk;    // weight rows per stage: 256 (a|b) or 128
-    static constexpr int kStages = EPI == 1 ? 4 : 8;
+    static constexpr int kStages = EPI == 1 ? 4 : 10;
     static constexpr int kCols = EPI == 1 ? 2 * kBT : kBT;     // tensor-memory columns per buffer
     static constexpr int kBufs = 4;                            // MMA runs up to 3 K blocks ahead of promotion
     uint8_t w[kStages][kW];
     uint8_t x[kStages][kXBytes];
-    float hs[2][kBT][kBM];                                      // SwiGLU output staged for the requant
+    float hs[EPI == 1 ? 2 : 1][EPI == 1 ? kBT : 1][kBM];       // SwiGLU output staged for the requant
+    float sa[kSaSlots][kBT];                                    // activation scales of one K block, 32 tokens
     uint64_t full[kStages];
     uint64_t empty[kStages];
+    uint64_t sfull[kSaSlots];
+    uint64_t sempty[kSaSlots];
     uint64_t tfull[kBufs];
     uint64_t tempty[kBufs];
     uint64_t red_bar[2];
     uint32_t tmem_base;
     volatile int abort_flag;
     int32_t P[kMaxE + 1];
+    int32_t M[kMaxE];                                           // tokens per expert (masked_m)
 };
 
 template <int EPI>
@@ -432,7 +446,9 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         if (lane == 0) sm.P[0] = 0;
         for (int b = 0; b < E; b += 32) {
             const int e = b + lane;
-            int32_t v = e < E ? NBt * ((masked_m[e] + kBT - 1) / kBT) : 0;
+            const int32_t m = e < E ? masked_m[e] : 0;
+            if (e < E) sm.M[e] = m;
+            int32_t v = NBt * ((m + kBT - 1) / kBT);
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
@@ -446,6 +462,10 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         for (int s = 0; s < S::kStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
+        }
+        for (int j = 0; j < kSaSlots; ++j) {
+            mbar_init(&sm.sfull[j], 1);
+            mbar_init(&sm.sempty[j], 4);
         }
         for (int b = 0; b < S::kBufs; ++b) {
             mbar_init(&sm.tfull[b], 1);
@@ -471,7 +491,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     };
     auto decode = [&](int tile, int& e, int& nb, int& tt, int& m_e) {
         e = find_group(sm.P, E, tile);
-        m_e = masked_m[e];
+        m_e = sm.M[e];
         const int ntt = (m_e + kBT - 1) / kBT;
         const int local = tile - sm.P[e];
         nb = local / ntt;
@@ -495,6 +515,12 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     tma_load_2d(sm.w[s], &tmW, &sm.full[s], kb * kBK, wrow);
                     if (EPI == 1) tma_load_2d(sm.w[s] + kWBlk, &tmW, &sm.full[s], kb * kBK, wrow + kBM);
                     tma_load_2d(sm.x[s], &tmX, &sm.full[s], kb * kBK, e * Mmax + tt * kBT);
+                    // the token tile's 32 activation scales of this K block, into the scale ring
+                    const int j = it % kSaSlots;
+                    if (!mbar_wait(&sm.sempty[j], ((it / kSaSlots) & 1) ^ 1, wait_ns)) { fail(); break; }
+                    mbar_arrive_expect_tx(&sm.sfull[j], kBT * sizeof(float));
+                    bulk_load(sm.sa[j], As + (static_cast<int64_t>(e) * KB + kb) * Mmax + tt * kBT, kBT * sizeof(float),
+                              &sm.sfull[j]);
                 }
             }
         }
@@ -530,6 +556,22 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         const int pw = warp - 2;                 // 0..3
         const int r = q * 32 + lane;
         uint32_t kbt = 0, ep = 0;
+        // lane l holds the weight-block scales of K blocks l, l + 32, l + 64, l + 96 of the tile's
+        // weight block(s) (K <= 16384), loaded one tile ahead so their latency hides behind a tile
+        float wa[4], wb[4];
+        auto load_w = [&](int tile) {
+            if (tile >= total) return;
+            int e, nb, tt, m_e;
+            decode(tile, e, nb, tt, m_e);
+            const float* pa = Bs + (static_cast<int64_t>(e) * NB + (EPI == 1 ? 2 * nb : nb)) * KB;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int kb = lane + 32 * i;
+                wa[i] = kb < KB ? pa[kb] : 0.0f;
+                wb[i] = EPI == 1 && kb < KB ? pa[KB + kb] : 0.0f;
+            }
+        };
+        load_w(blockIdx.x);
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             if (sm.abort_flag) break;
             int e, nb, tt, m_e;
@@ -537,32 +579,30 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             float acc[EPI == 1 ? 2 * kBT : kBT];
 #pragma unroll
             for (int i = 0; i < (EPI == 1 ? 2 * kBT : kBT); ++i) acc[i] = 0.0f;
-            const int blk_a = EPI == 1 ? 2 * nb : nb;
-            const float* bsa = Bs + (static_cast<int64_t>(e) * NB + blk_a) * KB;
-            const float* bsb = bsa + KB;
+            const float wta[4] = {wa[0], wa[1], wa[2], wa[3]};
+            const float wtb[4] = {wb[0], wb[1], wb[2], wb[3]};
+            load_w(tile + gridDim.x);
             bool ok = true;
-            // the token tile's scales for K block kb + 1 load while block kb is promoted
-            const float4* sa_base = reinterpret_cast<const float4*>(As + static_cast<int64_t>(e) * KB * Mmax + tt * kBT);
-            float4 nxt[kBT / 4];
-#pragma unroll
-            for (int i = 0; i < kBT / 4; ++i) nxt[i] = sa_base[i];
-            float nxt_wa = bsa[0], nxt_wb = EPI == 1 ? bsb[0] : 0.0f;
             for (int kb = 0; kb < KB; ++kb, ++kbt) {
                 const int buf = kbt % S::kBufs;
                 const uint32_t bph = (kbt / S::kBufs) & 1;
+                // scales: the token tile's 32 from the ring, the weight block's from the lane holding it
+                const int j = kbt % kSaSlots;
+                if (!mbar_wait(&sm.sfull[j], (kbt / kSaSlots) & 1, wait_ns)) { fail(); ok = false; break; }
                 float sa[kBT];
 #pragma unroll
                 for (int i = 0; i < kBT / 4; ++i) {
-                    sa[4 * i] = nxt[i].x; sa[4 * i + 1] = nxt[i].y; sa[4 * i + 2] = nxt[i].z; sa[4 * i + 3] = nxt[i].w;
+                    const float4 v4 = *reinterpret_cast<const float4*>(&sm.sa[j][4 * i]);
+                    sa[4 * i] = v4.x; sa[4 * i + 1] = v4.y; sa[4 * i + 2] = v4.z; sa[4 * i + 3] = v4.w;
                 }
-                const float swa = nxt_wa, swb = nxt_wb;
-                if (kb + 1 < KB) {
-                    const float4* p4 = sa_base + static_cast<int64_t>(kb + 1) * (Mmax / 4);
-#pragma unroll
-                    for (int i = 0; i < kBT / 4; ++i) nxt[i] = p4[i];
-                    nxt_wa = bsa[kb + 1];
-                    if (EPI == 1) nxt_wb = bsb[kb + 1];
-                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.sempty[j]);
+                const int wi = kb >> 5;
+                const float swa = __shfl_sync(0xffffffffu, wi == 0 ? wta[0] : wi == 1 ? wta[1] : wi == 2 ? wta[2] : wta[3],
+                                              kb & 31);
+                const float swb = EPI == 1 ? __shfl_sync(0xffffffffu, wi == 0 ? wtb[0] : wi == 1 ? wtb[1]
+                                                                      : wi == 2 ? wtb[2] : wtb[3], kb & 31)
+                                           : 0.0f;
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * S::kCols;
@@ -663,15 +703,17 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D map over a row-major bf16 matrix [rows, cols] written in 32 x 32 boxes (64-byte rows), 64-byte swizzle.
-static bool make_out_map(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows) {
+// 2-D map over a row-major matrix [rows, cols] of bf16 (elem_bytes 2) or bytes (1) written in boxes of
+// 32 rows x 64 bytes, 64-byte swizzle.
+static bool make_out_map(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, int elem_bytes) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kOutBox), static_cast<cuuint32_t>(kOutBox)};
+    const cuuint64_t strides[1] = {cols * elem_bytes};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(64 / elem_bytes), static_cast<cuuint32_t>(kOutBox)};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    return fn(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims,
+              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
@@ -700,7 +742,7 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
         if (!make_map(&mapA, A, K, static_cast<uint64_t>(M_rows), kBM)) return cudaErrorInvalidValue;
         if (!make_map(&mapB, B, K, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
         if (epilogue == 0) {
-            if (!make_out_map(&mapD, D, N, static_cast<uint64_t>(M_rows))) return cudaErrorInvalidValue;
+            if (!make_out_map(&mapD, D, N, static_cast<uint64_t>(M_rows), 2)) return cudaErrorInvalidValue;
             const size_t smem = sizeof(SmemC<0>) + 1024;
             cudaError_t err = set_smem(gg_contig_kernel<0>, smem);
             if (err == cudaSuccess) err = check_reg_split(gg_contig_kernel<0>);
@@ -708,11 +750,12 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
             gg_contig_kernel<0><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K,
                                                                   D, Ds, status, wait_ns);
         } else {
+            if (!make_out_map(&mapD, D, N / 2, static_cast<uint64_t>(M_rows), 1)) return cudaErrorInvalidValue;
             const size_t smem = sizeof(SmemC<1>) + 1024;
             cudaError_t err = set_smem(gg_contig_kernel<1>, smem);
             if (err == cudaSuccess) err = check_reg_split(gg_contig_kernel<1>);
             if (err != cudaSuccess) return err;
-            gg_contig_kernel<1><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, mapA, As, group_info, M_rows, Bs, E, N, K,
+            gg_contig_kernel<1><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K,
                                                                   D, Ds, status, wait_ns);
         }
     } else {
