@@ -12,7 +12,8 @@
 
 namespace moe {
 cudaError_t launch_router_softmax(const uint16_t* x, const float* Wg, const float* bias, float* logits, int T, int H,
-                                  int E, int k, int32_t* topk_idx, float* topk_w, int num_sms, cudaStream_t s);
+                                  int E, int k, int32_t* topk_idx, float* topk_w, int* status, uint64_t wait_ns,
+                                  int num_sms, cudaStream_t s);
 cudaError_t launch_router_hash(const int32_t* token_ids, int T, int E, int32_t* topk_idx, float* topk_w,
                                cudaStream_t s);
 size_t permute_scratch_bytes(int T, int E);
@@ -188,7 +189,8 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* Wg, 
     if (cfg->routing == MOE_ROUTE_HASH)
         return cuda_status(launch_router_hash(token_ids, cfg->T, cfg->E, topk_idx, topk_w, s));
     return cuda_status(launch_router_softmax(static_cast<const uint16_t*>(x), Wg, bias, static_cast<float*>(ws),
-                                             cfg->T, cfg->H, cfg->E, cfg->k, topk_idx, topk_w, dev->num_sms, s));
+                                             cfg->T, cfg->H, cfg->E, cfg->k, topk_idx, topk_w, dev->status, kWaitNs,
+                                             dev->num_sms, s));
 }
 
 moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, uint8_t* Aq, float* As,
@@ -272,7 +274,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
         e = launch_router_hash(token_ids, cfg->T, cfg->E, topk_idx, topk_w, s);
     else
         e = launch_router_softmax(static_cast<const uint16_t*>(x), Wg, bias, static_cast<float*>(w.step), cfg->T,
-                                  cfg->H, cfg->E, cfg->k, topk_idx, topk_w, dev->num_sms, s);
+                                  cfg->H, cfg->E, cfg->k, topk_idx, topk_w, dev->status, kWaitNs, dev->num_sms, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_permute(static_cast<const uint16_t*>(x), topk_idx, cfg->T, cfg->H, cfg->k, cfg->E, capacity_of(cfg),
                        masked ? cfg->masked_max_m : 0, rows, w.Aq, w.As, counts, w.kept, w.offsets, w.row_src,

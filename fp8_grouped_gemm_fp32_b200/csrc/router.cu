@@ -4,181 +4,140 @@
 // hash routing expert = hash(token_id) % E (DeepSeek-V4 lecture page, 2.2).
 //
 // Logits use one fixed fp32 order so the selected experts are reproducible
-// bit for bit: lane j of a warp owns h = j, j+32, j+64, ... and runs one
-// fused multiply-add chain over them in ascending h from +0; the 32 partial
-// sums are combined by an xor butterfly (j with j^16, then ^8, ^4, ^2, ^1),
-// which pairs j with j+16 first, then j+8, ... exactly; the bias is added last.
+// bit for bit: lane j of a warp owns h = 128 s + 4 j + i (i = 0..3, every
+// 128-wide block s of H) and runs one fused multiply-add chain over them in
+// ascending h from +0; the 32 partial sums are combined by an xor butterfly
+// (j with j^16, then ^8, ^4, ^2, ^1), which pairs j with j+16 first, then
+// j+8, ... exactly; the bias is added last.
 //
-// The logits kernel tiles tokens x experts so each W_g / x element staged in
-// shared memory feeds TR x ER register accumulators per lane (CUDA cores: the
-// fixed order rules out the tensor cores); logits go to scratch, and a
-// warp-per-token kernel selects the top-k and computes the weights in fp64.
-// W_g (7.3 MB at the largest size) stays L2-resident across token tiles.
+// The logits kernel tiles tokens x experts: a producer thread streams 128-wide
+// blocks of x ([tokens, h], bf16) and W_g ([experts, h], fp32) with TMA into a
+// ring of shared-memory stages, row-major as they lie in global memory, and
+// each compute warp keeps a TR x ER register tile per lane, so every 16-byte
+// W_g load feeds 4 * TR and every 8-byte x load 4 * ER multiply-adds (CUDA
+// cores: the fixed order rules out the tensor cores). Logits go to scratch,
+// and a warp-per-token kernel selects the top-k and computes the weights in
+// fp64. W_g (7.3 MB at the largest size) stays L2-resident across token tiles.
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int kRouterHS = 128;     // h values per stage
-constexpr int kPlaneRows = kRouterHS;
-constexpr int kPlaneBytes = kPlaneRows * 16;   // one plane: 128 rows x 16 bytes
-
-// Operands are staged h-major in "planes" of 16 bytes per h: 8 tokens (bf16) or 4
-// experts (fp32) per plane, so a lane fetches all the tokens (experts) it needs for
-// its h with one 16-byte load per plane. Rows are XOR-swizzled within each 8-row
-// group, and W planes are padded by 32 bytes, so both the transposing stores and the
-// 16-byte loads are free of bank conflicts.
-__device__ __forceinline__ int swz_row(int row) { return row ^ ((row >> 3) & 7); }
+constexpr int kRouterHS = 128;     // h values per stage: lane j takes h = 4j .. 4j+3 of each
 
 template <int TR, int ER, int WT, int WE>
-struct RouterTile {
-    static constexpr int TT = TR * WT;               // tokens per CTA
-    static constexpr int EC = ER * WE;               // experts per CTA
-    static constexpr int kThreads = 32 * WT * WE;
-    static constexpr int kXPlanes = TT / 8;
-    static constexpr int kWPlanes = EC / 4;
-    static constexpr int kWPlaneStride = kPlaneBytes + 32;
-    static constexpr int kXBytes = kXPlanes * kPlaneBytes;
-    static constexpr int kStageBytes = kXBytes + kWPlanes * kWPlaneStride;
-    static constexpr int kSmem = 2 * kStageBytes;
-    // global -> register chunks per thread per stage (16 bytes each)
-    static constexpr int kXChunks = TT * (kRouterHS / 8) / kThreads;     // 8 h of one token
-    static constexpr int kWChunks = EC * (kRouterHS / 4) / kThreads;     // 4 h of one expert
-    static_assert(TR % 8 == 0 && ER % 4 == 0, "register tile must cover whole planes");
-    static_assert(TT * (kRouterHS / 8) % kThreads == 0 && EC * (kRouterHS / 4) % kThreads == 0, "chunking");
+struct RouterCfg {
+    static constexpr int TT = TR * WT;                  // tokens per CTA
+    static constexpr int EC = ER * WE;                  // experts per CTA
+    static constexpr int kCompute = WT * WE;            // compute warps, after the producer warpgroup
+    static constexpr int kThreads = 32 * (kCompute + 4);
+    // large register tiles: the producer warpgroup gives registers to the compute warps
+    static constexpr bool kSplit = TR * ER >= 128;
+    static constexpr int kRegsLow = 40, kRegsHigh = 232;
+    static constexpr int kXBytes = TT * kRouterHS * 2;
+    static constexpr int kWBytes = EC * kRouterHS * 4;
+    static constexpr int kStageBytes = kXBytes + kWBytes;
+    static constexpr int kStages = 160 * 1024 / kStageBytes < 8 ? 160 * 1024 / kStageBytes : 8;
+    static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8 + 16 + 1024;
 };
 
 template <int TR, int ER, int WT, int WE>
-__global__ void __launch_bounds__(RouterTile<TR, ER, WT, WE>::kThreads, 1)
-router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ Wg, const float* __restrict__ bias,
-                     float* __restrict__ logits, int T, int H, int E) {
-    using Tile = RouterTile<TR, ER, WT, WE>;
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int t_base = blockIdx.x * Tile::TT;
-    const int e_base = blockIdx.y * Tile::EC;
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int wt = warp / WE, we = warp % WE;
+__global__ void __launch_bounds__(RouterCfg<TR, ER, WT, WE>::kThreads, 1)
+router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const float* __restrict__ bias, float* __restrict__ logits, int T, int H, int E, int* status,
+                     uint64_t wait_ns) {
+    using C = RouterCfg<TR, ER, WT, WE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+    uint64_t* empty = full + C::kStages;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::kStages);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t_base = blockIdx.x * C::TT, e_base = blockIdx.y * C::EC;
     const int nst = H / kRouterHS;
 
-    // Chunk c of a stage: x chunks are (token, 8-h piece) with 4 pieces of one token per
-    // 4 consecutive threads and 8 tokens per warp; W chunks are (expert, 4-h piece) alike.
-    uint4 xr[Tile::kXChunks], wr[Tile::kWChunks];
-    auto load_stage = [&](int st) {
-        const int h0 = st * kRouterHS;
-#pragma unroll
-        for (int i = 0; i < Tile::kXChunks; ++i) {
-            const int c = tid + i * Tile::kThreads;          // 0 .. TT*16
-            const int grp = c >> 5, l = c & 31;               // 32 chunks: 8 tokens x 4 pieces
-            const int tok = (grp % (Tile::TT / 8)) * 8 + (l >> 2);
-            const int piece = (grp / (Tile::TT / 8)) * 4 + (l & 3);
-            const int t = t_base + tok;
-            xr[i] = t < T ? *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H + h0 + piece * 8)
-                          : make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], C::kCompute);
         }
-#pragma unroll
-        for (int i = 0; i < Tile::kWChunks; ++i) {
-            const int c = tid + i * Tile::kThreads;          // 0 .. EC*32
-            const int grp = c >> 5, l = c & 31;               // 32 chunks: 8 experts x 4 pieces
-            const int ex = (grp % (Tile::EC / 8)) * 8 + (l >> 2);
-            const int piece = (grp / (Tile::EC / 8)) * 4 + (l & 3);
-            const int e = e_base + ex;
-            wr[i] = e < E ? *reinterpret_cast<const uint4*>(Wg + static_cast<int64_t>(e) * H + h0 + piece * 4)
-                          : make_uint4(0, 0, 0, 0);
-        }
-    };
-    auto store_stage = [&](int buf) {
-        uint8_t* sx = smem + buf * Tile::kStageBytes;
-        uint8_t* sw = sx + Tile::kXBytes;
-#pragma unroll
-        for (int i = 0; i < Tile::kXChunks; ++i) {
-            const int c = tid + i * Tile::kThreads;
-            const int grp = c >> 5, l = c & 31;
-            const int tok = (grp % (Tile::TT / 8)) * 8 + (l >> 2);
-            const int piece = (grp / (Tile::TT / 8)) * 4 + (l & 3);
-            uint8_t* plane = sx + (tok >> 3) * kPlaneBytes + (tok & 7) * 2;
-            const uint32_t u[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const int row = piece * 8 + r;
-                *reinterpret_cast<uint16_t*>(plane + swz_row(row) * 16) =
-                    static_cast<uint16_t>(r & 1 ? u[r >> 1] >> 16 : u[r >> 1] & 0xffffu);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < Tile::kWChunks; ++i) {
-            const int c = tid + i * Tile::kThreads;
-            const int grp = c >> 5, l = c & 31;
-            const int ex = (grp % (Tile::EC / 8)) * 8 + (l >> 2);
-            const int piece = (grp / (Tile::EC / 8)) * 4 + (l & 3);
-            uint8_t* plane = sw + (ex >> 2) * Tile::kWPlaneStride + (ex & 3) * 4;
-            const uint32_t u[4] = {wr[i].x, wr[i].y, wr[i].z, wr[i].w};
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int row = piece * 4 + r;
-                *reinterpret_cast<uint32_t*>(plane + swz_row(row) * 16) = u[r];
-            }
-        }
-    };
-
-    float acc[TR][ER];
-#pragma unroll
-    for (int i = 0; i < TR; ++i)
-#pragma unroll
-        for (int q = 0; q < ER; ++q) acc[i][q] = 0.0f;
-
-    load_stage(0);
-    store_stage(0);
-    if (nst > 1) load_stage(1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
     __syncthreads();
-    for (int st = 0; st < nst; ++st) {
-        const uint8_t* sx = smem + (st & 1) * Tile::kStageBytes;
-        const uint8_t* sxw = sx + (wt * (TR / 8)) * kPlaneBytes;
-        const uint8_t* sww = sx + Tile::kXBytes + (we * (ER / 4)) * Tile::kWPlaneStride;
-#pragma unroll
-        for (int s = 0; s < kRouterHS / 32; ++s) {
-            const int row16 = swz_row(s * 32 + lane) * 16;
-            float2 xv[TR / 2];
-            float wv[ER];
-#pragma unroll
-            for (int p = 0; p < TR / 8; ++p) {
-                const uint4 v = *reinterpret_cast<const uint4*>(sxw + p * kPlaneBytes + row16);
-                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    xv[p * 4 + i] = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
+    auto fail = [&]() {
+        set_status(status, kStatusTimeout);
+        *abort_flag = 1;
+    };
+
+    if (warp < 4) {
+        if constexpr (C::kSplit) setmaxnreg_dec<C::kRegsLow>();
+        if (warp == 0 && lane == 0) {
+            prefetch_tensormap(&tmX);
+            prefetch_tensormap(&tmW);
+            for (int st = 0; st < nst && !*abort_flag; ++st) {
+                const int s = st % C::kStages;
+                if (!mbar_wait(&empty[s], ((st / C::kStages) & 1) ^ 1, wait_ns)) { fail(); break; }
+                uint8_t* stage = smem + s * C::kStageBytes;
+                mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                tma_load_2d(stage, &tmX, &full[s], st * kRouterHS, t_base);
+                tma_load_2d(stage + C::kXBytes, &tmW, &full[s], st * kRouterHS, e_base);
             }
+        }
+    } else {
+        if constexpr (C::kSplit) setmaxnreg_inc<C::kRegsHigh>();
+        const int cw = warp - 4, wt = cw / WE, we = cw % WE;
+        float acc[TR][ER];
 #pragma unroll
-            for (int p = 0; p < ER / 4; ++p) {
-                const float4 v = *reinterpret_cast<const float4*>(sww + p * Tile::kWPlaneStride + row16);
-                wv[p * 4] = v.x; wv[p * 4 + 1] = v.y; wv[p * 4 + 2] = v.z; wv[p * 4 + 3] = v.w;
-            }
-            // lane j runs the chains for h = j (mod 32), ascending h
+        for (int i = 0; i < TR; ++i)
 #pragma unroll
-            for (int i = 0; i < TR / 2; ++i)
+            for (int q = 0; q < ER; ++q) acc[i][q] = 0.0f;
+        bool ok = true;
+        for (int st = 0; st < nst; ++st) {
+            const int s = st % C::kStages;
+            if (*abort_flag || !mbar_wait(&full[s], (st / C::kStages) & 1, wait_ns)) { fail(); ok = false; break; }
+            const uint8_t* stage = smem + s * C::kStageBytes;
+            const uint16_t* xs = reinterpret_cast<const uint16_t*>(stage) + (wt * TR) * kRouterHS + 4 * lane;
+            const float* ws = reinterpret_cast<const float*>(stage + C::kXBytes) + (we * ER) * kRouterHS + 4 * lane;
+            float4 wv[ER];
+#pragma unroll
+            for (int q = 0; q < ER; ++q) wv[q] = *reinterpret_cast<const float4*>(ws + q * kRouterHS);
+#pragma unroll
+            for (int i = 0; i < TR; ++i) {
+                const uint2 xr = *reinterpret_cast<const uint2*>(xs + i * kRouterHS);
+                const float x0 = __uint_as_float(xr.x << 16), x1 = __uint_as_float(xr.x & 0xffff0000u);
+                const float x2 = __uint_as_float(xr.y << 16), x3 = __uint_as_float(xr.y & 0xffff0000u);
+                // lane j's chain for (token, expert) runs over h = 4j, 4j+1, 4j+2, 4j+3 of this block in order
 #pragma unroll
                 for (int q = 0; q < ER; ++q) {
-                    acc[2 * i][q] = fmaf(xv[i].x, wv[q], acc[2 * i][q]);
-                    acc[2 * i + 1][q] = fmaf(xv[i].y, wv[q], acc[2 * i + 1][q]);
+                    acc[i][q] = fmaf(x0, wv[q].x, acc[i][q]);
+                    acc[i][q] = fmaf(x1, wv[q].y, acc[i][q]);
+                    acc[i][q] = fmaf(x2, wv[q].z, acc[i][q]);
+                    acc[i][q] = fmaf(x3, wv[q].w, acc[i][q]);
                 }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
-        if (st + 1 < nst) {
-            store_stage((st + 1) & 1);       // the buffer read at st - 1; every warp passed the barrier since
-            if (st + 2 < nst) load_stage(st + 2);
+        if (ok) {
+#pragma unroll
+            for (int i = 0; i < TR; ++i) {
+#pragma unroll
+                for (int q = 0; q < ER; ++q) {
+                    float v = acc[i][q];
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
+                    const int t = t_base + wt * TR + i, e = e_base + we * ER + q;
+                    if (lane == ((i * ER + q) & 31) && t < T && e < E)
+                        logits[static_cast<int64_t>(t) * E + e] = bias ? v + bias[e] : v;
+                }
+            }
         }
-        __syncthreads();
     }
-
-#pragma unroll
-    for (int i = 0; i < TR; ++i) {
-#pragma unroll
-        for (int q = 0; q < ER; ++q) {
-            float v = acc[i][q];
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
-            const int t = t_base + wt * TR + i, e = e_base + we * ER + q;
-            if (lane == ((i * ER + q) & 31) && t < T && e < E)
-                logits[static_cast<int64_t>(t) * E + e] = bias ? v + bias[e] : v;
-        }
+    __syncthreads();
+    if (*abort_flag) {
+        // let TMA copies that were already issued land before the shared memory is released
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000) __nanosleep(1000);
     }
 }
 
@@ -251,30 +210,59 @@ __global__ void router_hash_kernel(const int32_t* __restrict__ token_ids, int T,
     topk_w[t] = 1.0f;
 }
 
+// 2-D map over a row-major matrix [rows, cols] of 2- or 4-byte elements, read in boxes of 128 columns x
+// box_rows rows without swizzling; rows past the end read as zeros.
+static bool make_router_map(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
+                            uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = tensor_map_encoder();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * elem_bytes};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRouterHS), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 template <int TR, int ER, int WT, int WE>
 static cudaError_t launch_logits(const uint16_t* x, const float* Wg, const float* bias, float* logits, int T, int H,
-                                 int E, cudaStream_t s) {
-    using Tile = RouterTile<TR, ER, WT, WE>;
+                                 int E, int* status, uint64_t wait_ns, cudaStream_t s) {
+    using C = RouterCfg<TR, ER, WT, WE>;
+    CUtensorMap mx, mw;
+    if (!make_router_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, H, T, C::TT) ||
+        !make_router_map(&mw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, Wg, H, E, C::EC))
+        return cudaErrorInvalidValue;
     auto kern = router_logits_kernel<TR, ER, WT, WE>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile::kSmem);
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (err != cudaSuccess) return err;
-    dim3 grid((T + Tile::TT - 1) / Tile::TT, (E + Tile::EC - 1) / Tile::EC);
-    kern<<<grid, Tile::kThreads, Tile::kSmem, s>>>(x, Wg, bias, logits, T, H, E);
+    if constexpr (C::kSplit) {
+        // setmaxnreg.inc can only hand out registers the block was launched with: refuse a build whose
+        // launch allocation is smaller than the split instead of starting it
+        cudaFuncAttributes a;
+        err = cudaFuncGetAttributes(&a, kern);
+        if (err != cudaSuccess) return err;
+        if (a.numRegs * C::kThreads < 128 * C::kRegsLow + (C::kThreads - 128) * C::kRegsHigh)
+            return cudaErrorInvalidConfiguration;
+    }
+    dim3 grid((T + C::TT - 1) / C::TT, (E + C::EC - 1) / C::EC);
+    kern<<<grid, C::kThreads, C::kSmem, s>>>(mx, mw, bias, logits, T, H, E, status, wait_ns);
     return cudaGetLastError();
 }
 
 cudaError_t launch_router_softmax(const uint16_t* x, const float* Wg, const float* bias, float* logits, int T, int H,
-                                  int E, int k, int32_t* topk_idx, float* topk_w, int num_sms, cudaStream_t s) {
+                                  int E, int k, int32_t* topk_idx, float* topk_w, int* status, uint64_t wait_ns,
+                                  int num_sms, cudaStream_t s) {
     cudaError_t err;
     // the largest register tile whose CTAs still cover the GPU at least once
     const long ctas_big = static_cast<long>((T + 31) / 32) * ((E + 31) / 32);
     const long ctas_mid = static_cast<long>((T + 15) / 16) * ((E + 15) / 16);
     if (ctas_big >= num_sms)
-        err = launch_logits<16, 8, 2, 4>(x, Wg, bias, logits, T, H, E, s);      // 32 tokens x 32 experts
+        err = launch_logits<16, 8, 2, 4>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);   // 32 tokens x 32 experts
     else if (ctas_mid >= num_sms)
-        err = launch_logits<8, 4, 2, 4>(x, Wg, bias, logits, T, H, E, s);       // 16 tokens x 16 experts
+        err = launch_logits<8, 4, 2, 4>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);    // 16 tokens x 16 experts
     else
-        err = launch_logits<8, 4, 1, 4>(x, Wg, bias, logits, T, H, E, s);       // 8 tokens x 16 experts
+        err = launch_logits<8, 4, 1, 4>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);    // 8 tokens x 16 experts
     if (err != cudaSuccess) return err;
     const int blocks = (T + 7) / 8;
     if (E <= 64)

@@ -115,7 +115,8 @@ static void parallel_for(int64_t n, int nthreads, range_fn fn, void* ctx) {
 /* ------------------------------------------------------------------ */
 /* Canonical fp32 order for one logit (a reading: the pages fix no order, and
  * bit-identical expert selection needs one). With 32 partial sums:
- *   p_j = fma-chain over h = j, j+32, j+64, ... ascending, starting from +0;
+ *   p_j = fma-chain over h = 128 s + 4 j + i (i = 0..3, s = 0, 1, ...), that
+ *         is four consecutive h in every 128-wide block, ascending, from +0;
  *   then pairwise halving p_j <- p_j + p_{j+w} for w = 16, 8, 4, 2, 1;
  *   l = p_0 + b_e. */
 typedef struct { int H, E; const uint16_t* x; const float* Wg; const float* bias; float* logits; } logit_ctx;
@@ -132,7 +133,12 @@ static void logits_range(void* vctx, int64_t b, int64_t e) {
             float p[32];
             for (j = 0; j < 32; ++j) {
                 float acc = 0.0f;
-                for (h = j; h < c->H; h += 32) acc = fmaf(xf[h], wr[h], acc);
+                int s0, i;
+                for (s0 = 0; s0 < c->H; s0 += 128)
+                    for (i = 0; i < 4; ++i) {
+                        h = s0 + 4 * j + i;
+                        if (h < c->H) acc = fmaf(xf[h], wr[h], acc);
+                    }
                 p[j] = acc;
             }
             for (w = 16; w >= 1; w >>= 1)

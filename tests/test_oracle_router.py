@@ -18,32 +18,43 @@ def _bf16_bits(a):
 
 
 def test_logit_tree_pairs_lane_j_with_j_plus_16():
-    # H = 64: lane j sums h = j and j + 32. Put 2^24 in lane 0 and 1 in lanes 8 and 24.
-    # Canonical halving: (p8 + p24) = 2 meets 2^24 exactly at the w=8 level -> 2^24 + 2.
+    # H = 128: lane j sums h = 4j .. 4j+3. Put 2^24 in lane 0 (h = 0) and 1 in lanes 8 (h = 32) and
+    # 24 (h = 96). Canonical halving: (p8 + p24) = 2 meets 2^24 exactly at the w=8 level -> 2^24 + 2.
     # Any left-to-right order loses both 1s against 2^24 (ulp 2) -> 2^24.
-    H = 64
+    H = 128
     x = np.zeros((1, H), np.float32)
     W = np.zeros((1, H), np.float32)
-    x[0, [0, 8, 24]] = 1.0
+    x[0, [0, 32, 96]] = 1.0
     W[0, 0] = 2.0 ** 24
-    W[0, 8] = 1.0
-    W[0, 24] = 1.0
+    W[0, 32] = 1.0
+    W[0, 96] = 1.0
     l = oracle.router_logits(_bf16_bits(x), W, None, nthreads=1)
     assert l[0, 0] == np.float32(2.0 ** 24 + 2)
 
 
-def test_logit_lane_partial_uses_fused_multiply_add():
-    # One lane (j = 0) of H = 64 sums h = 0 then h = 32: p = fma(x32, w32, fma(x0, w0, 0)).
-    # x0*w0 = -(1 + 2^-7) exactly; x32*w32 = (1 + 2^-7)(1 + 2^-23) = 1 + 2^-7 + 2^-23 + 2^-30.
-    # The fused chain cancels exactly to 2^-23 + 2^-30; rounding the product first loses 2^-30.
-    H = 64
+def _cancelling_pair(H, h0, h1):
+    # x[h0] * W[h0] = -(1 + 2^-7) exactly; x[h1] * W[h1] = (1 + 2^-7)(1 + 2^-23) = 1 + 2^-7 + 2^-23 + 2^-30.
+    # In one fused multiply-add chain (h0 first) they cancel exactly to 2^-23 + 2^-30; rounding the second
+    # product on its own (a different lane, or no fused multiply-add) loses 2^-30.
     x = np.zeros((1, H), np.float32)
     W = np.zeros((1, H), np.float32)
-    x[0, 0], W[0, 0] = -1.0, 1.0 + 2.0 ** -7
-    x[0, 32], W[0, 32] = 1.0 + 2.0 ** -7, 1.0 + 2.0 ** -23
-    l = oracle.router_logits(_bf16_bits(x), W, None, nthreads=1)[0, 0]
-    assert l == np.float32(2.0 ** -23 + 2.0 ** -30)
+    x[0, h0], W[0, h0] = -1.0, 1.0 + 2.0 ** -7
+    x[0, h1], W[0, h1] = 1.0 + 2.0 ** -7, 1.0 + 2.0 ** -23
+    return oracle.router_logits(_bf16_bits(x), W, None, nthreads=1)[0, 0]
+
+
+def test_logit_lane_partial_uses_fused_multiply_add():
+    # h = 0 and h = 1 are consecutive in lane 0's chain: p = fma(x1, w1, fma(x0, w0, 0)).
+    assert _cancelling_pair(128, 0, 1) == np.float32(2.0 ** -23 + 2.0 ** -30)
     assert np.float32(2.0 ** -23 + 2.0 ** -30) != np.float32(2.0 ** -23)
+
+
+def test_logit_chain_takes_four_consecutive_h_per_128_block():
+    # lane 0's chain continues from h = 3 (end of its first group of four) to h = 128 (start of its
+    # group in the next 128-wide block): the pair still cancels inside one fused chain
+    assert _cancelling_pair(256, 3, 128) == np.float32(2.0 ** -23 + 2.0 ** -30)
+    # h = 4 and h = 32 belong to lanes 1 and 8: the second product is rounded before the lanes meet
+    assert _cancelling_pair(128, 4, 32) == np.float32(2.0 ** -23)
 
 
 def test_logits_within_fp32_bound_of_exact():
