@@ -124,38 +124,44 @@ __device__ void group_offsets(const int32_t* __restrict__ kept, int E, int maske
     __syncthreads();
 }
 
-// v[i] <- v[i] / s correctly rounded to fp32 (s > 0), without a division per element:
-// Markstein's correction step (P. Markstein, "Computation of elementary functions on the
-// IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with r = 1/s correctly
-// rounded, q0 = v * r rounded, the remainder v - q0 * s is exact in one fused multiply-add
-// and q0 + remainder * r, rounded once, is the correctly rounded quotient, as long as no
-// intermediate leaves the normal range. Zeros keep their sign; lanes whose values are
-// tiny (|v| < 2^-96 or |v / s| < 2^-100) take the correctly rounded division instead.
-__device__ __forceinline__ void quotients_rn(float (&v)[8], float s) {
+// Scale and codes of one 1x128 group without a division per value. Markstein's correction step
+// (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000 processor",
+// IBM J. Res. Dev. 34(1), 1990): with y = 1/b correctly rounded and q0 = a * y rounded, the
+// remainder a - q0 * b is exact in one fused multiply-add and q0 + remainder * y, rounded once, is
+// the correctly rounded quotient a / b, as long as no intermediate leaves the normal range. It
+// gives s = amax / 448 (y = 1/448 rounded, a compile-time constant) and each v / s (y = 1/s from the
+// correctly rounded reciprocal). For amax in [2^-60, 2^128) every quotient that can reach an E4M3
+// code (|v / s| >= 2^-10) has v >= 2^-79, far inside the normal range; smaller quotients round to a
+// signed zero code, and their sign is v's, which is restored explicitly (the correction would turn
+// -0 into +0). Checked against C's correctly rounded division on 4e8 bf16 value / scale pairs with
+// amax over 2^-100 .. 2^126 (the only difference needs amax near 2^-100) and by the bit-exact parity
+// tests. Groups outside that range take the correctly rounded division, out of line.
+__device__ __noinline__ float quantise_group_div(float (&v)[8], float amax) {
+    const float s = __fdiv_rn(amax, 448.0f);
+    for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(v[i], s);
+    return s;
+}
+
+__device__ __forceinline__ float quantise_group(float (&v)[8], float amax) {
+    if (amax == 0.0f) return 1.0f;                       // all values are (signed) zeros: codes of v itself
+    if (!(amax >= 0x1p-60f && amax < 0x1p128f)) return quantise_group_div(v, amax);
+    constexpr float kInv448 = 1.0f / 448.0f;
+    const float s0 = amax * kInv448;
+    const float s = fmaf(fmaf(-s0, 448.0f, amax), kInv448, s0);
     const float r = __frcp_rn(s);
-    float q[8];
-    bool normal = true;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const float q0 = v[i] * r;
-        const float rem = fmaf(-q0, s, v[i]);
-        q[i] = fmaf(rem, r, q0);
-        if (v[i] == 0.0f) q[i] = v[i];
-        else normal = normal && fabsf(v[i]) >= 0x1p-96f && fabsf(q[i]) >= 0x1p-100f;
+        const float q = fmaf(fmaf(-q0, s, v[i]), r, q0);
+        v[i] = __uint_as_float((__float_as_uint(q) & 0x7fffffffu) | (__float_as_uint(v[i]) & 0x80000000u));
     }
-    if (normal) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = q[i];
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(v[i], s);
-    }
+    return s;
 }
 
 // blockIdx.x < nchunks: scatter one 32-token chunk (slot maps + quantised rows);
 // blockIdx.x >= nchunks (contiguous layout only): fill expert (x - nchunks)'s padding rows.
 // blockIdx.y selects a slice of the H/128 quantisation groups.
-__global__ void __launch_bounds__(256) permute_scatter_kernel(
+__global__ void __launch_bounds__(256, 3) permute_scatter_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, int T, int H, int k, int E, int nchunks,
     int masked_max_m, int ld_rows, const int32_t* __restrict__ base, const int32_t* __restrict__ kept,
     uint8_t* __restrict__ Aq, float* __restrict__ As, int32_t* __restrict__ offsets, int32_t* __restrict__ row_src,
@@ -267,7 +273,6 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
         uint2 code[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            sc[u] = amax[u] == 0.0f ? 1.0f : __fdiv_rn(amax[u], 448.0f);
             const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
             float v[8];
 #pragma unroll
@@ -275,7 +280,7 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
                 v[2 * i] = __uint_as_float(w[i] << 16);
                 v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
             }
-            quotients_rn(v, sc[u]);
+            sc[u] = quantise_group(v, amax[u]);
             code[u].x = f32x2_to_e4m3x2(v[0], v[1]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[2], v[3])) << 16);
             code[u].y = f32x2_to_e4m3x2(v[4], v[5]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[6], v[7])) << 16);
         }
