@@ -10,7 +10,7 @@
 // (j with j^16, then ^8, ^4, ^2, ^1), which pairs j with j+16 first, then
 // j+8, ... exactly; the bias is added last.
 //
-// The logits kernel tiles tokens x experts: a producer thread streams 128-wide
+// The logits kernel tiles tokens x experts: one thread streams 128-wide
 // blocks of x ([tokens, h], bf16) and W_g ([experts, h], fp32) with TMA into a
 // ring of shared-memory stages, row-major as they lie in global memory, and
 // each compute warp keeps a TR x ER register tile per lane, so every 16-byte
@@ -24,15 +24,14 @@ namespace moe {
 
 constexpr int kRouterHS = 128;     // h values per stage: lane j takes h = 4j .. 4j+3 of each
 
-template <int TR, int ER, int WT, int WE>
+// DP: a dedicated producer warp issues the loads (small tiles, where the compute warps are few and
+// quick); otherwise thread 0, a compute thread, refills each stage's slot as soon as every warp is done.
+template <int TR, int ER, int WT, int WE, bool DP>
 struct RouterCfg {
     static constexpr int TT = TR * WT;                  // tokens per CTA
     static constexpr int EC = ER * WE;                  // experts per CTA
-    static constexpr int kCompute = WT * WE;            // compute warps, after the producer warpgroup
-    static constexpr int kThreads = 32 * (kCompute + 4);
-    // large register tiles: the producer warpgroup gives registers to the compute warps
-    static constexpr bool kSplit = TR * ER >= 128;
-    static constexpr int kRegsLow = 40, kRegsHigh = 232;
+    static constexpr int kWarps = WT * WE;              // compute warps
+    static constexpr int kThreads = 32 * (kWarps + (DP ? 1 : 0));
     static constexpr int kXBytes = TT * kRouterHS * 2;
     static constexpr int kWBytes = EC * kRouterHS * 4;
     static constexpr int kStageBytes = kXBytes + kWBytes;
@@ -40,96 +39,107 @@ struct RouterCfg {
     static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8 + 16 + 1024;
 };
 
-template <int TR, int ER, int WT, int WE>
-__global__ void __launch_bounds__(RouterCfg<TR, ER, WT, WE>::kThreads, 1)
+template <int TR, int ER, int WT, int WE, bool DP>
+__global__ void __launch_bounds__(RouterCfg<TR, ER, WT, WE, DP>::kThreads, 1)
 router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ bias, float* __restrict__ logits, int T, int H, int E, int* status,
                      uint64_t wait_ns) {
-    using C = RouterCfg<TR, ER, WT, WE>;
+    using C = RouterCfg<TR, ER, WT, WE, DP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
     uint64_t* empty = full + C::kStages;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::kStages);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31;
+    const int warp = (threadIdx.x >> 5) - (DP ? 1 : 0);             // compute warp index; -1: producer warp
+    const int wt = warp / WE, we = warp % WE;
     const int t_base = blockIdx.x * C::TT, e_base = blockIdx.y * C::EC;
     const int nst = H / kRouterHS;
+    const bool producer = threadIdx.x == 0;
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], C::kCompute);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
     auto fail = [&]() {
         set_status(status, kStatusTimeout);
         *abort_flag = 1;
     };
+    auto issue = [&](int st) {      // stage st into slot st % kStages
+        const int s = st % C::kStages;
+        uint8_t* stage = smem + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+        tma_load_2d(stage, &tmX, &full[s], st * kRouterHS, t_base);
+        tma_load_2d(stage + C::kXBytes, &tmW, &full[s], st * kRouterHS, e_base);
+    };
+    if (producer) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], C::kWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmX);
+        prefetch_tensormap(&tmW);
+        for (int st = 0; st < C::kStages && st < nst; ++st) issue(st);
+    }
+    __syncthreads();
 
-    if (warp < 4) {
-        if constexpr (C::kSplit) setmaxnreg_dec<C::kRegsLow>();
-        if (warp == 0 && lane == 0) {
-            prefetch_tensormap(&tmX);
-            prefetch_tensormap(&tmW);
-            for (int st = 0; st < nst && !*abort_flag; ++st) {
-                const int s = st % C::kStages;
-                if (!mbar_wait(&empty[s], ((st / C::kStages) & 1) ^ 1, wait_ns)) { fail(); break; }
-                uint8_t* stage = smem + s * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-                tma_load_2d(stage, &tmX, &full[s], st * kRouterHS, t_base);
-                tma_load_2d(stage + C::kXBytes, &tmW, &full[s], st * kRouterHS, e_base);
+    if (DP && warp < 0) {
+        // dedicated producer: refill each slot as soon as every compute warp has finished with it
+        if (producer)
+            for (int st = C::kStages; st < nst && !*abort_flag; ++st) {
+                const int u = st / C::kStages - 1;
+                if (!mbar_wait(&empty[st % C::kStages], u & 1, wait_ns)) { fail(); break; }
+                issue(st);
+            }
+        __syncthreads();
+        return;
+    }
+    float acc[TR][ER];
+#pragma unroll
+    for (int i = 0; i < TR; ++i)
+#pragma unroll
+        for (int q = 0; q < ER; ++q) acc[i][q] = 0.0f;
+    bool ok = true;
+    for (int st = 0; st < nst; ++st) {
+        // the slot of stage st - 1 takes stage st - 1 + kStages once every warp has finished with it
+        if (!DP && producer && st > 0 && st - 1 + C::kStages < nst) {
+            if (!mbar_wait(&empty[(st - 1) % C::kStages], ((st - 1) / C::kStages) & 1, wait_ns)) fail();
+            else issue(st - 1 + C::kStages);
+        }
+        const int s = st % C::kStages;
+        if (*abort_flag || !mbar_wait(&full[s], (st / C::kStages) & 1, wait_ns)) { fail(); ok = false; break; }
+        const uint8_t* stage = smem + s * C::kStageBytes;
+        const uint16_t* xs = reinterpret_cast<const uint16_t*>(stage) + (wt * TR) * kRouterHS + 4 * lane;
+        const float* ws = reinterpret_cast<const float*>(stage + C::kXBytes) + (we * ER) * kRouterHS + 4 * lane;
+        float4 wv[ER];
+#pragma unroll
+        for (int q = 0; q < ER; ++q) wv[q] = *reinterpret_cast<const float4*>(ws + q * kRouterHS);
+#pragma unroll
+        for (int i = 0; i < TR; ++i) {
+            const uint2 xr = *reinterpret_cast<const uint2*>(xs + i * kRouterHS);
+            const float x0 = __uint_as_float(xr.x << 16), x1 = __uint_as_float(xr.x & 0xffff0000u);
+            const float x2 = __uint_as_float(xr.y << 16), x3 = __uint_as_float(xr.y & 0xffff0000u);
+            // lane j's chain for (token, expert) runs over h = 4j, 4j+1, 4j+2, 4j+3 of this block in order
+#pragma unroll
+            for (int q = 0; q < ER; ++q) {
+                acc[i][q] = fmaf(x0, wv[q].x, acc[i][q]);
+                acc[i][q] = fmaf(x1, wv[q].y, acc[i][q]);
+                acc[i][q] = fmaf(x2, wv[q].z, acc[i][q]);
+                acc[i][q] = fmaf(x3, wv[q].w, acc[i][q]);
             }
         }
-    } else {
-        if constexpr (C::kSplit) setmaxnreg_inc<C::kRegsHigh>();
-        const int cw = warp - 4, wt = cw / WE, we = cw % WE;
-        float acc[TR][ER];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (ok) {
 #pragma unroll
-        for (int i = 0; i < TR; ++i)
+        for (int i = 0; i < TR; ++i) {
 #pragma unroll
-            for (int q = 0; q < ER; ++q) acc[i][q] = 0.0f;
-        bool ok = true;
-        for (int st = 0; st < nst; ++st) {
-            const int s = st % C::kStages;
-            if (*abort_flag || !mbar_wait(&full[s], (st / C::kStages) & 1, wait_ns)) { fail(); ok = false; break; }
-            const uint8_t* stage = smem + s * C::kStageBytes;
-            const uint16_t* xs = reinterpret_cast<const uint16_t*>(stage) + (wt * TR) * kRouterHS + 4 * lane;
-            const float* ws = reinterpret_cast<const float*>(stage + C::kXBytes) + (we * ER) * kRouterHS + 4 * lane;
-            float4 wv[ER];
+            for (int q = 0; q < ER; ++q) {
+                float v = acc[i][q];
 #pragma unroll
-            for (int q = 0; q < ER; ++q) wv[q] = *reinterpret_cast<const float4*>(ws + q * kRouterHS);
-#pragma unroll
-            for (int i = 0; i < TR; ++i) {
-                const uint2 xr = *reinterpret_cast<const uint2*>(xs + i * kRouterHS);
-                const float x0 = __uint_as_float(xr.x << 16), x1 = __uint_as_float(xr.x & 0xffff0000u);
-                const float x2 = __uint_as_float(xr.y << 16), x3 = __uint_as_float(xr.y & 0xffff0000u);
-                // lane j's chain for (token, expert) runs over h = 4j, 4j+1, 4j+2, 4j+3 of this block in order
-#pragma unroll
-                for (int q = 0; q < ER; ++q) {
-                    acc[i][q] = fmaf(x0, wv[q].x, acc[i][q]);
-                    acc[i][q] = fmaf(x1, wv[q].y, acc[i][q]);
-                    acc[i][q] = fmaf(x2, wv[q].z, acc[i][q]);
-                    acc[i][q] = fmaf(x3, wv[q].w, acc[i][q]);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-        }
-        if (ok) {
-#pragma unroll
-            for (int i = 0; i < TR; ++i) {
-#pragma unroll
-                for (int q = 0; q < ER; ++q) {
-                    float v = acc[i][q];
-#pragma unroll
-                    for (int o = 16; o >= 1; o >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
-                    const int t = t_base + wt * TR + i, e = e_base + we * ER + q;
-                    if (lane == ((i * ER + q) & 31) && t < T && e < E)
-                        logits[static_cast<int64_t>(t) * E + e] = bias ? v + bias[e] : v;
-                }
+                for (int o = 16; o >= 1; o >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
+                const int t = t_base + wt * TR + i, e = e_base + we * ER + q;
+                if (lane == ((i * ER + q) & 31) && t < T && e < E)
+                    logits[static_cast<int64_t>(t) * E + e] = bias ? v + bias[e] : v;
             }
         }
     }
@@ -225,26 +235,17 @@ static bool make_router_map(CUtensorMap* m, CUtensorMapDataType dt, int elem_byt
            CUDA_SUCCESS;
 }
 
-template <int TR, int ER, int WT, int WE>
+template <int TR, int ER, int WT, int WE, bool DP>
 static cudaError_t launch_logits(const uint16_t* x, const float* Wg, const float* bias, float* logits, int T, int H,
                                  int E, int* status, uint64_t wait_ns, cudaStream_t s) {
-    using C = RouterCfg<TR, ER, WT, WE>;
+    using C = RouterCfg<TR, ER, WT, WE, DP>;
     CUtensorMap mx, mw;
     if (!make_router_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, H, T, C::TT) ||
         !make_router_map(&mw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, Wg, H, E, C::EC))
         return cudaErrorInvalidValue;
-    auto kern = router_logits_kernel<TR, ER, WT, WE>;
+    auto kern = router_logits_kernel<TR, ER, WT, WE, DP>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (err != cudaSuccess) return err;
-    if constexpr (C::kSplit) {
-        // setmaxnreg.inc can only hand out registers the block was launched with: refuse a build whose
-        // launch allocation is smaller than the split instead of starting it
-        cudaFuncAttributes a;
-        err = cudaFuncGetAttributes(&a, kern);
-        if (err != cudaSuccess) return err;
-        if (a.numRegs * C::kThreads < 128 * C::kRegsLow + (C::kThreads - 128) * C::kRegsHigh)
-            return cudaErrorInvalidConfiguration;
-    }
     dim3 grid((T + C::TT - 1) / C::TT, (E + C::EC - 1) / C::EC);
     kern<<<grid, C::kThreads, C::kSmem, s>>>(mx, mw, bias, logits, T, H, E, status, wait_ns);
     return cudaGetLastError();
@@ -258,11 +259,11 @@ cudaError_t launch_router_softmax(const uint16_t* x, const float* Wg, const floa
     const long ctas_big = static_cast<long>((T + 31) / 32) * ((E + 31) / 32);
     const long ctas_mid = static_cast<long>((T + 15) / 16) * ((E + 15) / 16);
     if (ctas_big >= num_sms)
-        err = launch_logits<16, 8, 2, 4>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);   // 32 tokens x 32 experts
+        err = launch_logits<8, 8, 4, 4, false>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);  // 32 tokens x 32 experts
     else if (ctas_mid >= num_sms)
-        err = launch_logits<8, 4, 2, 4>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);    // 16 tokens x 16 experts
+        err = launch_logits<8, 4, 2, 4, true>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);   // 16 tokens x 16 experts
     else
-        err = launch_logits<8, 4, 1, 4>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);    // 8 tokens x 16 experts
+        err = launch_logits<8, 4, 1, 4, true>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);   // 8 tokens x 16 experts
     if (err != cudaSuccess) return err;
     const int blocks = (T + 7) / 8;
     if (E <= 64)
