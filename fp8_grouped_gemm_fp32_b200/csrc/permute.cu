@@ -13,6 +13,8 @@
 // of the chunk's tokens chose the expert (atomicOr commutes). A slot's rank
 // in its expert = the expert's count in earlier chunks (an exclusive scan
 // over chunks) + the popcount of the mask bits below the token's lane.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -135,16 +137,42 @@ __device__ void group_offsets(const int32_t* __restrict__ kept, int E, int maske
 // signed zero code, and their sign is v's, which is restored explicitly (the correction would turn
 // -0 into +0). Checked against C's correctly rounded division on 4e8 bf16 value / scale pairs with
 // amax over 2^-100 .. 2^126 (the only difference needs amax near 2^-100) and by the bit-exact parity
-// tests. Groups outside that range take the correctly rounded division, out of line.
-__device__ __noinline__ float quantise_group_div(float (&v)[8], float amax) {
-    const float s = __fdiv_rn(amax, 448.0f);
-    for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(v[i], s);
-    return s;
+// tests. Groups outside that range take the correctly rounded division, out of line (its arguments
+// and results pass by value, so the common path keeps its values in registers).
+struct GroupCodes {
+    uint2 code;     // 8 E4M3 codes, the first value in the lowest byte
+    float scale;
+};
+
+__device__ __forceinline__ uint2 pack_e4m3x8(const float (&v)[8]) {
+    return make_uint2(f32x2_to_e4m3x2(v[0], v[1]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[2], v[3])) << 16),
+                      f32x2_to_e4m3x2(v[4], v[5]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[6], v[7])) << 16));
 }
 
-__device__ __forceinline__ float quantise_group(float (&v)[8], float amax) {
-    if (amax == 0.0f) return 1.0f;                       // all values are (signed) zeros: codes of v itself
-    if (!(amax >= 0x1p-60f && amax < 0x1p128f)) return quantise_group_div(v, amax);
+__device__ __forceinline__ void unpack_bf16x8(uint4 raw, float (&v)[8]) {
+    const uint32_t q[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(q[i] << 16);
+        v[2 * i + 1] = __uint_as_float(q[i] & 0xffff0000u);
+    }
+}
+
+__device__ __noinline__ GroupCodes quantise_group_div(uint4 raw, float amax) {
+    float v[8];
+    unpack_bf16x8(raw, v);
+    const float s = __fdiv_rn(amax, 448.0f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(v[i], s);
+    return GroupCodes{pack_e4m3x8(v), s};
+}
+
+// Codes and scale of a lane's 8 values (bf16, packed in raw) of a group whose max |value| is amax.
+__device__ __forceinline__ GroupCodes quantise_group(uint4 raw, float amax) {
+    float v[8];
+    unpack_bf16x8(raw, v);
+    if (amax == 0.0f) return GroupCodes{pack_e4m3x8(v), 1.0f};   // all (signed) zeros: codes of v itself
+    if (!(amax >= 0x1p-60f && amax < 0x1p128f)) return quantise_group_div(raw, amax);
     constexpr float kInv448 = 1.0f / 448.0f;
     const float s0 = amax * kInv448;
     const float s = fmaf(fmaf(-s0, 448.0f, amax), kInv448, s0);
@@ -155,34 +183,33 @@ __device__ __forceinline__ float quantise_group(float (&v)[8], float amax) {
         const float q = fmaf(fmaf(-q0, s, v[i]), r, q0);
         v[i] = __uint_as_float((__float_as_uint(q) & 0x7fffffffu) | (__float_as_uint(v[i]) & 0x80000000u));
     }
-    return s;
+    return GroupCodes{pack_e4m3x8(v), s};
 }
 
-// blockIdx.x < nchunks: scatter one 32-token chunk (slot maps + quantised rows);
-// blockIdx.x >= nchunks (contiguous layout only): fill expert (x - nchunks)'s padding rows.
-// blockIdx.y selects a slice of the H/128 quantisation groups.
-__global__ void __launch_bounds__(256, 3) permute_scatter_kernel(
-    const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, int T, int H, int k, int E, int nchunks,
-    int masked_max_m, int ld_rows, const int32_t* __restrict__ base, const int32_t* __restrict__ kept,
-    uint8_t* __restrict__ Aq, float* __restrict__ As, int32_t* __restrict__ offsets, int32_t* __restrict__ row_src,
+// blockIdx.x < nchunks: the slot maps of one 32-token chunk (slot_row, row_src);
+// blockIdx.x >= nchunks (contiguous layout only): the padding rows of one expert, one slice of
+// pad_slices of its 128-groups (codes 0, scale 1, row_src -1). Block 0 also writes offsets.
+__global__ void __launch_bounds__(256) permute_map_kernel(
+    const int32_t* __restrict__ topk_idx, int T, int H, int k, int E, int nchunks, int pad_slices, int masked_max_m,
+    int ld_rows, const int32_t* __restrict__ base, const int32_t* __restrict__ kept, uint8_t* __restrict__ Aq,
+    float* __restrict__ As, int32_t* __restrict__ offsets, int32_t* __restrict__ row_src,
     int32_t* __restrict__ slot_row) {
     extern __shared__ int32_t sm[];
     int32_t* off_s = sm;                    // [E + 1]
     int32_t* kept_s = off_s + (E + 1);      // [E]
     uint32_t* masks = reinterpret_cast<uint32_t*>(kept_s + E);   // [E]
-    int32_t* dest = reinterpret_cast<int32_t*>(masks + E);        // [32][k]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = H / kGroup;
-    const int gpy = (G + gridDim.y - 1) / gridDim.y;
-    const int g0 = blockIdx.y * gpy, g1 = min(G, g0 + gpy);
-    const bool masked = masked_max_m > 0;
 
     group_offsets(kept, E, masked_max_m, off_s, kept_s);
-    if (blockIdx.x == 0 && blockIdx.y == 0)
+    if (blockIdx.x == 0)
         for (int e = tid; e <= E; e += blockDim.x) offsets[e] = off_s[e];
 
     if (blockIdx.x >= nchunks) {            // padding rows of one expert (contiguous layout)
-        const int e = blockIdx.x - nchunks;
+        const int e = (blockIdx.x - nchunks) / pad_slices, sl = (blockIdx.x - nchunks) % pad_slices;
+        const int gps = (G + pad_slices - 1) / pad_slices;
+        const int g0 = sl * gps, g1 = min(G, g0 + gps);
+        if (g0 >= g1) return;
         const int r0 = off_s[e] + kept_s[e], r1 = off_s[e + 1];
         const int per_row = (g1 - g0) * (kGroup / 16);           // 16-byte pieces per row slice
         for (int i = tid; i < (r1 - r0) * per_row; i += blockDim.x) {
@@ -193,7 +220,7 @@ __global__ void __launch_bounds__(256, 3) permute_scatter_kernel(
             const int r = r0 + i / (g1 - g0), g = g0 + i % (g1 - g0);
             As[static_cast<int64_t>(g) * ld_rows + r] = 1.0f;
         }
-        if (blockIdx.y == 0)
+        if (sl == 0)
             for (int r = r0 + tid; r < r1; r += blockDim.x) row_src[r] = -1;
         return;
     }
@@ -208,61 +235,59 @@ __global__ void __launch_bounds__(256, 3) permute_scatter_kernel(
             if (e >= 0 && e < E) atomicOr(&masks[e], 1u << lane);
         }
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 0 && t_lane < T) {
         for (int j = 0; j < k; ++j) {
             int32_t row = -1;
-            if (t_lane < T) {
-                const int e = topk_idx[static_cast<int64_t>(t_lane) * k + j];
-                if (e >= 0 && e < E) {   // an out-of-range expert index is treated as dropped
-                    const int32_t rank =
-                        base[static_cast<int64_t>(e) * nchunks + c] + __popc(masks[e] & ((1u << lane) - 1u));
-                    if (rank < kept_s[e]) row = off_s[e] + rank;
-                }
-                if (blockIdx.y == 0) {
-                    const int64_t s = static_cast<int64_t>(t_lane) * k + j;
-                    slot_row[s] = row;
-                    if (row >= 0) row_src[row] = static_cast<int32_t>(s);
-                }
+            const int e = topk_idx[static_cast<int64_t>(t_lane) * k + j];
+            if (e >= 0 && e < E) {   // an out-of-range expert index is treated as dropped
+                const int32_t rank =
+                    base[static_cast<int64_t>(e) * nchunks + c] + __popc(masks[e] & ((1u << lane) - 1u));
+                if (rank < kept_s[e]) row = off_s[e] + rank;
             }
-            dest[lane * k + j] = row;
+            const int64_t s = static_cast<int64_t>(t_lane) * k + j;
+            slot_row[s] = row;
+            if (row >= 0) row_src[row] = static_cast<int32_t>(s);
         }
     }
-    __syncthreads();
+}
 
-    // quantise: warp w takes the (token, group) items of tokens w, w + 8, w + 16, w + 24 of the chunk,
-    // 2U per pass: a half-warp per item, 8 values (16 bytes) per lane. Each phase runs over all
-    // U items of a lane before the next, so the loads, the max butterflies, the divisions and
-    // the stores of different items overlap.
+// Quantise x once per token and 1x128 group and write the codes and the scale to every kept
+// destination row of the token (slot_row). A warp takes one token and up to 8 of its groups, a
+// half-warp per group with 8 values (one 16-byte load) per lane, all four loads of a lane in flight
+// together; warps stride over (token, 8-group slice) items.
+__global__ void __launch_bounds__(256, 4) permute_quant_kernel(
+    const uint16_t* __restrict__ x, int T, int H, int k, int masked_max_m, int ld_rows,
+    const int32_t* __restrict__ slot_row, uint8_t* __restrict__ Aq, float* __restrict__ As) {
     constexpr int U = 4;
-    const int hl = lane & 15, hw = lane >> 4;
-    const int gs = g1 - g0;
-    const int ntok = min(kChunk, T - c * kChunk);
-    const int my_tok = ntok > warp ? (ntok - warp + 7) / 8 : 0;
-    const int my_items = my_tok * gs;
-    const uint32_t inv_gs = (65536u + gs - 1) / gs;          // it / gs == (it * inv_gs) >> 16 for it < 2^16 / 64
-    for (int p0 = 0; p0 < my_items; p0 += 2 * U) {
+    const int lane = threadIdx.x & 31, hl = lane & 15, hw = lane >> 4;
+    const int G = H / kGroup;
+    const int nsl = (G + 2 * U - 1) / (2 * U);
+    const bool masked = masked_max_m > 0;
+    const int64_t items = static_cast<int64_t>(T) * nsl;
+    for (int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < items;
+         w += static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5)) {
+        const int t = static_cast<int>(w / nsl);
+        const int g0 = static_cast<int>(w % nsl) * 2 * U;
+        const uint16_t* xrow = x + static_cast<int64_t>(t) * H;
+        // the token's destination rows load alongside its values (up to 8 here; more in the store loop)
+        constexpr int KR = 8;
+        int32_t rows[KR];
+#pragma unroll
+        for (int j = 0; j < KR; ++j) rows[j] = j < k ? slot_row[static_cast<int64_t>(t) * k + j] : -1;
         uint4 raw[U];
-        int row_r[U], grp[U];
-        bool live[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int it = p0 + 2 * u + hw;
-            const int q = static_cast<int>((static_cast<uint32_t>(it) * inv_gs) >> 16);
-            live[u] = it < my_items;
-            row_r[u] = warp + 8 * q;
-            grp[u] = g0 + it - q * gs;
-            raw[u] = live[u] ? *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(c * kChunk + row_r[u]) * H +
-                                                               grp[u] * kGroup + hl * 8)
-                             : make_uint4(0, 0, 0, 0);
+            const int g = g0 + 2 * u + hw;
+            raw[u] = g < G ? *reinterpret_cast<const uint4*>(xrow + g * kGroup + hl * 8) : make_uint4(0, 0, 0, 0);
         }
         float amax[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+            const uint32_t q[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
             float m = 0.0f;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xffff0000u))));
+                m = fmaxf(m, fmaxf(fabsf(__uint_as_float(q[i] << 16)), fabsf(__uint_as_float(q[i] & 0xffff0000u))));
             amax[u] = m;
         }
 #pragma unroll
@@ -273,30 +298,28 @@ __global__ void __launch_bounds__(256, 3) permute_scatter_kernel(
         uint2 code[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-            float v[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                v[2 * i] = __uint_as_float(w[i] << 16);
-                v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-            }
-            sc[u] = quantise_group(v, amax[u]);
-            code[u].x = f32x2_to_e4m3x2(v[0], v[1]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[2], v[3])) << 16);
-            code[u].y = f32x2_to_e4m3x2(v[4], v[5]) | (static_cast<uint32_t>(f32x2_to_e4m3x2(v[6], v[7])) << 16);
+            const GroupCodes gc = quantise_group(raw[u], amax[u]);
+            code[u] = gc.code;
+            sc[u] = gc.scale;
         }
+        for (int j = 0; j < k; ++j) {
+            int32_t row = -1;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            if (!live[u]) continue;
-            for (int j = 0; j < k; ++j) {
-                const int32_t row = dest[row_r[u] * k + j];
-                if (row < 0) continue;
-                *reinterpret_cast<uint2*>(Aq + static_cast<int64_t>(row) * H + grp[u] * kGroup + hl * 8) = code[u];
+            for (int i = 0; i < KR; ++i)
+                if (i == j) row = rows[i];
+            if (j >= KR) row = slot_row[static_cast<int64_t>(t) * k + j];
+            if (row < 0) continue;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int g = g0 + 2 * u + hw;
+                if (g >= G) continue;
+                *reinterpret_cast<uint2*>(Aq + static_cast<int64_t>(row) * H + g * kGroup + hl * 8) = code[u];
                 if (hl == 0) {
                     if (masked) {
                         const int e = row / masked_max_m, rr = row - e * masked_max_m;
-                        As[(static_cast<int64_t>(e) * G + grp[u]) * masked_max_m + rr] = sc[u];
+                        As[(static_cast<int64_t>(e) * G + g) * masked_max_m + rr] = sc[u];
                     } else {
-                        As[static_cast<int64_t>(grp[u]) * ld_rows + row] = sc[u];
+                        As[static_cast<int64_t>(g) * ld_rows + row] = sc[u];
                     }
                 }
             }
@@ -319,18 +342,22 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, int T, in
     permute_count_kernel<<<(nchunks + 7) / 8, 256, 8 * E * sizeof(uint32_t), s>>>(topk_idx, T, k, E, nchunks, cnt);
     permute_scan_kernel<<<E, 256, 0, s>>>(cnt, nchunks, cap, masked_max_m, base, counts, kept, status);
     const int G = H / kGroup;
-    const int gx = nchunks + (masked_max_m > 0 ? 0 : E);
-    const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1 + kChunk * k);
-    // as many group slices per chunk as keep every block resident at once (one wave)
+    // padding blocks: slices of four 128-groups per expert, so a block fills about 32 KB (64 rows)
+    const int pad_slices = masked_max_m > 0 ? 1 : (G + 3) / 4;
+    const int gx = nchunks + (masked_max_m > 0 ? 0 : E * pad_slices);
+    const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1);
+    permute_map_kernel<<<gx, 256, smem, s>>>(topk_idx, T, H, k, E, nchunks, pad_slices, masked_max_m, ld_rows, base,
+                                             kept, Aq, As, offsets, row_src, slot_row);
+    // one warp per (token, 8-group slice); enough blocks to keep every SM full, striding beyond that
+    const int64_t warps = static_cast<int64_t>(T) * ((G + 7) / 8);
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_scatter_kernel, 256, smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_quant_kernel, 256, 0) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
-    int gy = per_sm * num_sms / gx;
-    gy = gy < 1 ? 1 : (gy > G ? G : gy);
-    gy = (G + (G + gy - 1) / gy - 1) / ((G + gy - 1) / gy);   // no empty group slices
-    permute_scatter_kernel<<<dim3(gx, gy), 256, smem, s>>>(x, topk_idx, T, H, k, E, nchunks, masked_max_m, ld_rows,
-                                                           base, kept, Aq, As, offsets, row_src, slot_row);
+    const int64_t cap_blocks = static_cast<int64_t>(per_sm) * num_sms * 4;
+    const int blocks = static_cast<int>(std::min<int64_t>((warps + 7) / 8, cap_blocks));
+    if (blocks > 0)
+        permute_quant_kernel<<<blocks, 256, 0, s>>>(x, T, H, k, masked_max_m, ld_rows, slot_row, Aq, As);
     return cudaGetLastError();
 }
 
