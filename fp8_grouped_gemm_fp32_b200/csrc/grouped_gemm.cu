@@ -36,6 +36,7 @@ namespace moe {
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;
 constexpr int kSaSlots = 8;                   // ring of per-K-block activation scales (128 rows each)
+constexpr int kMaxKB = 128;                   // K <= 16384
 constexpr int kABytes = kBM * kBK;            // 16 KB
 constexpr int kBBytes = kBN * kBK;            // 32 KB
 constexpr int kThreadsC = 384;                // 12 warps
@@ -58,8 +59,11 @@ struct SmemC {
     uint8_t b[kStages][kBBytes];
     uint8_t out[EPI == 0 ? kOutStageBytes : 8 * kOutBoxBytes];
     float sa[kSaSlots][kBM];    // activation scales of one K block for the tile's 128 rows
+    float wsc[2][2][kMaxKB];    // weight-block scales of a tile (two tiles in flight): [tile & 1][block][kb]
     uint64_t full[kStages];
     uint64_t empty[kStages];
+    uint64_t wfull[2];
+    uint64_t wempty[2];
     uint64_t sfull[kSaSlots];
     uint64_t sempty[kSaSlots];
     uint64_t tfull[2];
@@ -134,6 +138,8 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             mbar_init(&sm.tfull[b], 1);
             mbar_init(&sm.tempty[b], 8);
             mbar_init(&sm.red_bar[b], 256);
+            mbar_init(&sm.wfull[b], 1);
+            mbar_init(&sm.wempty[b], 8);
         }
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -159,18 +165,65 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (warp < 4) {
       setmaxnreg_dec<kRegsLow>();
       if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- producer: TMA loads (lane 0) and, per tile, the weight-block scales (all lanes)
         if (lane == 0) {
             prefetch_tensormap(&tmA);
             prefetch_tensormap(&tmB);
-            uint32_t it = 0;
-            for (int tile = blockIdx.x; tile < total && !sm.abort_flag; tile += gridDim.x) {
-                const TileC t = decode_tile_c(sm.P, E, NT, N, tile);
+        }
+        // A tile's 2 x KB weight-block scales go to slot (tile index) & 1, freed when the promotion warps
+        // finish the tile two before. The next tile's scales are read into registers while this tile's
+        // loads are issued, so their latency stays off the TMA stream.
+        float wr0[4], wr1[4];
+        auto read_scales = [&](const TileC& u) {
+            const float* b0 = Bs + (static_cast<int64_t>(u.e) * NB + u.n0 / kBM) * KB;
+            const float* b1 = u.width == kBN ? b0 + KB : b0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int kb = lane + 32 * i;
+                wr0[i] = kb < KB ? b0[kb] : 0.0f;
+                wr1[i] = kb < KB ? b1[kb] : 0.0f;
+            }
+        };
+        auto publish_scales = [&](uint32_t ti) -> bool {
+            const int ws = ti & 1;
+            int ok = 1;
+            if (lane == 0) ok = !sm.abort_flag && mbar_wait(&sm.wempty[ws], ((ti >> 1) & 1) ^ 1, wait_ns);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int kb = lane + 32 * i;
+                if (kb < KB) {
+                    sm.wsc[ws][0][kb] = wr0[i];
+                    sm.wsc[ws][1][kb] = wr1[i];
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.wfull[ws]);
+            return true;
+        };
+        uint32_t it = 0, ti = 0;
+        TileC t = decode_tile_c(sm.P, E, NT, N, blockIdx.x);
+        if (blockIdx.x < total) {
+            read_scales(t);
+            if (!publish_scales(0)) {
+                if (lane == 0 && !sm.abort_flag) fail();
+                t.e = -1;
+            }
+        }
+        for (int tile = blockIdx.x; tile < total && t.e >= 0; tile += gridDim.x, ++ti) {
+            const int nxt = tile + gridDim.x;
+            TileC tn = t;
+            if (nxt < total) {
+                tn = decode_tile_c(sm.P, E, NT, N, nxt);
+                read_scales(tn);
+            }
+            int ok = 1;
+            if (lane == 0) {
                 const uint32_t bytes = kABytes + (t.width == kBN ? kBBytes : kBBytes / 2);
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % kStagesC;
                     const uint32_t ph = (it / kStagesC) & 1;
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1, wait_ns)) { fail(); break; }
+                    if (!mbar_wait(&sm.empty[s], ph ^ 1, wait_ns)) { fail(); ok = 0; break; }
                     mbar_arrive_expect_tx(&sm.full[s], bytes);
                     tma_load_2d(sm.a[s], &tmA, &sm.full[s], kb * kBK, t.m0);
                     tma_load_2d(sm.b[s], &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0);
@@ -178,12 +231,18 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         tma_load_2d(sm.b[s] + kBBytes / 2, &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0 + 128);
                     // the 128 activation scales of this K block, into the scale ring
                     const int j = it % kSaSlots;
-                    if (!mbar_wait(&sm.sempty[j], ((it / kSaSlots) & 1) ^ 1, wait_ns)) { fail(); break; }
+                    if (!mbar_wait(&sm.sempty[j], ((it / kSaSlots) & 1) ^ 1, wait_ns)) { fail(); ok = 0; break; }
                     mbar_arrive_expect_tx(&sm.sfull[j], kBM * sizeof(float));
                     bulk_load(sm.sa[j], As + static_cast<int64_t>(kb) * M_rows + t.m0, kBM * sizeof(float),
                               &sm.sfull[j]);
                 }
             }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (nxt < total && !publish_scales(ti + 1)) {
+                if (lane == 0 && !sm.abort_flag) fail();
+                break;
+            }
+            t = tn;
         }
       } else if (warp == 1) {
         // ---------------- MMA issuer
@@ -218,26 +277,14 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int half = (warp - 4) >> 2;       // which 64 columns of each 128-column half
         const int row = q * 32 + lane;          // row within the tile
         uint32_t kbt = 0, ep = 0;
-        // lane l holds the weight-block scales of K blocks l, l + 32, l + 64, l + 96 of the tile's
-        // (up to) two 128-row weight blocks; loaded one tile ahead, so their latency hides behind a tile
-        float wb0[4], wb1[4];
-        auto load_wb = [&](int tile) {
-            if (tile >= total) return;
-            const TileC u = decode_tile_c(sm.P, E, NT, N, tile);
-            const float* b0 = Bs + (static_cast<int64_t>(u.e) * NB + u.n0 / kBM) * KB;
-            const float* b1 = u.width == kBN ? b0 + KB : b0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int kb = lane + 32 * i;
-                wb0[i] = kb < KB ? b0[kb] : 0.0f;
-                wb1[i] = kb < KB ? b1[kb] : 0.0f;
-            }
-        };
-        load_wb(blockIdx.x);
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        uint32_t ti = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++ti) {
             if (sm.abort_flag) break;
             const TileC t = decode_tile_c(sm.P, E, NT, N, tile);
             const bool full = t.width == kBN;
+            // the tile's weight-block scales, staged by the producer warp
+            const int ws = ti & 1;
+            if (!mbar_wait(&sm.wfull[ws], (ti >> 1) & 1, wait_ns)) { fail(); break; }
             // acc2[i] holds columns (2i, 2i+1) of this thread's 128 (64 from each 128-column half)
             float2 acc2[64];
 #pragma unroll
@@ -254,11 +301,8 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const float sa = sm.sa[j][row];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.sempty[j]);
-                const int wi = kb >> 5;
-                const float w0 = __shfl_sync(0xffffffffu, wi == 0 ? wb0[0] : wi == 1 ? wb0[1] : wi == 2 ? wb0[2] : wb0[3],
-                                             kb & 31);
-                const float w1 = __shfl_sync(0xffffffffu, wi == 0 ? wb1[0] : wi == 1 ? wb1[1] : wi == 2 ? wb1[2] : wb1[3],
-                                             kb & 31);
+                const float w0 = sm.wsc[ws][0][kb];
+                const float w1 = sm.wsc[ws][1][kb];
                 const float f0 = sa * w0;
                 const float f1 = sa * w1;
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
@@ -296,7 +340,8 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
             }
             if (!ok) break;
-            load_wb(tile + gridDim.x);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.wempty[ws]);          // the tile's weight scales are no longer read
             const int64_t grow = t.m0 + row;
             if constexpr (EPI == 0) {
                 // this warp's 32 rows x 128 columns as four 32 x 32 boxes: box (r, c) holds columns
