@@ -445,7 +445,11 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 constexpr int kBT = 32;                       // tokens per tile (the MMA's N)
 constexpr int kXBytes = kBT * kBK;            // 4 KB
 constexpr int kWBlk = kBM * kBK;              // 16 KB: 128 weight rows x 128 K bytes
-constexpr int kThreadsM = 192;                // 6 warps
+// threads: warp 0 TMA, warp 1 MMA, then the promotion warps: four for SwiGLU (a thread holds a weight
+// row's 32 gate and 32 up columns), eight for the bf16 output (two warps per lane quadrant, 16 token
+// columns each, so two warps share each scheduler's promotion work)
+template <int EPI>
+__host__ __device__ constexpr int masked_threads() { return EPI == 1 ? 192 : 320; }
 
 template <int EPI>
 struct SmemM {
@@ -453,6 +457,7 @@ struct SmemM {
     static constexpr int kStages = EPI == 1 ? 4 : 10;
     static constexpr int kCols = EPI == 1 ? 2 * kBT : kBT;     // tensor-memory columns per buffer
     static constexpr int kBufs = 4;                            // MMA runs up to 3 K blocks ahead of promotion
+    static constexpr int kSaSlots = 16;                        // scale ring deeper than the stage ring
     uint8_t w[kStages][kW];
     uint8_t x[kStages][kXBytes];
     float hs[EPI == 1 ? 2 : 1][EPI == 1 ? kBT : 1][kBM];       // SwiGLU output staged for the requant
@@ -471,7 +476,7 @@ struct SmemM {
 };
 
 template <int EPI>
-__global__ void __launch_bounds__(kThreadsM, 1)
+__global__ void __launch_bounds__(masked_threads<EPI>(), 1)
 gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ As, const int32_t* __restrict__ masked_m, int Mmax,
                  const float* __restrict__ Bs, int E, int N, int K, void* __restrict__ D, float* __restrict__ Ds,
@@ -508,13 +513,14 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
-        for (int j = 0; j < kSaSlots; ++j) {
+        constexpr int kPW = (masked_threads<EPI>() - 64) / 32;   // promotion warps
+        for (int j = 0; j < S::kSaSlots; ++j) {
             mbar_init(&sm.sfull[j], 1);
-            mbar_init(&sm.sempty[j], 4);
+            mbar_init(&sm.sempty[j], kPW);
         }
         for (int b = 0; b < S::kBufs; ++b) {
             mbar_init(&sm.tfull[b], 1);
-            mbar_init(&sm.tempty[b], 4);
+            mbar_init(&sm.tempty[b], kPW);
         }
         for (int b = 0; b < 2; ++b) mbar_init(&sm.red_bar[b], 128);
         sm.abort_flag = 0;
@@ -561,8 +567,8 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     if (EPI == 1) tma_load_2d(sm.w[s] + kWBlk, &tmW, &sm.full[s], kb * kBK, wrow + kBM);
                     tma_load_2d(sm.x[s], &tmX, &sm.full[s], kb * kBK, e * Mmax + tt * kBT);
                     // the token tile's 32 activation scales of this K block, into the scale ring
-                    const int j = it % kSaSlots;
-                    if (!mbar_wait(&sm.sempty[j], ((it / kSaSlots) & 1) ^ 1, wait_ns)) { fail(); break; }
+                    const int j = it % S::kSaSlots;
+                    if (!mbar_wait(&sm.sempty[j], ((it / S::kSaSlots) & 1) ^ 1, wait_ns)) { fail(); break; }
                     mbar_arrive_expect_tx(&sm.sfull[j], kBT * sizeof(float));
                     bulk_load(sm.sa[j], As + (static_cast<int64_t>(e) * KB + kb) * Mmax + tt * kBT, kBT * sizeof(float),
                               &sm.sfull[j]);
@@ -596,10 +602,13 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
         }
     } else {
-        // promotion + epilogue: 4 warps, thread = tensor-memory lane = weight row
+        // promotion + epilogue: thread = tensor-memory lane = weight row; for the bf16 output two warps
+        // per lane quadrant take token columns [16 * hh, 16 * hh + 16)
         const int q = warp & 3;
-        const int pw = warp - 2;                 // 0..3
+        const int pw = warp - 2;                 // 0..3 (SwiGLU) or 0..7
         const int r = q * 32 + lane;
+        constexpr int kC = EPI == 1 ? kBT : kBT / 2;     // token columns per thread
+        const int cof = EPI == 1 ? 0 : (pw >> 2) * kC;  // its first token column
         uint32_t kbt = 0, ep = 0;
         // lane l holds the weight-block scales of K blocks l, l + 32, l + 64, l + 96 of the tile's
         // weight block(s) (K <= 16384), loaded one tile ahead so their latency hides behind a tile
@@ -621,9 +630,9 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             if (sm.abort_flag) break;
             int e, nb, tt, m_e;
             decode(tile, e, nb, tt, m_e);
-            float acc[EPI == 1 ? 2 * kBT : kBT];
+            float acc[EPI == 1 ? 2 * kBT : kC];
 #pragma unroll
-            for (int i = 0; i < (EPI == 1 ? 2 * kBT : kBT); ++i) acc[i] = 0.0f;
+            for (int i = 0; i < (EPI == 1 ? 2 * kBT : kC); ++i) acc[i] = 0.0f;
             const float wta[4] = {wa[0], wa[1], wa[2], wa[3]};
             const float wtb[4] = {wb[0], wb[1], wb[2], wb[3]};
             load_w(tile + gridDim.x);
@@ -632,12 +641,12 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 const int buf = kbt % S::kBufs;
                 const uint32_t bph = (kbt / S::kBufs) & 1;
                 // scales: the token tile's 32 from the ring, the weight block's from the lane holding it
-                const int j = kbt % kSaSlots;
-                if (!mbar_wait(&sm.sfull[j], (kbt / kSaSlots) & 1, wait_ns)) { fail(); ok = false; break; }
-                float sa[kBT];
+                const int j = kbt % S::kSaSlots;
+                if (!mbar_wait(&sm.sfull[j], (kbt / S::kSaSlots) & 1, wait_ns)) { fail(); ok = false; break; }
+                float sa[kC];
 #pragma unroll
-                for (int i = 0; i < kBT / 4; ++i) {
-                    const float4 v4 = *reinterpret_cast<const float4*>(&sm.sa[j][4 * i]);
+                for (int i = 0; i < kC / 4; ++i) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(&sm.sa[j][cof + 4 * i]);
                     sa[4 * i] = v4.x; sa[4 * i + 1] = v4.y; sa[4 * i + 2] = v4.z; sa[4 * i + 3] = v4.w;
                 }
                 __syncwarp();
@@ -651,7 +660,13 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * S::kCols;
-                {
+                if constexpr (EPI == 0) {
+                    float v[16];
+                    tmem_ld16(taddr + cof, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < kC; ++c) acc[c] = fmaf(v[c], sa[c] * swa, acc[c]);
+                } else {
                     float v[32];
                     tmem_ld32(taddr, v);
                     tmem_ld_wait();
@@ -673,10 +688,10 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const int nv = min(kBT, m_e - tt * kBT);       // valid tokens in this tile
             const int64_t row0 = static_cast<int64_t>(e) * Mmax + tt * kBT;
             if constexpr (EPI == 0) {
-                uint16_t* out = static_cast<uint16_t*>(D) + row0 * N + nb * kBM + r;
+                uint16_t* out = static_cast<uint16_t*>(D) + (row0 + cof) * N + nb * kBM + r;
 #pragma unroll
-                for (int c = 0; c < kBT; ++c)
-                    if (c < nv) out[static_cast<int64_t>(c) * N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[c]));
+                for (int c = 0; c < kC; ++c)
+                    if (cof + c < nv) out[static_cast<int64_t>(c) * N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[c]));
             } else {
                 const int I = N / 2;
                 const int p = ep & 1;
@@ -794,13 +809,13 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
             const size_t smem = sizeof(SmemM<0>) + 1024;
             cudaError_t err = set_smem(gg_masked_kernel<0>, smem);
             if (err != cudaSuccess) return err;
-            gg_masked_kernel<0><<<num_sms, kThreadsM, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
+            gg_masked_kernel<0><<<num_sms, masked_threads<0>(), smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
                                                                   Ds, status, wait_ns);
         } else {
             const size_t smem = sizeof(SmemM<1>) + 1024;
             cudaError_t err = set_smem(gg_masked_kernel<1>, smem);
             if (err != cudaSuccess) return err;
-            gg_masked_kernel<1><<<num_sms, kThreadsM, smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
+            gg_masked_kernel<1><<<num_sms, masked_threads<1>(), smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
                                                                   Ds, status, wait_ns);
         }
     }
