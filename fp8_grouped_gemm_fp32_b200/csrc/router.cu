@@ -130,17 +130,37 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         if (lane == 0) mbar_arrive(&empty[s]);
     }
     if (ok) {
+        // The 32 chains of each (token, expert) meet in the canonical halving tree: lanes j and j ^ 16,
+        // then j ^ 8, ^4, ^2, ^1. As a reduce-scatter: at each level a lane keeps half of its remaining
+        // values, adds its partner's copy of them (the same pair of partial sums, so the same fp32
+        // sums as the full butterfly: addition is commutative) and sends the other half, so the
+        // TR * ER sums cost TR * ER - TR * ER / 32 shuffles instead of 5 per sum; each lane ends with
+        // TR * ER / 32 finished logits.
+        constexpr int NV = TR * ER;
+        static_assert(NV % 32 == 0, "the register tile must spread evenly over the lanes");
+        float* v = &acc[0][0];
+        int base = 0;
 #pragma unroll
-        for (int i = 0; i < TR; ++i) {
+        for (int lvl = 0; lvl < 5; ++lvl) {
+            const int w = 16 >> lvl;
+            constexpr int kC0 = NV;
+            const int half = (kC0 >> lvl) >> 1;
+            const bool upper = (lane & w) != 0;
 #pragma unroll
-            for (int q = 0; q < ER; ++q) {
-                float v = acc[i][q];
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
-                const int t = t_base + wt * TR + i, e = e_base + we * ER + q;
-                if (lane == ((i * ER + q) & 31) && t < T && e < E)
-                    logits[static_cast<int64_t>(t) * E + e] = bias ? v + bias[e] : v;
+            for (int m = 0; m < (NV >> 1); ++m) {
+                if (m < half) {
+                    const float send = upper ? v[m] : v[m + half];
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, w);
+                    v[m] = (upper ? v[m + half] : v[m]) + recv;
+                }
             }
+            base += upper ? half : 0;
+        }
+#pragma unroll
+        for (int m = 0; m < NV / 32; ++m) {
+            const int n = base + m;
+            const int t = t_base + wt * TR + n / ER, e = e_base + we * ER + n % ER;
+            if (t < T && e < E) logits[static_cast<int64_t>(t) * E + e] = bias ? v[m] + bias[e] : v[m];
         }
     }
     __syncthreads();

@@ -113,6 +113,48 @@ def test_permute_bit_exact(name, T):
         assert np.count_nonzero(ref["slot_row"] < 0) > 0
 
 
+def test_permute_extreme_magnitudes_bit_exact():
+    """x quantisation across the whole bf16 range: groups scaled from the subnormals (2^-133) to 2^124,
+    either side of the 2^-60 switch between the multiply-and-correct quotients and the division, groups
+    of signed zeros, a single nonzero value, and values on exact E4M3 rounding midpoints (amax = 448 * 2^k,
+    so every quotient is a tie that must round to even). Codes and scales bit-exact with the oracle."""
+    import types
+    ensure_lib()
+    base = CONFIGS["tiny"]
+    T = 96
+    cfg = base.replace(T=T)
+    G = cfg.H // 128
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((T, cfg.H)).astype(np.float64)
+    mags = [2.0 ** -133, 2.0 ** -124, 2.0 ** -100, 2.0 ** -70, 2.0 ** -61, 2.0 ** -60, 2.0 ** -59, 2.0 ** -20,
+            1.0, 2.0 ** 50, 2.0 ** 100, 2.0 ** 124]
+    for t in range(T):
+        for g in range(G):
+            x[t, g * 128:(g + 1) * 128] *= mags[(t * G + g) % len(mags)]
+    x[0, 0:128] = 0.0
+    x[1, 0:128] = -0.0
+    x[2, 0:128] = 0.0
+    x[2, 5] = -3.0
+    mids = np.array([(1 + (m + 0.5) / 8) * 2.0 ** e for e in range(-6, 8) for m in range(8)
+                     if (1 + (m + 0.5) / 8) * 2.0 ** e < 448])
+    for t in range(3, T, 7):
+        k = int(rng.integers(-80, 80))
+        grp = rng.choice(mids, 128) * rng.choice([-1.0, 1.0], 128)
+        grp[int(rng.integers(0, 128))] = 448.0
+        x[t, 128:256] = grp * 2.0 ** k
+    xb = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+    assert torch.isfinite(xb.float()).all()
+    topk = np.stack([rng.permutation(cfg.E)[:cfg.k] for _ in range(T)]).astype(np.int32)
+    inp = types.SimpleNamespace(x=xb.cuda())
+    got, rows = _permute(cfg, inp, topk)
+    ref = oracle.permute(cfg, xb.view(torch.int16).numpy().view(np.uint16), topk, rows)
+    used = ref["offsets"][-1]
+    assert np.array_equal(got["slot_row"], ref["slot_row"])
+    assert np.array_equal(got["Aq"][:used], ref["Aq"][:used])
+    assert np.array_equal(got["As"][:, :used], ref["As"][:, :used])
+    assert np.any(ref["Aq"][:used] == 0x80)                    # negative zeros survive as codes
+
+
 def _rand_codes(rng, shape):
     c = rng.integers(0, 256, size=shape, dtype=np.uint8)
     c[(c & 0x7F) == 0x7F] = 0x3C                              # no NaN codes
