@@ -15,13 +15,16 @@
 //
 // * contiguous layout (prefill): tiles of 128 rows x 256 columns over the
 //   flattened, 128-padded M of all groups (the pages' global tile scheduler,
-//   3.2). Warp 0 issues TMA loads into a 4-stage shared-memory ring; warp 1
-//   issues tcgen05.mma (kind::f8f6f4, M=128, N=256, K=32) for each 128-wide K
-//   block into one of two tensor-memory buffers; 8 promotion warps read each
+//   3.2). Warp 0 issues TMA loads into a 3- or 4-stage shared-memory ring,
+//   bulk copies of each K block's 128 activation scales into a ring of their
+//   own, and stages each tile's weight-block scales; warp 1 issues
+//   tcgen05.mma (kind::f8f6f4, M=128, N=256, K=32) for each 128-wide K block
+//   into one of two tensor-memory buffers; 8 promotion warps read each
 //   finished block with tcgen05.ld and fold it into fp32 register
-//   accumulators scaled by sa[row] * sw[block], then run the epilogue. Tiles
-//   are ordered expert -> N tile -> M tile, so the CTAs working at the same
-//   time share one weight tile through L2.
+//   accumulators scaled by sa[row] * sw[block], then run the epilogue, whose
+//   output leaves through shared memory and TMA stores. Tiles are ordered
+//   expert -> N tile -> M tile, so the CTAs working at the same time share
+//   one weight tile through L2.
 // * masked layout (decode, few tokens per expert): swap-AB. The weight block
 //   is the MMA's M=128 operand and up to 32 tokens are its N, so weights
 //   stream from HBM in 16 KB (or 2 x 16 KB) stages while the token tile is

@@ -98,9 +98,9 @@ size_t moe_workspace_size(const moe_config_t* cfg, int for_forward);
  *   topk_idx  [T, k] int32 out: experts in descending score, ties to the lower index
  *   topk_w    [T, k] fp32 out: w_j = exp(l_j - m) / sum_{top-k} exp(l_i - m)
  *   ws        scratch of at least moe_workspace_size(cfg, 0) bytes (holds the T x E logits)
- * Logits are fp32 with one fixed summation order: 32 interleaved fused
- * multiply-add chains over h = j, j+32, ..., halved pairwise (j with j+16,
- * then j+8, 4, 2, 1), then + b. Hash routing (DeepSeek-V4 lecture page,
+ * Logits are fp32 with one fixed summation order: 32 fused multiply-add
+ * chains, chain j over h = 128 s + 4 j + i (i = 0..3, every 128-wide block s
+ * in order), halved pairwise (j with j+16, then j+8, 4, 2, 1), then + b. Hash routing (DeepSeek-V4 lecture page,
  * section 2.2, hash(token_id) % num_experts): expert =
  * (uint32)(token_id * 2654435761) % E, k = 1, weight 1.
  */
