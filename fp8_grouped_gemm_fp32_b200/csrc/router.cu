@@ -35,7 +35,8 @@ struct RouterCfg {
     static constexpr int kXBytes = TT * kRouterHS * 2;
     static constexpr int kWBytes = EC * kRouterHS * 4;
     static constexpr int kStageBytes = kXBytes + kWBytes;
-    static constexpr int kStages = 160 * 1024 / kStageBytes < 8 ? 160 * 1024 / kStageBytes : 8;
+    // a power of two (slot and phase of a stage by mask and shift), up to 8, within 200 KB
+    static constexpr int kStages = 8 * kStageBytes <= 200 * 1024 ? 8 : 4 * kStageBytes <= 200 * 1024 ? 4 : 2;
     static constexpr int kSmem = kStages * kStageBytes + 2 * kStages * 8 + 16 + 1024;
 };
 
