@@ -297,11 +297,18 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of the ranks' values (a device time: the job is as slow as its slowest rank)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    on_gpu = torch.distributed.get_backend() == "nccl"
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if on_gpu else "cpu")
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time per step."""
+    return world * tokens_per_rank / (ms_max / 1e3)
 
 
 class _HostExperts:
@@ -376,7 +383,7 @@ def run_ours(args):
     ms_max = max_over_ranks(ms, world)
     st = api.moe_get_device_status()
     assert st == api.MOE_OK, api.STATUS_NAMES.get(st)
-    value = world * cfg.T / (ms_max / 1e3)
+    value = job_tokens_per_s(cfg.T, world, ms_max)
 
     # End to end through the public call with host buffers: every step copies its tokens (x, and the
     # token ids for hash routing) from pinned host memory to the device, runs moe_forward and copies y
@@ -439,7 +446,7 @@ def run_ours(args):
                  "frac_fp8_nominal_4500": gemm_tflops / 4500.0, "ms": gemm_ms, "rows_kept": Rk,
                  "experts_touched": touched},
         "kernels_ms": per,
-        "e2e": {"value": world * cfg.T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_tokens_per_s(cfg.T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": layer.launches_per_step * args.steps,
         "clocks": clk.summary(),
