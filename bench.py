@@ -192,7 +192,8 @@ class Layer:
         self.offsets = z(E + 1, dt=torch.int32)
         self.row_src = z(rows, dt=torch.int32)
         self.step_ws = z(api.moe_workspace_size(self.c, False), dt=torch.uint8)
-        self.launches_per_step = (1 if cfg.routing == "hash" else 2) + 3 + 2 + 1
+        # router (logits + top-k, or hash) + permute (count, scan, map, quantise) + 2 GEMMs + combine
+        self.launches_per_step = (1 if cfg.routing == "hash" else 2) + 4 + 2 + 1
 
     def forward(self, x=None, stream=None):
         a = self.api
