@@ -361,6 +361,8 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     cfg = CONFIGS[args.config]
+    if args.experts:
+        cfg = cfg.replace(E=args.experts)
     from fp8_grouped_gemm_fp32_b200 import api
     api.lib()                                      # fails loudly if the native library is missing
     layer = Layer(cfg, dev, seed_offset=rank)
@@ -498,6 +500,8 @@ def main():
     ap.add_argument("--config", default="page", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the workload's expert count (reduced cases for profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
