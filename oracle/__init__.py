@@ -86,6 +86,7 @@ def _declare(L):
     L.orc_expert_rows.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i]
     L.orc_grouped_gemm.argtypes = [_i, _i, _i, _i, _p, _p, _p, _i, _p, _p, _i, _p, _p, _i]
     L.orc_combine.argtypes = [_i, _i, _i, _p, _p, _p, _p]
+    L.orc_balance_bias.argtypes = [_i, _p, _p, _p, ctypes.c_float, _i]
 
 
 def _ptr(a: Optional[np.ndarray]):
@@ -239,6 +240,18 @@ def combine(slot_row: np.ndarray, topk_w: np.ndarray, O: np.ndarray, T: int, k: 
 
 
 # ---------------------------------------------------------------- pipeline
+def balance_bias(counts: np.ndarray, load: np.ndarray, bias: np.ndarray, gamma: float, update: bool):
+    """Auxiliary-loss-free bias balancing (MegaMoE page, 2.2), one step, in place:
+    load (int64) += counts; on an update step the bias (fp32) of every expert whose
+    load is above the mean drops by gamma, below it rises by gamma, and load is cleared."""
+    assert load.dtype == np.int64 and bias.dtype == np.float32
+    assert load.flags["C_CONTIGUOUS"] and bias.flags["C_CONTIGUOUS"]
+    c = _c(counts, np.int32)
+    E = c.shape[0]
+    assert load.shape == (E,) and bias.shape == (E,)
+    lib().orc_balance_bias(E, _ptr(c), _ptr(load), _ptr(bias), float(gamma), int(bool(update)))
+
+
 def route(cfg, x_bits, Wg, bias, token_ids, nthreads=None):
     """Routing step of the layer: (topk_idx [T,k], topk_w [T,k], logits or None)."""
     if cfg.routing == "hash":

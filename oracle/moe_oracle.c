@@ -441,3 +441,24 @@ void orc_combine(int T, int k, int H, const int32_t* slot_row, const float* topk
     }
     free(acc);
 }
+
+/* Auxiliary-loss-free load balancing ([P1] 2.2): every expert keeps a routing
+ * bias; the load each expert received is tallied over the update interval and,
+ * when the interval ends, an expert that received more than the mean has its
+ * bias lowered by the step gamma, one that received less has it raised, and
+ * one exactly at the mean keeps it. The mean is compared exactly, in integers:
+ * E * load[e] against the total. The bias is stored in fp32, so the step is
+ * one fp32 addition or subtraction. The tally restarts after an update. */
+void orc_balance_bias(int E, const int32_t* counts, int64_t* load, float* bias, float gamma, int update) {
+    int e;
+    int64_t total = 0;
+    for (e = 0; e < E; ++e) load[e] += counts[e];
+    if (!update) return;
+    for (e = 0; e < E; ++e) total += load[e];
+    for (e = 0; e < E; ++e) {
+        const int64_t scaled = (int64_t)E * load[e];
+        if (scaled > total) bias[e] = bias[e] - gamma;        /* overloaded: lower */
+        else if (scaled < total) bias[e] = bias[e] + gamma;   /* underloaded: raise */
+        load[e] = 0;
+    }
+}

@@ -35,7 +35,11 @@
  *    fp32-rounded v / scale;
  *  - dequantisation to fp32 (code * scale rounded to fp32), fp64 sums,
  *    h = silu(a) * b in fp64 rounded to fp32 and requantised as above,
- *    o rounded to bf16 (RNE), y = fp64 weighted sum rounded to bf16.
+ *    o rounded to bf16 (RNE), y = fp64 weighted sum rounded to bf16;
+ *  - bias balancing ([P1] 2.2 gives the direction, the step size and the
+ *    interval): an expert's load is the number of slots routed to it (before
+ *    any capacity drop), summed over the interval; above the mean -> bias
+ *    minus gamma, below -> plus gamma, at the mean -> unchanged.
  *
  * Parity pins live in tests/ (run with -m "not gpu").
  */
@@ -88,6 +92,10 @@ void orc_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const f
 /* Combine: y[t,:] = sum_j [kept] w[t,j] * O[slot_row[t*k+j], :], fp64, -> bf16. */
 void orc_combine(int T, int k, int H, const int32_t* slot_row, const float* topk_w,
                  const uint16_t* O, uint16_t* y);
+/* Auxiliary-loss-free bias balancing: load += counts; if update, each bias
+ * moves by -gamma / +gamma / 0 as E*load[e] is above / below / equal to
+ * sum(load) (fp32 arithmetic), and load is cleared. */
+void orc_balance_bias(int E, const int32_t* counts, int64_t* load, float* bias, float gamma, int update);
 
 #ifdef __cplusplus
 }
