@@ -408,6 +408,35 @@ def run_ours(args):
     kept = layer.kept.cpu().numpy()
     work, Rk, touched = algorithmic_work(cfg, kept)
 
+    # training side, outside the forward step: the auxiliary-loss-free bias update fed by this step's
+    # counts, one launch per training step with an update every 100th (the page's interval). The 100
+    # launches are replayed from a CUDA graph so that the device time, not the host's per-call cost, is
+    # measured.
+    bal_load = torch.zeros(cfg.E, dtype=torch.int64, device=layer.counts.device)
+    bal_bias = layer.inp.bias.clone()
+    side = torch.cuda.Stream(layer.counts.device)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            api.moe_balance_bias(cfg.E, layer.counts, bal_load, bal_bias, 1e-3, False, side)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        gs = torch.cuda.current_stream()
+        for i in range(100):
+            api.moe_balance_bias(cfg.E, layer.counts, bal_load, bal_bias, 1e-3, i == 99, gs)
+    graph.replay()
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record()
+    for _ in range(2):
+        graph.replay()
+    b1.record()
+    torch.cuda.synchronize()
+    del graph
+    balance = {"us_per_call": 1e3 * b0.elapsed_time(b1) / 200, "calls": 200, "timing": "CUDA graph replay",
+               "bytes_per_call": 28 * cfg.E, "bound": "launch latency (one block, 28 B per expert)"}
+
     peaks, peak_src = load_peaks()
     hbm = float(peaks["hbm_gbs"])
     fp8_sus = FP8_PER_BF16 * float(peaks["bf16_tflops_sustained"])
@@ -449,6 +478,7 @@ def run_ours(args):
                  "frac_fp8_nominal_4500": gemm_tflops / 4500.0, "ms": gemm_ms, "rows_kept": Rk,
                  "experts_touched": touched},
         "kernels_ms": per,
+        "balance_bias": balance,
         "e2e": {"value": job_tokens_per_s(cfg.T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": layer.launches_per_step * args.steps,

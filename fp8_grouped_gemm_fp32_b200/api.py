@@ -30,7 +30,7 @@ LAYOUT_CONTIGUOUS, LAYOUT_MASKED = 0, 1
 EPI_BF16, EPI_SWIGLU_FP8 = 0, 1
 EXPORTS = ("moe_rows_capacity", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_gemm_fp8",
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string",
-           "moe_permute_noalloc")
+           "moe_permute_noalloc", "moe_balance_bias")
 
 
 class MoeError(RuntimeError):
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_gemm_fp8.argtypes = [I, I, I, I, P, P, P, I, P, P, I, P, P, P]
         L.moe_combine.argtypes = [CP, P, P, P, P, P]
         L.moe_forward.argtypes = [CP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_balance_bias.argtypes = [I, P, P, P, ctypes.c_float, I, P]
         L.moe_get_device_status.argtypes = [P]
         L.moe_selftest_wait_timeout.argtypes = [I, P]
         L.moe_status_string.argtypes = [I]
@@ -153,6 +154,13 @@ def moe_forward(cfg, x, Wg, bias, token_ids, W13, S13, W2, S2, y, topk_idx, topk
     _check(lib().moe_forward(ctypes.byref(cfg), _p(x), _p(Wg), _p(bias), _p(token_ids), _p(W13), _p(S13), _p(W2),
                              _p(S2), _p(y), _p(topk_idx), _p(topk_w), _p(counts), _p(slot_row), _p(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+
+
+def moe_balance_bias(E, counts, load, bias, gamma, update, stream=None):
+    """Auxiliary-loss-free bias step: load (int64) += counts; if update, bias (fp32) moves by -gamma / +gamma
+    for experts above / below the mean tally, and load is cleared."""
+    _check(lib().moe_balance_bias(E, _p(counts), _p(load), _p(bias), float(gamma), int(bool(update)),
+                                  _stream(stream)), "moe_balance_bias")
 
 
 def moe_get_device_status(stream=None) -> int:

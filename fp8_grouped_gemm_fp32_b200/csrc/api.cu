@@ -2,6 +2,7 @@
 // carving, the per-device status word and the launch sequence of moe_forward.
 // Nothing here allocates device memory or synchronises the host, except
 // moe_get_device_status, whose job is to synchronise and read the status.
+#include <math.h>
 #include <string.h>
 
 #include <algorithm>
@@ -27,6 +28,8 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
 cudaError_t launch_combine(const uint16_t* O, const int32_t* slot_row, const float* topk_w, int T, int k, int H,
                            uint16_t* y, cudaStream_t s);
 cudaError_t launch_selftest_wait(int* status, uint64_t wait_ns, cudaStream_t s);
+cudaError_t launch_balance_bias(int E, const int32_t* counts, int64_t* load, float* bias, float gamma, int update,
+                                cudaStream_t s);
 
 // The device status word (one per device that loads the library).
 __device__ int g_status;
@@ -288,6 +291,17 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_combine(w.O, slot_row, topk_w, cfg->T, cfg->k, cfg->H, static_cast<uint16_t*>(y), s);
     return cuda_status(e);
+}
+
+moe_status_t moe_balance_bias(int E, const int32_t* counts, int64_t* load, float* bias, float gamma, int update,
+                              void* stream) {
+    if (E <= 0) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!ptr_ok(counts) || !ptr_ok(load) || !ptr_ok(bias) || !isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+    moe_status_t st;
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    return cuda_status(launch_balance_bias(E, counts, load, bias, gamma, update != 0, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_get_device_status(void* stream) {

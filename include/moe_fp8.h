@@ -15,6 +15,8 @@
  *                        in fp32 promotion; epilogue bf16 or SwiGLU + FP8 requant
  *   moe_combine          weighted un-permute y = sum_j w_j * o_j
  *   moe_forward          all of the above on one stream, no host sync
+ * and, for training, moe_balance_bias: the auxiliary-loss-free update of the
+ * routing bias b from the per-expert counts moe_permute reports.
  *
  * Conventions (every entry point):
  *  - Every array argument is a DEVICE pointer owned by the caller, except the
@@ -218,6 +220,29 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
 moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
                                  uint8_t* Aq, float* As, int32_t* counts, int32_t* kept, int32_t* offsets,
                                  int32_t* row_src, int32_t* slot_row, void* stream);
+
+/*
+ * Auxiliary-loss-free load balancing. Source: MegaMoE page, section 2.2: each
+ * expert keeps a bias b_e inside the router softmax (moe_route's `bias`); while
+ * training, the bias of an expert with high load goes down and of one with low
+ * load goes up, by a step of order 1e-3, once every 100 or so steps. One call
+ * per training step:
+ *   counts  [E] int32: slots routed to each expert this step (moe_permute's
+ *           `counts`, before any capacity drop); must be >= 0
+ *   load    [E] int64 in/out: the tally since the last update; zero it once
+ *           before the first step
+ *   bias    [E] fp32 in/out
+ *   gamma   the step, finite (a negative step reverses the direction)
+ *   update  0: load += counts only. Nonzero (the last step of an interval):
+ *           load += counts; then b_e -= gamma where E * load[e] > sum(load),
+ *           b_e += gamma where E * load[e] < sum(load), unchanged where equal
+ *           (the mean compared exactly in 64-bit integers; one fp32
+ *           round-to-nearest-even addition per expert); then load = 0.
+ * E in 1..MOE_MAX_EXPERTS (MOE_ERR_UNSUPPORTED_SHAPE above it). One block of
+ * one thread per expert; the tally must stay below 2^63 / E.
+ */
+moe_status_t moe_balance_bias(int E, const int32_t* counts, int64_t* load, float* bias, float gamma, int update,
+                              void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: MOE_OK, MOE_ERR_CAPACITY or MOE_ERR_DEVICE_TIMEOUT. */

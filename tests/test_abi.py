@@ -86,6 +86,15 @@ def test_hash_routing_needs_k1_and_masked_needs_rows(L):
     assert api.moe_workspace_size(c) == 0
 
 
+@pytest.mark.parametrize("E,gamma,ptr,code", [
+    (0, 1e-3, 4096, api.MOE_ERR_INVALID_ARG), (513, 1e-3, 4096, api.MOE_ERR_UNSUPPORTED_SHAPE),
+    (8, float("nan"), 4096, api.MOE_ERR_INVALID_ARG), (8, float("inf"), 4096, api.MOE_ERR_INVALID_ARG),
+    (8, 1e-3, 4100, api.MOE_ERR_INVALID_ARG), (8, 1e-3, 0, api.MOE_ERR_INVALID_ARG)])
+def test_bad_balance_arguments_rejected_before_any_device_work(L, E, gamma, ptr, code):
+    p = ctypes.c_void_p(ptr)                   # never dereferenced: the call returns first
+    assert L.moe_balance_bias(E, p, p, p, gamma, 1, None) == code
+
+
 def test_product_and_oracle_share_no_code():
     pkg = os.path.join(ROOT, "fp8_grouped_gemm_fp32_b200")
     for dirpath, _, files in os.walk(pkg):

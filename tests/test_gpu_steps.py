@@ -6,7 +6,8 @@
   slot_row and the quantised rows Aq / scales As bit-exact, padding included;
 * moe_grouped_gemm_fp8: both layouts x both epilogues on ragged groups
   (empty groups, 1 row, tiles plus a ragged tail, a half-width N tile);
-* moe_combine (fed the oracle's expert outputs), with dropped slots.
+* moe_combine (fed the oracle's expert outputs), with dropped slots;
+* moe_balance_bias: tallies and biases bit-exact over a sequence of steps.
 """
 import numpy as np
 import pytest
@@ -262,6 +263,58 @@ def test_combine_with_drops():
     assert len(all_dropped) > 0 and np.all(to_np(y)[all_dropped] == 0)
     assert_close_bf16(to_np(y), y_ref)
     assert np.mean(to_np(y) == y_ref) > 0.99
+
+
+@pytest.mark.parametrize("E", [1, 3, 64, 256, 512])
+def test_balance_bias_bit_exact(E):
+    # several update intervals of random counts (ties with the mean included), biases of both signs and
+    # sizes where the step is partly or wholly lost to fp32 rounding; tallies and biases bit-exact
+    ensure_lib()
+    rng = np.random.default_rng(E)
+    bias = np.concatenate([rng.uniform(-0.01, 0.01, E), [1.0, -1.0, 3e5, 0.0]])[:E].astype(np.float32)
+    load = np.zeros(E, np.int64)
+    b_dev = torch.from_numpy(bias.copy()).cuda()
+    l_dev = torch.zeros(E, dtype=torch.int64, device="cuda")
+    for step in range(12):
+        if step == 4:
+            counts = np.full(E, 7, np.int32)                  # every expert at the mean
+        elif step == 8:
+            counts = np.zeros(E, np.int32)                    # an empty step
+        else:
+            counts = rng.integers(0, 3000, E).astype(np.int32)
+        update = step % 4 == 3 or step == 4
+        gamma = [1e-3, 2.0 ** -25, -5e-4][step % 3]
+        oracle.balance_bias(counts, load, bias, gamma, update)
+        api.moe_balance_bias(E, torch.from_numpy(counts).cuda(), l_dev, b_dev, gamma, update)
+        torch.cuda.synchronize()
+        assert np.array_equal(to_np(l_dev), load), step
+        assert np.array_equal(to_np(b_dev).view(np.uint32), bias.view(np.uint32)), step
+
+
+def test_balance_bias_from_routed_counts():
+    # the counts moe_permute reports feed the update directly, on the device
+    ensure_lib()
+    cfg = MoeConfig("zipf", T=2048, H=512, E=64, I=128, k=2, bias="zipf", cap_num=5, cap_den=4, seed=5)
+    inp = gpu_inputs(cfg)
+    c = api.Config.from_moe(cfg)
+    idx, _w = _route(cfg, inp)
+    rows = api.moe_rows_capacity(c)
+    d = lambda *s, dt=torch.int32: torch.empty(*s, dtype=dt, device="cuda")
+    counts = d(cfg.E)
+    ws = torch.empty(max(api.moe_workspace_size(c), 16), dtype=torch.uint8, device="cuda")
+    api.moe_permute(c, inp.x, torch.from_numpy(idx).cuda(), d(rows, cfg.H, dt=torch.uint8), d(rows * cfg.H // 128,
+                    dt=torch.float32), counts, d(cfg.E), d(cfg.E + 1), d(rows), d(cfg.T * cfg.k), ws)
+    load = torch.zeros(cfg.E, dtype=torch.int64, device="cuda")
+    bias = inp.bias.clone()
+    api.moe_balance_bias(cfg.E, counts, load, bias, 1e-3, True)
+    torch.cuda.synchronize()
+    ref_load = np.zeros(cfg.E, np.int64)
+    ref_bias = to_np(inp.bias).copy()
+    oracle.balance_bias(np.bincount(idx.ravel(), minlength=cfg.E).astype(np.int32), ref_load, ref_bias, 1e-3, True)
+    assert np.array_equal(to_np(bias).view(np.uint32), ref_bias.view(np.uint32))
+    assert np.array_equal(to_np(load), ref_load)
+    # the Zipf prior makes expert 0 the busiest: its bias goes down
+    assert to_np(bias)[0] < to_np(inp.bias)[0]
 
 
 def test_empty_batch_is_a_no_op():
