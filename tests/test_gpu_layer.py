@@ -8,9 +8,11 @@ configuration the benchmark times) run the oracle's routing and dispatch on
 every token and its expert math on a sample of tokens."""
 import numpy as np
 import pytest
+import torch
 
 import oracle
-from fp8_grouped_gemm_fp32_b200.inputs import CONFIGS, MoeConfig
+from fp8_grouped_gemm_fp32_b200 import api
+from fp8_grouped_gemm_fp32_b200.inputs import CONFIGS, MoeConfig, interleave_w13
 from gpu_helpers import (W_RTOL, assert_close_bf16, ensure_lib, gpu_forward, gpu_inputs, oracle_inputs,
                          sample_tokens, to_np)
 
@@ -63,3 +65,52 @@ def test_layer_full_size_sampled(name, n_tokens):
     _check_layer(cfg, inp, ref, out, toks)
     if cfg.cap_num:
         assert np.count_nonzero(ref["slot_row"] < 0) > 0        # the capacity really drops slots
+
+
+@pytest.mark.parametrize("name", ["tiny", "masked_small"])
+def test_forward_replays_from_a_cuda_graph(name):
+    # moe_forward allocates nothing, synchronises nothing and reads no device state on the host, so a
+    # stream capture records the whole layer; replayed on new tokens written into the captured input
+    # buffer, it gives bit for bit what a direct call on those tokens gives
+    ensure_lib()
+    cfg, T = SMALL[name]
+    inp = gpu_inputs(cfg, T=T)
+    cfg = inp.cfg
+    c = api.Config.from_moe(cfg)
+    W13, S13 = interleave_w13(inp.W1q, inp.S1, inp.W3q, inp.S3)
+    dev = inp.x.device
+    out = dict(y=torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev),
+               topk_idx=torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev),
+               topk_w=torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev),
+               counts=torch.empty(cfg.E, dtype=torch.int32, device=dev),
+               slot_row=torch.empty(cfg.T * cfg.k, dtype=torch.int32, device=dev))
+    ws = torch.empty(api.moe_workspace_size(c, True), dtype=torch.uint8, device=dev)
+
+    def call(stream):
+        api.moe_forward(c, inp.x, inp.Wg, inp.bias, inp.token_ids, W13, S13, inp.W2q, inp.S2, out["y"],
+                        out["topk_idx"], out["topk_w"], out["counts"], out["slot_row"], ws, stream)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        call(side)
+    torch.cuda.synchronize()
+
+    inp.x.copy_(gpu_inputs(cfg.replace(seed=cfg.seed + 100), T=cfg.T).x)   # new tokens, same buffer
+    call(None)
+    torch.cuda.synchronize()
+    direct = {k: v.clone() for k, v in out.items()}
+    for v in out.values():
+        v.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert api.moe_get_device_status() == api.MOE_OK
+    for k in out:
+        assert torch.equal(out[k], direct[k]), k
+    ref = oracle.forward(cfg, oracle_inputs(inp))
+    _check_layer(cfg, inp, ref, out, np.arange(cfg.T))
+    del graph
