@@ -101,6 +101,37 @@ def test_grouped_gemm_equals_per_expert_dense_gemms():
         assert np.array_equal(Dq[r0:r1], hq) and np.array_equal(Ds[:, r0:r1].T, hs)
 
 
+def test_masked_grouped_gemm_equals_per_expert_dense_gemms():
+    # masked layout: block e of A holds masked_m[e] rows of expert e; its scales are [E][K/128][M_rows].
+    # Each block's product equals one dense float64 matmul over those rows, the SwiGLU epilogue equals the
+    # per-row expert function, and rows at or past masked_m[e] stay untouched (zero here).
+    cfg = MoeConfig("gm", T=80, H=256, E=4, I=128, k=2, bias="uniform", layout="masked", masked_max_m=64,
+                    seed=6)
+    t = make_inputs(cfg)
+    inp = oracle.moe_inputs_to_numpy(t)
+    idx, w, _ = oracle.route(cfg, inp["x"], inp["Wg"], inp["bias"], inp["token_ids"])
+    M = cfg.masked_max_m
+    d = oracle.permute(cfg, inp["x"], idx, cfg.E * M)
+    mm = d["kept"]
+    assert mm.min() > 0 and mm.max() < M                     # every block ragged, none full
+    Aq = d["Aq"].reshape(cfg.E * M, cfg.H)
+    As = d["As"].reshape(cfg.E, cfg.H // 128, M)
+    B, Bs = np.ascontiguousarray(inp["W1q"]), np.ascontiguousarray(inp["S1"])
+    D, _ = oracle.grouped_gemm(1, cfg.E, cfg.I, cfg.H, Aq, As, mm, M, B, Bs, 0)
+    W13, S13 = interleave_w13(t.W1q, t.S1, t.W3q, t.S3)
+    Dq, Ds = oracle.grouped_gemm(1, cfg.E, 2 * cfg.I, cfg.H, Aq, As, mm, M, W13.numpy(), S13.numpy(), 1)
+    for e in range(cfg.E):
+        r0, n = e * M, int(mm[e])
+        A = torch.from_numpy(Aq[r0:r0 + n]).view(torch.float8_e4m3fn).to(torch.float32)
+        sA = torch.from_numpy(As[e, :, :n].T.copy()).repeat_interleave(128, 1)
+        ref = ((A * sA).to(torch.float64) @ _deq_w(B[e], Bs[e]).T).numpy()
+        _close_bf16(D[r0:r0 + n], ref)
+        assert not D[r0 + n:r0 + M].any() and not Dq[r0 + n:r0 + M].any() and not Ds[e, :, n:].any()
+        hq, hs, _ = oracle.expert_rows(Aq[r0:r0 + n], np.ascontiguousarray(As[e, :, :n].T), inp["W1q"][e],
+                                       inp["S1"][e], inp["W3q"][e], inp["S3"][e], inp["W2q"][e], inp["S2"][e])
+        assert np.array_equal(Dq[r0:r0 + n], hq) and np.array_equal(Ds[e, :, :n].T, hs)
+
+
 def _brute_layer(cfg, inp, tokens):
     """Per token, straight from the formulas: fp64 logits, softmax over all E, top-k
     (ties to lower index), renormalise, y = sum_i w_i * E_i(x) with each expert
