@@ -9,6 +9,8 @@
 * moe_combine (fed the oracle's expert outputs), with dropped slots;
 * moe_balance_bias: tallies and biases bit-exact over a sequence of steps.
 """
+from types import SimpleNamespace
+
 import numpy as np
 import pytest
 import torch
@@ -60,6 +62,41 @@ def test_route_ties_and_ragged_shapes():
     assert np.array_equal(idx, ref_idx)
     assert np.allclose(w, ref_w, rtol=W_RTOL, atol=0)
     assert np.any(logits[:, 2] == logits[:, 5])
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "masked"])
+def test_route_and_permute_at_the_limits(layout):
+    # the largest shapes the boundary accepts: E = 512 experts, k = 32 per token, H = 16384, with a T
+    # that fills no tile; routing and the permutation (capacity drops in the contiguous case) bit-exact
+    ensure_lib()
+    extra = dict(cap_num=5, cap_den=4) if layout == "contiguous" else dict(layout="masked", masked_max_m=32)
+    cfg = MoeConfig("limits", T=40, H=16384, E=512, I=128, k=32, bias="uniform", seed=41, **extra)
+    g = torch.Generator().manual_seed(41)
+    x = torch.randn(cfg.T, cfg.H, generator=g).to(torch.bfloat16)
+    Wg = torch.randn(cfg.E, cfg.H, generator=g) * 0.02
+    bias = torch.rand(cfg.E, generator=g) * 0.02 - 0.01
+    inp = SimpleNamespace(x=x.cuda(), Wg=Wg.cuda(), bias=bias.cuda(), token_ids=None)
+    idx, w = _route(cfg, inp)
+    x_bits = x.view(torch.int16).numpy().view(np.uint16)
+    ref_idx, ref_w, _ = oracle.route(cfg, x_bits, Wg.numpy(), bias.numpy(), None)
+    assert np.array_equal(idx, ref_idx)
+    assert np.allclose(w, ref_w, rtol=W_RTOL, atol=0)
+    got, rows = _permute(cfg, inp, ref_idx)
+    ref = oracle.permute(cfg, x_bits, ref_idx, rows)
+    for key in ("counts", "kept", "offsets", "slot_row"):
+        assert np.array_equal(got[key], ref[key]), key
+    if layout == "masked":
+        M = cfg.masked_max_m
+        for e in np.nonzero(ref["kept"])[0]:
+            r0, n = e * M, ref["kept"][e]
+            assert np.array_equal(got["Aq"][r0:r0 + n], ref["Aq"][r0:r0 + n])
+            assert np.array_equal(got["As"][e, :, :n], ref["As"][e, :, :n])
+    else:
+        used = ref["offsets"][-1]
+        assert np.array_equal(got["row_src"][:used], ref["row_src"][:used])
+        assert np.array_equal(got["Aq"][:used], ref["Aq"][:used])
+        assert np.array_equal(got["As"][:, :used], ref["As"][:, :used])
+        assert np.count_nonzero(ref["slot_row"] < 0) > 0          # capacity 3 of 2.5 average drops slots
 
 
 def _permute(cfg, inp, topk_idx):
@@ -216,6 +253,12 @@ GEMM_CASES = [
     (1, 0, 4, 384, 256, [0, 5, 33, 64], 64),
     (1, 1, 4, 512, 256, [0, 5, 33, 64], 64),
     (1, 1, 3, 256, 512, [32, 1, 0], 96),
+    # the largest K (128 K blocks: every weight-block scale slot in use) and the largest N (H = 16384)
+    (0, 0, 2, 256, 16384, [130, 1], None),
+    (0, 1, 2, 256, 16384, [130, 1], None),
+    (0, 0, 2, 16384, 128, [130, 1], None),
+    (1, 0, 2, 256, 16384, [5, 32], 32),
+    (1, 1, 2, 256, 16384, [32, 7], 32),
 ]
 
 
