@@ -110,6 +110,24 @@ def quantize_weight_blocks(w: torch.Tensor):
     return q.reshape(N, K).view(torch.uint8), scale.contiguous()
 
 
+def quantize_weight_int4(w: torch.Tensor):
+    """Offline 4-bit weight quantisation (setup; DeepSeek-V4 lecture page, 3.1: per-channel blocks,
+    each scaled by its max-abs, levels round((w / max|w|) * (2^3 - 1))): [N, K] fp32 ->
+    (codes uint8 [N, K/2], fp32 scales [N, K/128]). A block is one row by 128 consecutive k; the level
+    is rounded half to even (torch.round) from the exact ratio (float64); the stored scale is
+    max-abs / 7 in fp32 (1.0 for an all-zero block), so a weight dequantises to level * scale. Two
+    levels per byte, the even k in the low nibble, as 4-bit two's-complement integers."""
+    N, K = w.shape
+    blk = w.reshape(N, K // BLOCK, BLOCK)
+    amax = blk.abs().amax(dim=2)
+    lev = torch.where(amax[..., None] > 0, (blk.double() * 7.0 / amax.double()[..., None]).round(),
+                      torch.zeros_like(blk, dtype=torch.float64))
+    lev = lev.to(torch.int16).reshape(N, K // 2, 2) & 15
+    codes = (lev[..., 0] | (lev[..., 1] << 4)).to(torch.uint8)
+    scale = torch.where(amax > 0, amax / 7.0, torch.ones_like(amax))
+    return codes.contiguous(), scale.contiguous()
+
+
 def _bias(cfg: MoeConfig, g: torch.Generator, device) -> torch.Tensor:
     if cfg.bias == "zero":
         return torch.zeros(cfg.E, dtype=torch.float32, device=device)

@@ -87,6 +87,9 @@ def _declare(L):
     L.orc_grouped_gemm.argtypes = [_i, _i, _i, _i, _p, _p, _p, _i, _p, _p, _i, _p, _p, _i]
     L.orc_combine.argtypes = [_i, _i, _i, _p, _p, _p, _p]
     L.orc_balance_bias.argtypes = [_i, _p, _p, _p, ctypes.c_float, _i]
+    L.orc_grouped_gemm_w4.argtypes = [_i, _i, _i, _i, _p, _p, _p, _i, _p, _p, _i, _p, _p, _i]
+    L.orc_w4_decode.argtypes = [ctypes.c_uint8, _i]
+    L.orc_w4_decode.restype = _i
 
 
 def _ptr(a: Optional[np.ndarray]):
@@ -208,9 +211,16 @@ def expert_rows(xq, xs, W1q, S1, W3q, S3, W2q, S2, nthreads: Optional[int] = Non
     return hq, hs, o
 
 
+def w4_decode(byte: int, high: bool) -> int:
+    """One 4-bit weight code (DeepSeek-V4 lecture page, 3.1): nibble `high` of `byte`, sign-extended."""
+    return int(lib().orc_w4_decode(byte, int(bool(high))))
+
+
 def grouped_gemm(layout: int, E: int, N: int, K: int, A, As, group_info, M_rows: int, B, Bs,
-                 epilogue: int, nthreads: Optional[int] = None):
-    """Oracle of moe_grouped_gemm_fp8. Rows outside every group are left 0."""
+                 epilogue: int, nthreads: Optional[int] = None, w4: bool = False):
+    """Oracle of moe_grouped_gemm_fp8. Rows outside every group are left 0. With w4, B holds
+    4-bit weight codes [E, N, K/2] and Bs one scale per weight row per 128-wide K block
+    [E, N, K/128] (DeepSeek-V4 lecture page, 3.1)."""
     A = _c(A, np.uint8)
     As = _c(As, np.float32)
     gi = _c(group_info, np.int32)
@@ -224,8 +234,9 @@ def grouped_gemm(layout: int, E: int, N: int, K: int, A, As, group_info, M_rows:
         D = np.zeros((rows, N // 2), dtype=np.uint8)
         G = N // 2 // GROUP
         Ds = np.zeros((G, M_rows) if layout == 0 else (E, G, M_rows), dtype=np.float32)
-    lib().orc_grouped_gemm(layout, E, N, K, _ptr(A), _ptr(As), _ptr(gi), M_rows, _ptr(B), _ptr(Bs),
-                           epilogue, _ptr(D), _ptr(Ds), nthreads or default_threads())
+    fn = lib().orc_grouped_gemm_w4 if w4 else lib().orc_grouped_gemm
+    fn(layout, E, N, K, _ptr(A), _ptr(As), _ptr(gi), M_rows, _ptr(B), _ptr(Bs), epilogue, _ptr(D), _ptr(Ds),
+       nthreads or default_threads())
     return D, Ds
 
 

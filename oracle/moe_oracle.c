@@ -290,6 +290,26 @@ static double dot_row(int K, const uint8_t* a, const float* a_s, const uint8_t* 
     return acc;
 }
 
+/* 4-bit weight codes ([P3] 3.1): the integer levels -7..7 of a block scaled by
+ * its max-abs, round((w / max|w|) * (2^3 - 1)). Two codes per byte, the even k
+ * in the low nibble, each a 4-bit two's-complement integer. */
+int orc_w4_decode(uint8_t byte, int high) {
+    int v = high ? (byte >> 4) : (byte & 15);
+    return v >= 8 ? v - 16 : v;
+}
+
+/* As dot_row, with a row of 4-bit weight codes and the row's K/128 scales
+ * (max-abs / 7 per block); the dequantised weight is code * scale in fp32. */
+static double dot_row_w4(int K, const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s) {
+    double acc = 0.0;
+    int kk;
+    for (kk = 0; kk < K; ++kk) {
+        float wd = (float)orc_w4_decode(w[kk >> 1], kk & 1) * w_s[kk / GROUP];
+        acc += (double)deq(a[kk], a_s[kk / GROUP]) * (double)wd;
+    }
+    return acc;
+}
+
 static double silu(double a) { return a / (1.0 + exp(-a)); }
 
 typedef struct {
@@ -348,6 +368,7 @@ void orc_expert_rows(int n, int H, int I, const uint8_t* xq, const float* xs,
 /* ------------------------------------------------------------------ */
 typedef struct {
     int layout, E, N, K, M_rows, epilogue;
+    int w4;            /* 0: E4M3 weights, 128x128 block scales; 1: 4-bit weights, 1x128 row scales */
     const uint8_t* A; const float* As; const int32_t* gi;
     const uint8_t* B; const float* Bs;
     void* D; float* Ds;
@@ -365,6 +386,17 @@ static int gg_row_expert(const gg_ctx* c, int64_t row) {
     return (row % c->M_rows) < c->gi[e] ? e : -1;
 }
 
+/* Output column n of expert e for one activation row: E4M3 weights are [E, N, K]
+ * with scales [E, N/128, K/128]; 4-bit weights are [E, N, K/2] with scales
+ * [E, N, K/128]. */
+static double gg_dot(const gg_ctx* c, const uint8_t* ar, const float* a_s, int e, int64_t n) {
+    const int K = c->K, KB = K / GROUP;
+    const int64_t row = (int64_t)e * c->N + n;
+    if (!c->w4)
+        return dot_row(K, ar, a_s, c->B + row * K, c->Bs + ((int64_t)e * (c->N / GROUP) + n / GROUP) * KB);
+    return dot_row_w4(K, ar, a_s, c->B + row * (K / 2), c->Bs + row * KB);
+}
+
 static void gg_range(void* vctx, int64_t b, int64_t end) {
     gg_ctx* c = (gg_ctx*)vctx;
     int K = c->K, N = c->N, KB = K / GROUP, n, kb;
@@ -373,21 +405,18 @@ static void gg_range(void* vctx, int64_t b, int64_t end) {
     int64_t row;
     for (row = b; row < end; ++row) {
         int e = gg_row_expert(c, row);
-        const uint8_t *ar, *Be;
-        const float *Bse, *As_base;
+        const uint8_t* ar;
+        const float* As_base;
         int64_t srow;
         if (e < 0) continue;
         ar = c->A + row * K;
-        Be = c->B + (int64_t)e * N * K;
-        Bse = c->Bs + (int64_t)e * (N / GROUP) * KB;
         srow = (c->layout == 0) ? row : row % c->M_rows;              /* scale column */
         As_base = (c->layout == 0) ? c->As : c->As + (int64_t)e * KB * c->M_rows;
         for (kb = 0; kb < KB; ++kb) a_s[kb] = As_base[(int64_t)kb * c->M_rows + srow];
         if (c->epilogue == 0) {
             uint16_t* D = (uint16_t*)c->D;
             for (n = 0; n < N; ++n)
-                D[row * N + n] = orc_f64_to_bf16(
-                    dot_row(K, ar, a_s, Be + (int64_t)n * K, Bse + (int64_t)(n / GROUP) * KB));
+                D[row * N + n] = orc_f64_to_bf16(gg_dot(c, ar, a_s, e, n));
         } else {
             int I = N / 2, G = I / GROUP, g;
             uint8_t* Dq = (uint8_t*)c->D;
@@ -397,8 +426,8 @@ static void gg_range(void* vctx, int64_t b, int64_t end) {
                 int blk = n / GROUP, w = n % GROUP;
                 int64_t r1 = (int64_t)(2 * blk) * GROUP + w;       /* gate row (W1) */
                 int64_t r3 = (int64_t)(2 * blk + 1) * GROUP + w;   /* up row (W3) */
-                double a = dot_row(K, ar, a_s, Be + r1 * K, Bse + (int64_t)(2 * blk) * KB);
-                double bb = dot_row(K, ar, a_s, Be + r3 * K, Bse + (int64_t)(2 * blk + 1) * KB);
+                double a = gg_dot(c, ar, a_s, e, r1);
+                double bb = gg_dot(c, ar, a_s, e, r3);
                 h[n] = (float)(silu(a) * bb);
             }
             for (g = 0; g < G; g += 64) {
@@ -412,14 +441,26 @@ static void gg_range(void* vctx, int64_t b, int64_t end) {
     free(h);
 }
 
-void orc_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
-                      const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
-                      int epilogue, void* D, float* Ds, int nthreads) {
+static void grouped_gemm(int w4, int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                         const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
+                         int epilogue, void* D, float* Ds, int nthreads) {
     gg_ctx c;
-    c.layout = layout; c.E = E; c.N = N; c.K = K; c.M_rows = M_rows; c.epilogue = epilogue;
+    c.layout = layout; c.E = E; c.N = N; c.K = K; c.M_rows = M_rows; c.epilogue = epilogue; c.w4 = w4;
     c.A = A; c.As = As; c.gi = group_info; c.B = B; c.Bs = Bs; c.D = D; c.Ds = Ds;
     c.nrows = (layout == 0) ? group_info[E] : (int64_t)E * M_rows;
     parallel_for(c.nrows, nthreads, gg_range, &c);
+}
+
+void orc_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                      const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
+                      int epilogue, void* D, float* Ds, int nthreads) {
+    grouped_gemm(0, layout, E, N, K, A, As, group_info, M_rows, B, Bs, epilogue, D, Ds, nthreads);
+}
+
+void orc_grouped_gemm_w4(int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                         const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
+                         int epilogue, void* D, float* Ds, int nthreads) {
+    grouped_gemm(1, layout, E, N, K, A, As, group_info, M_rows, B, Bs, epilogue, D, Ds, nthreads);
 }
 
 /* ------------------------------------------------------------------ */

@@ -15,7 +15,8 @@
  *       renormalisation inside the top-k), 3.2 / 4.2 (capacity, dropping).
  *  [P3] "DeepSeek-V4 lecture 4: routing, FP4 experts, parallelism"
  *       (tqpw.cn), 2.2 (hash routing hash(token_id) % num_experts),
- *       2.3 (fp32 softmax even for a bf16 model).
+ *       2.3 (fp32 softmax even for a bf16 model), 3.1 (4-bit expert
+ *       weights: per-channel blocks scaled by their max-abs, 7 levels a side).
  *  [P4] "DeepSeek MoE architecture" (mooersco.com), chapter 1 (top-2
  *       pseudo-code: top-k of the logits, softmax over the selected ones),
  *       2.5 (capacity = ceil(top-k * N / E) * alpha, worked example -> 76;
@@ -36,6 +37,10 @@
  *  - dequantisation to fp32 (code * scale rounded to fp32), fp64 sums,
  *    h = silu(a) * b in fp64 rounded to fp32 and requantised as above,
  *    o rounded to bf16 (RNE), y = fp64 weighted sum rounded to bf16;
+ *  - 4-bit expert weights ([P3] 3.1 gives the formula, not the block): the
+ *    block is one weight row (output channel) by 128 consecutive k, the
+ *    granularity of the activation scales and of the GEMM's K blocks; the
+ *    level rounds half to even; the stored scale is max-abs / 7 in fp32;
  *  - bias balancing ([P1] 2.2 gives the direction, the step size and the
  *    interval): an expert's load is the number of slots routed to it (before
  *    any capacity drop), summed over the interval; above the mean -> bias
@@ -89,6 +94,16 @@ void orc_expert_rows(int n, int H, int I, const uint8_t* xq, const float* xs,
 void orc_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                       const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
                       int epilogue, void* D, float* Ds, int nthreads);
+/* The same grouped GEMM with 4-bit weights ([P3] 3.1): B = [E, N, K/2] bytes,
+ * two codes each (even k in the low nibble, 4-bit two's complement, levels
+ * -7..7), Bs = [E, N, K/128] fp32 (one scale per weight row per 128-wide K
+ * block: max-abs / 7); a weight dequantises to code * scale in fp32. With the
+ * SwiGLU epilogue the rows of B follow the same W1/W3 128-row alternation. */
+void orc_grouped_gemm_w4(int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                         const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
+                         int epilogue, void* D, float* Ds, int nthreads);
+/* One 4-bit weight code: nibble `high` (0 = low) of `byte`, sign-extended. */
+int orc_w4_decode(uint8_t byte, int high);
 /* Combine: y[t,:] = sum_j [kept] w[t,j] * O[slot_row[t*k+j], :], fp64, -> bf16. */
 void orc_combine(int T, int k, int H, const int32_t* slot_row, const float* topk_w,
                  const uint16_t* O, uint16_t* y);
