@@ -2,9 +2,10 @@
 
 This module is shared by the CUDA path's tests and benchmark and by the CPU
 oracle's tests. It draws random data and lays it out; it holds none of the
-layer's arithmetic (routing, permutation, GEMM, SwiGLU, combine). The one
-piece of setup arithmetic here is the offline quantisation of the expert
-weights to E4M3 with one fp32 scale per 128x128 block: the layer receives its
+layer's arithmetic (routing, permutation, GEMM, SwiGLU, combine). The setup
+arithmetic here is the offline quantisation of the expert weights, to E4M3
+with one fp32 scale per 128x128 block (and, as a second format, to 4-bit
+levels with one scale per row per 128 k, quantize_weight_int4): the layer receives its
 weights already quantised (DeepGEMM's grouped call takes FP8 operands plus
 fine-grained scales; discosf.com "MegaMoE ... DeepGEMM" page, sections 3.2-3.3;
 DeepSeek open-source week page, "Day 3"), so weight quantisation is not a step
