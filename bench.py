@@ -307,6 +307,15 @@ def max_over_ranks(v: float, world: int) -> float:
     return float(t.item())
 
 
+def routing_stats(counts, kept) -> dict:
+    """Per-expert slot counts of the last step (the router's choice) and the slots the capacity dropped."""
+    counts = np.asarray(counts, dtype=np.int64)
+    kept = np.asarray(kept, dtype=np.int64)
+    return {"count_min": int(counts.min()), "count_max": int(counts.max()), "count_mean": float(counts.mean()),
+            "max_over_mean": float(counts.max() / max(counts.mean(), 1e-9)),
+            "dropped_slots": int(counts.sum() - kept.sum())}
+
+
 def job_tokens_per_s(tokens_per_rank: int, world: int, ms_max: float) -> float:
     """Whole-job throughput: every rank's tokens over the slowest rank's time per step."""
     return world * tokens_per_rank / (ms_max / 1e3)
@@ -478,6 +487,7 @@ def run_ours(args):
                  "frac_fp8_nominal_4500": gemm_tflops / 4500.0, "ms": gemm_ms, "rows_kept": Rk,
                  "experts_touched": touched},
         "kernels_ms": per,
+        "routing": routing_stats(layer.counts.cpu().numpy(), kept),
         "balance_bias": balance,
         "e2e": {"value": job_tokens_per_s(cfg.T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

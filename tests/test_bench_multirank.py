@@ -58,3 +58,11 @@ def test_two_gloo_ranks_take_the_max_time_and_count_every_rank():
         assert m == 4.0                                     # every rank sees the slowest rank's time
         assert value == pytest.approx(2 * 4096 / 4.0e-3)    # all ranks' tokens over that time
     assert res[1][3] == "returned"
+
+
+def test_routing_stats_counts_drops():
+    import numpy as np
+
+    import bench
+    st = bench.routing_stats(np.array([3, 5, 0, 8]), np.array([3, 4, 0, 6]))
+    assert st == {"count_min": 0, "count_max": 8, "count_mean": 4.0, "max_over_mean": 2.0, "dropped_slots": 3}

@@ -286,6 +286,45 @@ def test_grouped_gemm(case):
         assert np.allclose(s, sr, rtol=1e-5, atol=0)
 
 
+@pytest.mark.parametrize("layout,epi", [(0, 0), (0, 1), (1, 0), (1, 1)])
+def test_grouped_gemm_writes_nothing_outside_its_groups(layout, epi):
+    # canary-filled outputs with guard rows past the end: rows outside every group (contiguous) or at
+    # and past a block's count (masked) keep the canary, as do the guard rows and their scales
+    ensure_lib()
+    E, N, K = 3, 512, 256
+    groups, Mr = ([130, 0, 1], None) if layout == 0 else ([5, 0, 32], 64)
+    A, As, gi, M, B, Bs = _gemm_case(layout, epi, E, N, K, groups, Mr, seed=77)
+    rows = A.shape[0]
+    guard = 64
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    if epi == 0:
+        Dfull = torch.full((rows + guard, N), 0x5A5A, dtype=torch.int16, device="cuda")
+        Dsfull = None
+    else:
+        Dfull = torch.full((rows + guard, N // 2), 0x5A, dtype=torch.uint8, device="cuda")
+        G = N // 256
+        Dsfull = torch.full(((G, M) if layout == 0 else (E, G, M)), -3.0, dtype=torch.float32, device="cuda")
+    D = Dfull[:rows]
+    api.moe_grouped_gemm_fp8(layout, E, N, K, d(A), d(As), d(gi), M, d(B), d(Bs), epi, D, Dsfull)
+    torch.cuda.synchronize()
+    assert api.moe_get_device_status() == api.MOE_OK
+    Dh = to_np(Dfull)
+    canary = 0x5A5A if epi == 0 else 0x5A
+    valid = np.zeros(rows + guard, bool)
+    valid[_valid_rows(layout, gi, M, E)] = True
+    if layout == 0:
+        assert np.all(Dh[gi[-1]:] == canary)                       # past the last group, guard rows too
+        if epi == 1:
+            assert np.all(to_np(Dsfull)[:, gi[-1]:] == -3.0)
+    else:
+        assert np.all(Dh[~valid] == canary)
+        if epi == 1:
+            Ds = to_np(Dsfull)
+            for e in range(E):
+                assert np.all(Ds[e, :, gi[e]:] == -3.0)
+                assert np.all(Ds[e, :, :gi[e]] > 0)
+
+
 def test_combine_with_drops():
     ensure_lib()
     cfg = MoeConfig("comb", T=300, H=384, E=4, I=128, k=3, bias="uniform", cap_num=1, cap_den=2, seed=31)
