@@ -16,7 +16,7 @@ import pytest
 import torch
 
 import oracle
-from fp8_grouped_gemm_fp32_b200.inputs import MoeConfig, make_inputs, interleave_w13
+from fp8_grouped_gemm_fp32_b200.inputs import MoeConfig, interleave_w13, make_inputs, quantize_weight_int4
 
 
 def _deq_w(q, s):
@@ -183,3 +183,34 @@ def test_all_dropped_token_gives_zero():
     dropped = np.nonzero(out["slot_row"] < 0)[0]
     assert len(dropped) > 0
     assert np.all(out["y"][dropped] == 0)
+
+
+def test_results_do_not_depend_on_the_thread_count():
+    # the oracle splits work items (rows, columns) across threads, never a sum: 1, 3 and 8 threads
+    # give identical bits for the router, the grouped GEMM (both epilogues, both weight formats) and
+    # the expert rows
+    cfg = MoeConfig("thr", T=70, H=256, E=4, I=256, k=2, bias="uniform", seed=9)
+    t = make_inputs(cfg)
+    inp = oracle.moe_inputs_to_numpy(t)
+    logits = [oracle.router_logits(inp["x"], inp["Wg"], inp["bias"], nthreads=n) for n in (1, 3, 8)]
+    assert all(np.array_equal(logits[0].view(np.uint32), l.view(np.uint32)) for l in logits[1:])
+    idx, w, _ = oracle.route(cfg, inp["x"], inp["Wg"], inp["bias"], inp["token_ids"])
+    rows_cap = -(-(cfg.T * cfg.k + cfg.E * 127) // 128) * 128
+    d = oracle.permute(cfg, inp["x"], idx, rows_cap)
+    W13, S13 = interleave_w13(t.W1q, t.S1, t.W3q, t.S3)
+    q4, s4 = quantize_weight_int4(torch.randn(cfg.E * 2 * cfg.I, cfg.H, generator=torch.Generator().manual_seed(3)))
+    B4 = q4.numpy().reshape(cfg.E, 2 * cfg.I, cfg.H // 2)
+    S4 = s4.numpy().reshape(cfg.E, 2 * cfg.I, cfg.H // 128)
+    for B, Bs, w4 in ((W13.numpy(), S13.numpy(), False), (B4, S4, True)):
+        for epi in (0, 1):
+            outs = [oracle.grouped_gemm(0, cfg.E, 2 * cfg.I, cfg.H, d["Aq"], d["As"], d["offsets"], rows_cap, B, Bs,
+                                        epi, nthreads=n, w4=w4) for n in (1, 3, 8)]
+            for D, Ds in outs[1:]:
+                assert np.array_equal(D, outs[0][0])
+                assert Ds is None or np.array_equal(Ds.view(np.uint32), outs[0][1].view(np.uint32))
+    e, n = 0, int(d["kept"][0])
+    xs = np.ascontiguousarray(d["As"][:, :n].T)
+    rows = [oracle.expert_rows(d["Aq"][:n], xs, inp["W1q"][e], inp["S1"][e], inp["W3q"][e], inp["S3"][e],
+                               inp["W2q"][e], inp["S2"][e], nthreads=k) for k in (1, 3, 8)]
+    for r in rows[1:]:
+        assert all(np.array_equal(a, b) for a, b in zip(r, rows[0]))
