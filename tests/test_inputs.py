@@ -2,7 +2,6 @@
 arrays; the W1/W3 interleave is a pure re-layout (gate block j, then up block
 j); the E4M3 weight quantiser keeps every block within one E4M3 step of the
 fp32 weights; the row bound of the permuted buffers matches the C ABI's."""
-import numpy as np
 import torch
 
 from fp8_grouped_gemm_fp32_b200 import api
