@@ -219,8 +219,8 @@ def w4_decode(byte: int, high: bool) -> int:
 def grouped_gemm(layout: int, E: int, N: int, K: int, A, As, group_info, M_rows: int, B, Bs,
                  epilogue: int, nthreads: Optional[int] = None, w4: bool = False):
     """Oracle of moe_grouped_gemm_fp8. Rows outside every group are left 0. With w4, B holds
-    4-bit weight codes [E, N, K/2] and Bs one scale per weight row per 128-wide K block
-    [E, N, K/128] (DeepSeek-V4 lecture page, 3.1)."""
+    4-bit weight codes [E, N, K/2] and Bs one scale per weight row per 128-wide K block,
+    K-block-major [E, K/128, N] (DeepSeek-V4 lecture page, 3.1)."""
     A = _c(A, np.uint8)
     As = _c(As, np.float32)
     gi = _c(group_info, np.int32)

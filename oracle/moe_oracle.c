@@ -299,12 +299,14 @@ int orc_w4_decode(uint8_t byte, int high) {
 }
 
 /* As dot_row, with a row of 4-bit weight codes and the row's K/128 scales
- * (max-abs / 7 per block); the dequantised weight is code * scale in fp32. */
-static double dot_row_w4(int K, const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s) {
+ * (max-abs / 7 per block), w_s[kb * ws_stride]; the dequantised weight is
+ * code * scale in fp32. */
+static double dot_row_w4(int K, const uint8_t* a, const float* a_s, const uint8_t* w, const float* w_s,
+                         int64_t ws_stride) {
     double acc = 0.0;
     int kk;
     for (kk = 0; kk < K; ++kk) {
-        float wd = (float)orc_w4_decode(w[kk >> 1], kk & 1) * w_s[kk / GROUP];
+        float wd = (float)orc_w4_decode(w[kk >> 1], kk & 1) * w_s[(int64_t)(kk / GROUP) * ws_stride];
         acc += (double)deq(a[kk], a_s[kk / GROUP]) * (double)wd;
     }
     return acc;
@@ -388,13 +390,14 @@ static int gg_row_expert(const gg_ctx* c, int64_t row) {
 
 /* Output column n of expert e for one activation row: E4M3 weights are [E, N, K]
  * with scales [E, N/128, K/128]; 4-bit weights are [E, N, K/2] with scales
- * [E, N, K/128]. */
+ * [E, K/128, N] (K-block-major: the scales of one K block for consecutive rows
+ * lie together). */
 static double gg_dot(const gg_ctx* c, const uint8_t* ar, const float* a_s, int e, int64_t n) {
     const int K = c->K, KB = K / GROUP;
     const int64_t row = (int64_t)e * c->N + n;
     if (!c->w4)
         return dot_row(K, ar, a_s, c->B + row * K, c->Bs + ((int64_t)e * (c->N / GROUP) + n / GROUP) * KB);
-    return dot_row_w4(K, ar, a_s, c->B + row * (K / 2), c->Bs + row * KB);
+    return dot_row_w4(K, ar, a_s, c->B + row * (K / 2), c->Bs + (int64_t)e * KB * c->N + n, c->N);
 }
 
 static void gg_range(void* vctx, int64_t b, int64_t end) {

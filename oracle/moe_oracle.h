@@ -96,8 +96,9 @@ void orc_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const f
                       int epilogue, void* D, float* Ds, int nthreads);
 /* The same grouped GEMM with 4-bit weights ([P3] 3.1): B = [E, N, K/2] bytes,
  * two codes each (even k in the low nibble, 4-bit two's complement, levels
- * -7..7), Bs = [E, N, K/128] fp32 (one scale per weight row per 128-wide K
- * block: max-abs / 7); a weight dequantises to code * scale in fp32. With the
+ * -7..7), Bs = [E, K/128, N] fp32 (one scale per weight row per 128-wide K
+ * block: max-abs / 7, K-block-major); a weight dequantises to code * scale in
+ * fp32. With the
  * SwiGLU epilogue the rows of B follow the same W1/W3 128-row alternation. */
 void orc_grouped_gemm_w4(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                          const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,

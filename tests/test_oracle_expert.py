@@ -200,7 +200,7 @@ def test_results_do_not_depend_on_the_thread_count():
     W13, S13 = interleave_w13(t.W1q, t.S1, t.W3q, t.S3)
     q4, s4 = quantize_weight_int4(torch.randn(cfg.E * 2 * cfg.I, cfg.H, generator=torch.Generator().manual_seed(3)))
     B4 = q4.numpy().reshape(cfg.E, 2 * cfg.I, cfg.H // 2)
-    S4 = s4.numpy().reshape(cfg.E, 2 * cfg.I, cfg.H // 128)
+    S4 = np.ascontiguousarray(s4.numpy().reshape(cfg.E, 2 * cfg.I, cfg.H // 128).transpose(0, 2, 1))
     for B, Bs, w4 in ((W13.numpy(), S13.numpy(), False), (B4, S4, True)):
         for epi in (0, 1):
             outs = [oracle.grouped_gemm(0, cfg.E, 2 * cfg.I, cfg.H, d["Aq"], d["As"], d["offsets"], rows_cap, B, Bs,

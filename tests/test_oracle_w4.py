@@ -114,7 +114,9 @@ def _rand_e4m3(rng, shape):
 def _w4_weights(rng, E, N, K):
     w = torch.from_numpy(rng.standard_normal((E * N, K)).astype(np.float32) * 0.02)
     codes, scale = quantize_weight_int4(w)
-    return codes.numpy().reshape(E, N, K // 2), scale.numpy().reshape(E, N, K // 128)
+    # scales K-block-major, [E, K/128, N]
+    return codes.numpy().reshape(E, N, K // 2), np.ascontiguousarray(scale.numpy().reshape(E, N, K // 128)
+                                                                      .transpose(0, 2, 1))
 
 
 def _a_deq(A, As_rows):
@@ -164,7 +166,7 @@ def test_w4_grouped_gemm_equals_dense_fp64(layout):
         if len(rows) == 0:
             continue
         a = _a_deq(A[rows], np.ascontiguousarray(as_rows))
-        wd = _deq_w4(B[e], Bs[e])
+        wd = _deq_w4(B[e], Bs[e].T)
         ref = (a @ wd.T).numpy()
         _close_bf16(D[rows], ref)
         gate = torch.cat([wd[2 * j * 128:(2 * j + 1) * 128] for j in range(I // 128)])
