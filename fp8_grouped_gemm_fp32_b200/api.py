@@ -30,7 +30,7 @@ LAYOUT_CONTIGUOUS, LAYOUT_MASKED = 0, 1
 EPI_BF16, EPI_SWIGLU_FP8 = 0, 1
 EXPORTS = ("moe_rows_capacity", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_gemm_fp8",
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string",
-           "moe_permute_noalloc", "moe_balance_bias")
+           "moe_permute_noalloc", "moe_balance_bias", "moe_grouped_gemm_w4")
 
 
 class MoeError(RuntimeError):
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.moe_permute.argtypes = [CP, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.moe_permute_noalloc.argtypes = [CP, P, P, P, P, P, P, P, P, P, P]
         L.moe_grouped_gemm_fp8.argtypes = [I, I, I, I, P, P, P, I, P, P, I, P, P, P]
+        L.moe_grouped_gemm_w4.argtypes = [I, I, I, I, P, P, P, I, P, P, I, P, P, P]
         L.moe_combine.argtypes = [CP, P, P, P, P, P]
         L.moe_forward.argtypes = [CP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.moe_balance_bias.argtypes = [I, P, P, P, ctypes.c_float, I, P]
@@ -142,6 +143,12 @@ def moe_permute_noalloc(cfg, x, topk_idx, Aq, As, counts, kept, offsets, row_src
 def moe_grouped_gemm_fp8(layout, E, N, K, A, As, group_info, M_rows, B, Bs, epilogue, D, Ds=None, stream=None):
     _check(lib().moe_grouped_gemm_fp8(layout, E, N, K, _p(A), _p(As), _p(group_info), M_rows, _p(B), _p(Bs),
                                       epilogue, _p(D), _p(Ds), _stream(stream)), "moe_grouped_gemm_fp8")
+
+
+def moe_grouped_gemm_w4(layout, E, N, K, A, As, group_info, M_rows, B, Bs, epilogue, D, Ds=None, stream=None):
+    """moe_grouped_gemm_fp8 with 4-bit weights: B [E, N, K/2] packed levels, Bs [E, K/128, N] row scales."""
+    _check(lib().moe_grouped_gemm_w4(layout, E, N, K, _p(A), _p(As), _p(group_info), M_rows, _p(B), _p(Bs),
+                                     epilogue, _p(D), _p(Ds), _stream(stream)), "moe_grouped_gemm_w4")
 
 
 def moe_combine(cfg, O, slot_row, topk_w, y, stream=None):

@@ -25,6 +25,9 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, int T, in
 cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                                 const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs, int epilogue,
                                 void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s);
+cudaError_t launch_grouped_gemm_w4(int E, int N, int K, const uint8_t* A, const float* As, const int32_t* masked_m,
+                                   int M_rows, const uint8_t* B, const float* Bs, int epilogue, void* D, float* Ds,
+                                   int* status, uint64_t wait_ns, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t* O, const int32_t* slot_row, const float* topk_w, int T, int k, int H,
                            uint16_t* y, cudaStream_t s);
 cudaError_t launch_selftest_wait(int* status, uint64_t wait_ns, cudaStream_t s);
@@ -236,6 +239,29 @@ moe_status_t moe_grouped_gemm_fp8(int layout, int E, int N, int K, const uint8_t
     if ((st = device_info(&dev)) != MOE_OK) return st;
     return cuda_status(launch_grouped_gemm(layout, E, N, K, A, As, group_info, M_rows, B, Bs, epilogue, D, Ds,
                                            dev->status, kWaitNs, dev->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_gemm_w4(int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                                 const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
+                                 int epilogue, void* D, float* Ds, void* stream) {
+    if (layout != MOE_LAYOUT_CONTIGUOUS && layout != MOE_LAYOUT_MASKED) return MOE_ERR_INVALID_ARG;
+    if (epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_SWIGLU_FP8) return MOE_ERR_INVALID_ARG;
+    if (E <= 0 || N <= 0 || K <= 0 || M_rows <= 0) return MOE_ERR_INVALID_ARG;
+    if (layout != MOE_LAYOUT_MASKED) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (E > MOE_MAX_EXPERTS || N % kGroup || K % kGroup) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (epilogue == MOE_EPI_SWIGLU_FP8 && N % (2 * kGroup)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (K > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (M_rows % 32) return MOE_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(E) * N >= (1ll << 31) || static_cast<int64_t>(E) * M_rows >= (1ll << 31))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!ptr_ok(A) || !ptr_ok(As) || !ptr_ok(group_info) || !ptr_ok(B) || !ptr_ok(Bs) || !ptr_ok(D))
+        return MOE_ERR_INVALID_ARG;
+    if (epilogue == MOE_EPI_SWIGLU_FP8 && !ptr_ok(Ds)) return MOE_ERR_INVALID_ARG;
+    moe_status_t st;
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    return cuda_status(launch_grouped_gemm_w4(E, N, K, A, As, group_info, M_rows, B, Bs, epilogue, D, Ds, dev->status,
+                                              kWaitNs, dev->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_combine(const moe_config_t* cfg, const void* O, const int32_t* slot_row, const float* topk_w,

@@ -28,7 +28,12 @@
 // * masked layout (decode, few tokens per expert): swap-AB. The weight block
 //   is the MMA's M=128 operand and up to 32 tokens are its N, so weights
 //   stream from HBM in 16 KB (or 2 x 16 KB) stages while the token tile is
-//   tiny; experts with no tokens produce no tiles.
+//   tiny; experts with no tokens produce no tiles. A second weight format,
+//   4-bit levels -7..7 with one fp32 scale per weight row per 128-wide K
+//   block (DeepSeek-V4 lecture page, 3.1), runs through the same kernel:
+//   TMA brings the packed levels, four converter warps expand them to E4M3
+//   codes (every level is exact in E4M3) in the swizzled layout the MMA
+//   reads, and each promotion thread applies its own row's scale.
 //
 // Every wait on an mbarrier is bounded; a wait that runs out records
 // MOE_ERR_DEVICE_TIMEOUT, the CTA stops issuing work, lets copies and MMAs in
@@ -451,22 +456,43 @@ constexpr int kWBlk = kBM * kBK;              // 16 KB: 128 weight rows x 128 K 
 // threads: warp 0 TMA, warp 1 MMA, then the promotion warps: four for SwiGLU (a thread holds a weight
 // row's 32 gate and 32 up columns), eight for the bf16 output (two warps per lane quadrant, 16 token
 // columns each, so two warps share each scheduler's promotion work)
-template <int EPI>
-__host__ __device__ constexpr int masked_threads() { return EPI == 1 ? 192 : 320; }
+// With 4-bit weights (W4) four more warps expand each stage's packed levels to E4M3 codes.
+template <int EPI, bool W4 = false>
+__host__ __device__ constexpr int masked_threads() { return (EPI == 1 ? 192 : 320) + (W4 ? 128 : 0); }
 
-template <int EPI>
+// 4-bit weight levels, four per 16 bits in k order (4-bit two's complement), to four E4M3 codes: one
+// byte permute reads the codes of 0..7, one the codes of -8..-1, and one in sign-replicate mode builds
+// the byte mask of the negative levels.
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t w4x4_to_e4m3x4(uint32_t h) {
+    const uint32_t sel = h & 0x7777u;
+    const uint32_t pos = prmt_b32(0x44403800u, 0x4e4c4a48u, sel);
+    const uint32_t neg = prmt_b32(0xcaccced0u, 0xb8c0c4c8u, sel);
+    const uint32_t sg = h & 0x8888u;
+    const uint32_t mask = prmt_b32(0x00008000u, 0u, sg | (sg >> 3));
+    return (pos & ~mask) | (neg & mask);
+}
+
+template <int EPI, bool W4 = false>
 struct SmemM {
     static constexpr int kW = EPI == 1 ? 2 * kWBlk : kWBlk;    // weight rows per stage: 256 (a|b) or 128
-    static constexpr int kStages = EPI == 1 ? 4 : 10;
+    static constexpr int kStages = W4 ? (EPI == 1 ? 3 : 6) : (EPI == 1 ? 4 : 10);
+    static constexpr int kWP = W4 ? kW / 2 : 16;               // packed 4-bit levels per stage
     static constexpr int kCols = EPI == 1 ? 2 * kBT : kBT;     // tensor-memory columns per buffer
     static constexpr int kBufs = 4;                            // MMA runs up to 3 K blocks ahead of promotion
     static constexpr int kSaSlots = 16;                        // scale ring deeper than the stage ring
     uint8_t w[kStages][kW];
     uint8_t x[kStages][kXBytes];
+    uint8_t wp[kStages][kWP];                                   // packed levels (W4), 64 bytes per row
     float hs[EPI == 1 ? 2 : 1][EPI == 1 ? kBT : 1][kBM];       // SwiGLU output staged for the requant
     float sa[kSaSlots][kBT];                                    // activation scales of one K block, 32 tokens
     uint64_t full[kStages];
     uint64_t empty[kStages];
+    uint64_t conv[kStages];                                     // W4: the stage's levels are expanded
     uint64_t sfull[kSaSlots];
     uint64_t sempty[kSaSlots];
     uint64_t tfull[kBufs];
@@ -478,16 +504,18 @@ struct SmemM {
     int32_t M[kMaxE];                                           // tokens per expert (masked_m)
 };
 
-template <int EPI>
-__global__ void __launch_bounds__(masked_threads<EPI>(), 1)
+template <int EPI, bool W4>
+__global__ void __launch_bounds__(masked_threads<EPI, W4>(), 1)
 gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ As, const int32_t* __restrict__ masked_m, int Mmax,
                  const float* __restrict__ Bs, int E, int N, int K, void* __restrict__ D, float* __restrict__ Ds,
                  int* status, uint64_t wait_ns) {
-    using S = SmemM<EPI>;
+    using S = SmemM<EPI, W4>;
     extern __shared__ uint8_t smem_raw[];
     S& sm = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kPW = EPI == 1 ? 4 : 8;                      // promotion warps (2 .. 2 + kPW - 1)
+    constexpr int kConvWarp0 = 2 + kPW;                        // W4: converter warps, four of them
     const int KB = K / kBK;
     const int NB = N / kBM;                          // 128-row weight blocks per expert
     const int NBt = EPI == 1 ? NB / 2 : NB;          // weight tiles per expert
@@ -515,8 +543,8 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         for (int s = 0; s < S::kStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
+            if (W4) mbar_init(&sm.conv[s], 4);
         }
-        constexpr int kPW = (masked_threads<EPI>() - 64) / 32;   // promotion warps
         for (int j = 0; j < S::kSaSlots; ++j) {
             mbar_init(&sm.sfull[j], 1);
             mbar_init(&sm.sempty[j], kPW);
@@ -565,9 +593,15 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     const int s = it % S::kStages;
                     const uint32_t ph = (it / S::kStages) & 1;
                     if (!mbar_wait(&sm.empty[s], ph ^ 1, wait_ns)) { fail(); break; }
-                    mbar_arrive_expect_tx(&sm.full[s], S::kW + kXBytes);
-                    tma_load_2d(sm.w[s], &tmW, &sm.full[s], kb * kBK, wrow);
-                    if (EPI == 1) tma_load_2d(sm.w[s] + kWBlk, &tmW, &sm.full[s], kb * kBK, wrow + kBM);
+                    if constexpr (W4) {
+                        mbar_arrive_expect_tx(&sm.full[s], S::kWP + kXBytes);
+                        tma_load_2d(sm.wp[s], &tmW, &sm.full[s], kb * (kBK / 2), wrow);
+                        if (EPI == 1) tma_load_2d(sm.wp[s] + kWBlk / 2, &tmW, &sm.full[s], kb * (kBK / 2), wrow + kBM);
+                    } else {
+                        mbar_arrive_expect_tx(&sm.full[s], S::kW + kXBytes);
+                        tma_load_2d(sm.w[s], &tmW, &sm.full[s], kb * kBK, wrow);
+                        if (EPI == 1) tma_load_2d(sm.w[s] + kWBlk, &tmW, &sm.full[s], kb * kBK, wrow + kBM);
+                    }
                     tma_load_2d(sm.x[s], &tmX, &sm.full[s], kb * kBK, e * Mmax + tt * kBT);
                     // the token tile's 32 activation scales of this K block, into the scale ring
                     const int j = it % S::kSaSlots;
@@ -589,6 +623,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     const int buf = kbt % S::kBufs;
                     const uint32_t bph = (kbt / S::kBufs) & 1;
                     if (!mbar_wait(&sm.full[s], ph, wait_ns)) { fail(); break; }
+                    if (W4 && !mbar_wait(&sm.conv[s], ph, wait_ns)) { fail(); break; }
                     if (!mbar_wait(&sm.tempty[buf], bph ^ 1, wait_ns)) { fail(); break; }
                     tc_fence_after();
                     const uint32_t w0 = smem_u32(sm.w[s]), x0 = smem_u32(sm.x[s]);
@@ -602,6 +637,37 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     umma_commit(&sm.empty[s]);
                     umma_commit(&sm.tfull[buf]);
                 }
+            }
+        }
+    } else if (W4 && warp >= kConvWarp0) {
+        // expansion of each stage's packed levels: thread ct takes 16-byte chunk cc of rows cr + 16 j, so
+        // a warp reads four whole packed rows and writes four whole 128-byte rows in the 128-byte
+        // swizzled layout the MMA descriptor reads (chunk c of row r at c ^ (r & 7))
+        const int ct = threadIdx.x - kConvWarp0 * 32;
+        const int cr = ct >> 3, cc = ct & 7;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb, ++it) {
+                if (sm.abort_flag) { ok = false; break; }
+                const int s = it % S::kStages;
+                const uint32_t ph = (it / S::kStages) & 1;
+                if (!mbar_wait(&sm.full[s], ph, wait_ns)) { fail(); ok = false; break; }
+#pragma unroll
+                for (int b = 0; b < (EPI == 1 ? 2 : 1); ++b) {
+                    const uint8_t* src = sm.wp[s] + b * (kWBlk / 2);
+                    const uint32_t dst = smem_u32(sm.w[s] + b * kWBlk);
+#pragma unroll
+                    for (int j = 0; j < kBM / 16; ++j) {
+                        const int r = cr + 16 * j;
+                        const uint2 p = *reinterpret_cast<const uint2*>(src + r * (kBK / 2) + cc * 8);
+                        st_shared_v4(dst + r * kBK + ((cc ^ (r & 7)) << 4), w4x4_to_e4m3x4(p.x),
+                                     w4x4_to_e4m3x4(p.x >> 16), w4x4_to_e4m3x4(p.y), w4x4_to_e4m3x4(p.y >> 16));
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.conv[s]);
             }
         }
     } else {
@@ -628,7 +694,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 wb[i] = EPI == 1 && kb < KB ? pa[KB + kb] : 0.0f;
             }
         };
-        load_w(blockIdx.x);
+        if constexpr (!W4) load_w(blockIdx.x);
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             if (sm.abort_flag) break;
             int e, nb, tt, m_e;
@@ -638,7 +704,14 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             for (int i = 0; i < (EPI == 1 ? 2 * kBT : kC); ++i) acc[i] = 0.0f;
             const float wta[4] = {wa[0], wa[1], wa[2], wa[3]};
             const float wtb[4] = {wb[0], wb[1], wb[2], wb[3]};
-            load_w(tile + gridDim.x);
+            if constexpr (!W4) load_w(tile + gridDim.x);
+            // W4: this thread's weight row(s) carry their own scale per K block, [E, K/128, N]
+            const float* wsr = Bs + static_cast<int64_t>(e) * KB * N + (EPI == 1 ? 2 * nb : nb) * kBM + r;
+            float nsa = 0.0f, nsb = 0.0f;
+            if constexpr (W4) {
+                nsa = wsr[0];
+                if (EPI == 1) nsb = wsr[kBM];
+            }
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb, ++kbt) {
                 const int buf = kbt % S::kBufs;
@@ -654,12 +727,22 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.sempty[j]);
-                const int wi = kb >> 5;
-                const float swa = __shfl_sync(0xffffffffu, wi == 0 ? wta[0] : wi == 1 ? wta[1] : wi == 2 ? wta[2] : wta[3],
-                                              kb & 31);
-                const float swb = EPI == 1 ? __shfl_sync(0xffffffffu, wi == 0 ? wtb[0] : wi == 1 ? wtb[1]
-                                                                      : wi == 2 ? wtb[2] : wtb[3], kb & 31)
-                                           : 0.0f;
+                float swa, swb;
+                if constexpr (W4) {
+                    swa = nsa;
+                    swb = nsb;
+                    if (kb + 1 < KB) {
+                        nsa = wsr[static_cast<int64_t>(kb + 1) * N];
+                        if (EPI == 1) nsb = wsr[static_cast<int64_t>(kb + 1) * N + kBM];
+                    }
+                } else {
+                    const int wi = kb >> 5;
+                    swa = __shfl_sync(0xffffffffu, wi == 0 ? wta[0] : wi == 1 ? wta[1] : wi == 2 ? wta[2] : wta[3],
+                                      kb & 31);
+                    swb = EPI == 1 ? __shfl_sync(0xffffffffu, wi == 0 ? wtb[0] : wi == 1 ? wtb[1]
+                                                              : wi == 2 ? wtb[2] : wtb[3], kb & 31)
+                                   : 0.0f;
+                }
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * S::kCols;
@@ -810,17 +893,54 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
         if (!make_map(&mapB, B, K, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
         if (epilogue == 0) {
             const size_t smem = sizeof(SmemM<0>) + 1024;
-            cudaError_t err = set_smem(gg_masked_kernel<0>, smem);
+            cudaError_t err = set_smem(gg_masked_kernel<0, false>, smem);
             if (err != cudaSuccess) return err;
-            gg_masked_kernel<0><<<num_sms, masked_threads<0>(), smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
+            gg_masked_kernel<0, false><<<num_sms, masked_threads<0>(), smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
                                                                   Ds, status, wait_ns);
         } else {
             const size_t smem = sizeof(SmemM<1>) + 1024;
-            cudaError_t err = set_smem(gg_masked_kernel<1>, smem);
+            cudaError_t err = set_smem(gg_masked_kernel<1, false>, smem);
             if (err != cudaSuccess) return err;
-            gg_masked_kernel<1><<<num_sms, masked_threads<1>(), smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
+            gg_masked_kernel<1, false><<<num_sms, masked_threads<1>(), smem, s>>>(mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D,
                                                                   Ds, status, wait_ns);
         }
+    }
+    return cudaGetLastError();
+}
+
+// 2-D map over a row-major byte matrix [rows, cols] read in boxes of 64 bytes x box_rows, unswizzled
+// (4-bit weights: 64 bytes hold a row's 128 levels of one K block).
+static bool make_packed_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = tensor_map_encoder();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK / 2), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Masked layout with 4-bit weights: B = [E, N, K/2] packed levels, Bs = [E, K/128, N] row scales.
+cudaError_t launch_grouped_gemm_w4(int E, int N, int K, const uint8_t* A, const float* As, const int32_t* masked_m,
+                                   int M_rows, const uint8_t* B, const float* Bs, int epilogue, void* D, float* Ds,
+                                   int* status, uint64_t wait_ns, int num_sms, cudaStream_t s) {
+    CUtensorMap mapA, mapB;
+    if (!make_map(&mapA, A, K, static_cast<uint64_t>(E) * M_rows, kBT)) return cudaErrorInvalidValue;
+    if (!make_packed_map(&mapB, B, K / 2, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
+    if (epilogue == 0) {
+        const size_t smem = sizeof(SmemM<0, true>) + 1024;
+        cudaError_t err = set_smem(gg_masked_kernel<0, true>, smem);
+        if (err != cudaSuccess) return err;
+        gg_masked_kernel<0, true><<<num_sms, masked_threads<0, true>(), smem, s>>>(mapA, mapB, As, masked_m, M_rows, Bs,
+                                                                                 E, N, K, D, Ds, status, wait_ns);
+    } else {
+        const size_t smem = sizeof(SmemM<1, true>) + 1024;
+        cudaError_t err = set_smem(gg_masked_kernel<1, true>, smem);
+        if (err != cudaSuccess) return err;
+        gg_masked_kernel<1, true><<<num_sms, masked_threads<1, true>(), smem, s>>>(mapA, mapB, As, masked_m, M_rows, Bs,
+                                                                                 E, N, K, D, Ds, status, wait_ns);
     }
     return cudaGetLastError();
 }

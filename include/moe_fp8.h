@@ -16,7 +16,9 @@
  *   moe_combine          weighted un-permute y = sum_j w_j * o_j
  *   moe_forward          all of the above on one stream, no host sync
  * and, for training, moe_balance_bias: the auxiliary-loss-free update of the
- * routing bias b from the per-expert counts moe_permute reports.
+ * routing bias b from the per-expert counts moe_permute reports; and
+ * moe_grouped_gemm_w4: the grouped GEMM with 4-bit expert weights (masked
+ * layout).
  *
  * Conventions (every entry point):
  *  - Every array argument is a DEVICE pointer owned by the caller, except the
@@ -171,6 +173,27 @@ moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* 
 moe_status_t moe_grouped_gemm_fp8(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                                   const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
                                   int epilogue, void* D, float* Ds, void* stream);
+
+/*
+ * The same grouped GEMM with 4-bit expert weights, masked layout. Source:
+ * DeepSeek-V4 lecture page, section 3.1: expert weights cut into per-channel
+ * blocks, each scaled by its max-abs, stored as the integer levels
+ * round((w / max|w|) * (2^3 - 1)) in 4 bits.
+ *   layout      MOE_LAYOUT_MASKED only (MOE_ERR_UNSUPPORTED_SHAPE otherwise);
+ *               A, As, group_info (masked_m), M_rows, epilogue, D and Ds as in
+ *               moe_grouped_gemm_fp8
+ *   B           [E, N, K/2] u8: two levels per byte, the even k in the low
+ *               nibble, each a 4-bit two's-complement integer in -7..7
+ *   Bs          [E, K/128, N] fp32 (K-block-major): the scale of weight row n
+ *               for K block kb, max-abs / 7 of its 128 weights; a weight is
+ *               level * scale
+ * N, K and M_rows follow moe_grouped_gemm_fp8's masked-layout rules. The
+ * levels are expanded to E4M3 codes on the chip (all of -7..7 are exact), so
+ * the arithmetic is the FP8 GEMM's with per-row weight scales.
+ */
+moe_status_t moe_grouped_gemm_w4(int layout, int E, int N, int K, const uint8_t* A, const float* As,
+                                 const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
+                                 int epilogue, void* D, float* Ds, void* stream);
 
 /*
  * Combine. Source: y = sum_{i in TopK} G(x)_i * E_i(x) (MegaMoE page,

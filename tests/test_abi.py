@@ -86,6 +86,18 @@ def test_hash_routing_needs_k1_and_masked_needs_rows(L):
     assert api.moe_workspace_size(c) == 0
 
 
+@pytest.mark.parametrize("layout,N,K,M_rows,epi,code", [
+    (0, 256, 256, 128, 0, api.MOE_ERR_UNSUPPORTED_SHAPE),      # 4-bit weights: masked layout only
+    (1, 200, 256, 32, 0, api.MOE_ERR_UNSUPPORTED_SHAPE),
+    (1, 384, 256, 32, 1, api.MOE_ERR_UNSUPPORTED_SHAPE),
+    (1, 256, 16512, 32, 0, api.MOE_ERR_UNSUPPORTED_SHAPE),
+    (1, 256, 256, 48, 0, api.MOE_ERR_INVALID_ARG),
+    (1, 256, 256, 32, 2, api.MOE_ERR_INVALID_ARG)])
+def test_bad_w4_gemm_shape_rejected_before_any_device_work(L, layout, N, K, M_rows, epi, code):
+    p = ctypes.c_void_p(4096)
+    assert L.moe_grouped_gemm_w4(layout, 4, N, K, p, p, p, M_rows, p, p, epi, p, p, None) == code
+
+
 @pytest.mark.parametrize("E,gamma,ptr,code", [
     (0, 1e-3, 4096, api.MOE_ERR_INVALID_ARG), (513, 1e-3, 4096, api.MOE_ERR_UNSUPPORTED_SHAPE),
     (8, float("nan"), 4096, api.MOE_ERR_INVALID_ARG), (8, float("inf"), 4096, api.MOE_ERR_INVALID_ARG),

@@ -7,7 +7,8 @@
 * moe_grouped_gemm_fp8: both layouts x both epilogues on ragged groups
   (empty groups, 1 row, tiles plus a ragged tail, a half-width N tile);
 * moe_combine (fed the oracle's expert outputs), with dropped slots;
-* moe_balance_bias: tallies and biases bit-exact over a sequence of steps.
+* moe_balance_bias: tallies and biases bit-exact over a sequence of steps;
+* moe_grouped_gemm_w4: the masked GEMM with 4-bit weights, both epilogues.
 """
 from types import SimpleNamespace
 
@@ -283,6 +284,54 @@ def test_grouped_gemm(case):
         else:
             s = np.concatenate([Ds[e, :, :gi[e]] for e in range(E)], axis=1)
             sr = np.concatenate([Dsr[e, :, :gi[e]] for e in range(E)], axis=1)
+        assert np.allclose(s, sr, rtol=1e-5, atol=0)
+
+
+W4_CASES = [
+    # E, N, K, masked_m, M_rows, epilogue, seed: empty and full blocks, ragged token tiles, the largest K
+    (4, 256, 384, [0, 5, 32, 64], 64, 0, 1),
+    (4, 512, 384, [7, 0, 33, 64], 64, 1, 2),
+    (3, 384, 1024, [1, 31, 64], 64, 0, 3),
+    (2, 256, 16384, [5, 32], 32, 0, 4),
+    (2, 512, 16384, [32, 9], 32, 1, 5),
+]
+
+
+@pytest.mark.parametrize("case", W4_CASES)
+def test_grouped_gemm_w4(case):
+    # 4-bit weights (levels -7..7, a scale per weight row per K block) through the masked kernel
+    ensure_lib()
+    from fp8_grouped_gemm_fp32_b200.inputs import quantize_weight_int4
+    E, N, K, mm, M, epi, seed = case
+    rng = np.random.default_rng(seed)
+    A = _rand_codes(rng, (E * M, K))
+    As = rng.uniform(0.002, 0.02, (E, K // 128, M)).astype(np.float32)
+    q, s4 = quantize_weight_int4(torch.from_numpy(rng.standard_normal((E * N, K)).astype(np.float32) * 0.02))
+    B = q.numpy().reshape(E, N, K // 2)
+    Bs = np.ascontiguousarray(s4.numpy().reshape(E, N, K // 128).transpose(0, 2, 1))
+    gi = np.array(mm, np.int32)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    if epi == 0:
+        D = torch.zeros(E * M, N, dtype=torch.bfloat16, device="cuda")
+        Ds = None
+    else:
+        D = torch.zeros(E * M, N // 2, dtype=torch.uint8, device="cuda")
+        Ds = torch.zeros(E, N // 256, M, dtype=torch.float32, device="cuda")
+    api.moe_grouped_gemm_w4(1, E, N, K, d(A), d(As), d(gi), M, d(B), d(Bs), epi, D, Ds)
+    torch.cuda.synchronize()
+    assert api.moe_get_device_status() == api.MOE_OK
+    Dr, Dsr = oracle.grouped_gemm(1, E, N, K, A, As, gi, M, B, Bs, epi, w4=True)
+    rows = _valid_rows(1, gi, M, E)
+    Dg = to_np(D)
+    if epi == 0:
+        assert_close_bf16(Dg[rows], Dr[rows], "D")
+        assert np.mean(Dg[rows] == Dr[rows]) > 0.95
+    else:
+        same = Dg[rows] == Dr[rows]
+        assert same.mean() > 0.999, same.mean()
+        assert np.all(np.abs(Dg[rows].astype(np.int32) - Dr[rows].astype(np.int32))[~same] == 1)
+        s = np.concatenate([to_np(Ds)[e, :, :gi[e]] for e in range(E)], axis=1)
+        sr = np.concatenate([Dsr[e, :, :gi[e]] for e in range(E)], axis=1)
         assert np.allclose(s, sr, rtol=1e-5, atol=0)
 
 
