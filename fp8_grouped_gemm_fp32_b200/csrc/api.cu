@@ -37,6 +37,39 @@ cudaError_t launch_balance_bias(int E, const int32_t* counts, int64_t* load, flo
 // The device status word (one per device that loads the library).
 __device__ int g_status;
 
+// Configuration rules shared by every entry point that takes a moe_config_t (moe_permute and its
+// workspace-free twin included), the capacity they imply and the rows of the permuted buffers.
+moe_status_t check_cfg(const moe_config_t* c) {
+    if (!c) return MOE_ERR_INVALID_ARG;
+    if (c->T < 0 || c->H <= 0 || c->I <= 0 || c->E <= 0 || c->k <= 0) return MOE_ERR_INVALID_ARG;
+    if (c->H % kGroup || c->I % kGroup || c->H > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->E > MOE_MAX_EXPERTS || c->k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->k > c->E) return MOE_ERR_INVALID_ARG;
+    if (c->routing != MOE_ROUTE_SOFTMAX_TOPK && c->routing != MOE_ROUTE_HASH) return MOE_ERR_INVALID_ARG;
+    if (c->routing == MOE_ROUTE_HASH && c->k != 1) return MOE_ERR_INVALID_ARG;
+    if (c->cap_num < 0 || c->cap_den < 0 || ((c->cap_num == 0) != (c->cap_den == 0))) return MOE_ERR_INVALID_ARG;
+    if (c->layout != MOE_LAYOUT_CONTIGUOUS && c->layout != MOE_LAYOUT_MASKED) return MOE_ERR_INVALID_ARG;
+    if (c->layout == MOE_LAYOUT_MASKED && (c->masked_max_m <= 0 || c->masked_max_m % 32)) return MOE_ERR_INVALID_ARG;
+    const int64_t rows = c->layout == MOE_LAYOUT_MASKED
+                             ? static_cast<int64_t>(c->E) * c->masked_max_m
+                             : static_cast<int64_t>(c->T) * c->k + static_cast<int64_t>(c->E) * (kGroup - 1);
+    if (rows >= (1ll << 31) / kGroup) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+int64_t capacity_of(const moe_config_t* c) {
+    if (c->cap_num == 0) return -1;
+    const int64_t R = static_cast<int64_t>(c->T) * c->k;
+    return (R + c->E - 1) / c->E * c->cap_num / c->cap_den;
+}
+
+size_t rows_of(const moe_config_t* c) {
+    if (c->layout == MOE_LAYOUT_MASKED) return static_cast<size_t>(c->E) * c->masked_max_m;
+    const size_t r = static_cast<size_t>(c->T) * c->k + static_cast<size_t>(c->E) * (kGroup - 1);
+    return (r + kGroup - 1) / kGroup * kGroup;
+}
+
+
 namespace {
 
 constexpr uint64_t kWaitNs = 4000000000ull;   // a legitimate wait never comes near 4 s
@@ -77,36 +110,6 @@ moe_status_t device_info(DeviceInfo** out) {
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 inline bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
-
-moe_status_t check_cfg(const moe_config_t* c) {
-    if (!c) return MOE_ERR_INVALID_ARG;
-    if (c->T < 0 || c->H <= 0 || c->I <= 0 || c->E <= 0 || c->k <= 0) return MOE_ERR_INVALID_ARG;
-    if (c->H % kGroup || c->I % kGroup || c->H > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (c->E > MOE_MAX_EXPERTS || c->k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (c->k > c->E) return MOE_ERR_INVALID_ARG;
-    if (c->routing != MOE_ROUTE_SOFTMAX_TOPK && c->routing != MOE_ROUTE_HASH) return MOE_ERR_INVALID_ARG;
-    if (c->routing == MOE_ROUTE_HASH && c->k != 1) return MOE_ERR_INVALID_ARG;
-    if (c->cap_num < 0 || c->cap_den < 0 || ((c->cap_num == 0) != (c->cap_den == 0))) return MOE_ERR_INVALID_ARG;
-    if (c->layout != MOE_LAYOUT_CONTIGUOUS && c->layout != MOE_LAYOUT_MASKED) return MOE_ERR_INVALID_ARG;
-    if (c->layout == MOE_LAYOUT_MASKED && (c->masked_max_m <= 0 || c->masked_max_m % 32)) return MOE_ERR_INVALID_ARG;
-    const int64_t rows = c->layout == MOE_LAYOUT_MASKED
-                             ? static_cast<int64_t>(c->E) * c->masked_max_m
-                             : static_cast<int64_t>(c->T) * c->k + static_cast<int64_t>(c->E) * (kGroup - 1);
-    if (rows >= (1ll << 31) / kGroup) return MOE_ERR_UNSUPPORTED_SHAPE;
-    return MOE_OK;
-}
-
-int64_t capacity_of(const moe_config_t* c) {
-    if (c->cap_num == 0) return -1;
-    const int64_t R = static_cast<int64_t>(c->T) * c->k;
-    return (R + c->E - 1) / c->E * c->cap_num / c->cap_den;
-}
-
-size_t rows_of(const moe_config_t* c) {
-    if (c->layout == MOE_LAYOUT_MASKED) return static_cast<size_t>(c->E) * c->masked_max_m;
-    const size_t r = static_cast<size_t>(c->T) * c->k + static_cast<size_t>(c->E) * (kGroup - 1);
-    return (r + kGroup - 1) / kGroup * kGroup;
-}
 
 size_t route_scratch(const moe_config_t* c) {
     return c->routing == MOE_ROUTE_SOFTMAX_TOPK ? align_up(sizeof(float) * static_cast<size_t>(c->T) * c->E) : 0;
@@ -358,7 +361,7 @@ const char* moe_status_string(moe_status_t s) {
         case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
         case MOE_ERR_UNSUPPORTED_DEVICE: return "FP8 not supported on this GPU (needs sm_100)";
         case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
-        case MOE_ERR_CAPACITY: return "a masked group had more rows than masked_max_m";
+        case MOE_ERR_CAPACITY: return "a group had more rows than its bound (masked_max_m or M_rows)";
         case MOE_ERR_CUDA: return "CUDA error";
         case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
     }

@@ -131,8 +131,30 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int NB = N / kBM;                 // 128-wide weight blocks along N
     const int NT = (N + kBN - 1) / kBN;
 
-    // group prefix in M tiles: P[e] = offsets[e] / 128
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) sm.P[e] = offsets[e] / kBM;
+    // group prefix in M tiles: P[e] = offsets[e] / 128. Offsets that are not non-decreasing multiples of
+    // 128 within [0, M_rows] (P[0] = 0) are forced into that shape by a running maximum of the clamped
+    // values and reported, so that no tile reads or writes past row M_rows
+    if (warp == 0) {
+        int carry = 0;
+        bool bad = false;
+        for (int b = 0; b <= E; b += 32) {
+            const int e = b + lane;
+            const int o = e <= E ? offsets[e] : 0;
+            int v = e == 0 ? 0 : min(max(o, 0), M_rows) / kBM;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, v, d);
+                if (lane >= d) v = max(v, u);
+            }
+            v = max(v, carry);
+            if (e <= E) {
+                sm.P[e] = v;
+                bad |= o != v * kBM;
+            }
+            carry = __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, kStatusCapacity);
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStagesC; ++s) {
             mbar_init(&sm.full[s], 1);
@@ -392,7 +414,6 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
             } else {
                 // SwiGLU on (a = acc[0..63], b = acc[64..127]) for h columns n0/2 + half*64 + [0, 64)
-                const int I = N / 2;
                 float amax = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 64; ++i) {
@@ -527,7 +548,11 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         if (lane == 0) sm.P[0] = 0;
         for (int b = 0; b < E; b += 32) {
             const int e = b + lane;
-            const int32_t m = e < E ? masked_m[e] : 0;
+            // a block holds at most Mmax rows: a count outside [0, Mmax] is clamped (and reported) so
+            // that no tile reads or writes past its expert's block
+            const int32_t m_in = e < E ? masked_m[e] : 0;
+            const int32_t m = min(max(m_in, 0), Mmax);
+            if (m != m_in) set_status(status, kStatusCapacity);
             if (e < E) sm.M[e] = m;
             int32_t v = NBt * ((m + kBT - 1) / kBT);
 #pragma unroll

@@ -29,6 +29,10 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, int T, in
                            int32_t* offsets, int32_t* row_src, int32_t* slot_row, void* scratch, int* status,
                            int num_sms, cudaStream_t s);
 int* device_status_word();   // api.cu: the status word of the current device, or nullptr
+// api.cu: the configuration rules, capacity and row count that moe_permute applies
+moe_status_t check_cfg(const moe_config_t* c);
+int64_t capacity_of(const moe_config_t* c);
+size_t rows_of(const moe_config_t* c);
 
 static __device__ __align__(256) int32_t g_noalloc_scratch[MOE_PERMUTE_NOALLOC_MAX_SCRATCH_BYTES / sizeof(int32_t)];
 
@@ -76,39 +80,30 @@ using namespace moe;
 extern "C" moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
                                             uint8_t* Aq, float* As, int32_t* counts, int32_t* kept,
                                             int32_t* offsets, int32_t* row_src, int32_t* slot_row, void* stream) {
-    // the same configuration rules as moe_permute
-    if (!cfg) return MOE_ERR_INVALID_ARG;
+    // the same configuration rules as moe_permute (one validator serves both entry points)
+    moe_status_t st = check_cfg(cfg);
+    if (st != MOE_OK) return st;
     const moe_config_t& c = *cfg;
-    if (c.T < 0 || c.H <= 0 || c.I <= 0 || c.E <= 0 || c.k <= 0) return MOE_ERR_INVALID_ARG;
-    if (c.H % kGroup || c.I % kGroup || c.H > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (c.E > MOE_MAX_EXPERTS || c.k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (c.k > c.E) return MOE_ERR_INVALID_ARG;
-    if (c.routing != MOE_ROUTE_SOFTMAX_TOPK && c.routing != MOE_ROUTE_HASH) return MOE_ERR_INVALID_ARG;
-    if (c.routing == MOE_ROUTE_HASH && c.k != 1) return MOE_ERR_INVALID_ARG;
-    if (c.cap_num < 0 || c.cap_den < 0 || ((c.cap_num == 0) != (c.cap_den == 0))) return MOE_ERR_INVALID_ARG;
-    if (c.layout != MOE_LAYOUT_CONTIGUOUS && c.layout != MOE_LAYOUT_MASKED) return MOE_ERR_INVALID_ARG;
-    if (c.layout == MOE_LAYOUT_MASKED && (c.masked_max_m <= 0 || c.masked_max_m % 32)) return MOE_ERR_INVALID_ARG;
     const bool masked = c.layout == MOE_LAYOUT_MASKED;
-    const int64_t rows_needed = masked ? static_cast<int64_t>(c.E) * c.masked_max_m
-                                       : static_cast<int64_t>(c.T) * c.k + static_cast<int64_t>(c.E) * (kGroup - 1);
-    if (rows_needed >= (1ll << 31) / kGroup) return MOE_ERR_UNSUPPORTED_SHAPE;
     // the fixed scratch must hold this call's per-chunk counts and bases
     if (permute_scratch_bytes(c.T, c.E) > MOE_PERMUTE_NOALLOC_MAX_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED_SHAPE;
     NoAllocDevice* dev;
-    moe_status_t st = noalloc_device(&dev);
-    if (st != MOE_OK) return st;
+    if ((st = noalloc_device(&dev)) != MOE_OK) return st;
+    // the status word receives MOE_ERR_CAPACITY from the kernels; without it an overflow would go
+    // unreported, so refuse to launch
+    int* status = device_status_word();
+    if (status == nullptr) return MOE_ERR_CUDA;
     if (!ptr16(x) || !ptr16(topk_idx) || !ptr16(Aq) || !ptr16(As) || !ptr16(counts) || !ptr16(kept) ||
         !ptr16(offsets) || !ptr16(row_src) || !ptr16(slot_row))
         return MOE_ERR_INVALID_ARG;
     if (c.T == 0) return MOE_OK;
-    const int64_t cap = c.cap_num == 0 ? -1
-                                       : (static_cast<int64_t>(c.T) * c.k + c.E - 1) / c.E * c.cap_num / c.cap_den;
-    const int rows = masked ? c.E * c.masked_max_m : static_cast<int>((rows_needed + kGroup - 1) / kGroup * kGroup);
+    const int64_t cap = capacity_of(cfg);
+    const int rows = static_cast<int>(rows_of(cfg));
     // Nothing in the scratch has to start at zero: the count kernel writes every
     // count it holds before the scan reads them, and the scan writes every base.
     const cudaError_t e = launch_permute(static_cast<const uint16_t*>(x), topk_idx, c.T, c.H, c.k, c.E, cap,
                                          masked ? c.masked_max_m : 0, rows, Aq, As, counts, kept, offsets, row_src,
-                                         slot_row, dev->scratch, device_status_word(), dev->num_sms,
+                                         slot_row, dev->scratch, status, dev->num_sms,
                                          static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

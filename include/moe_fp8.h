@@ -53,7 +53,7 @@ typedef enum {
     MOE_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100 ("FP8 not supported on this GPU",
                                        MegaMoE page, section 5.1, problem three) */
     MOE_ERR_WORKSPACE_TOO_SMALL = 4,
-    MOE_ERR_CAPACITY = 5,           /* device status: a masked group had more rows than masked_max_m */
+    MOE_ERR_CAPACITY = 5,           /* device status: a group had more rows than its bound (masked_max_m, M_rows) */
     MOE_ERR_CUDA = 6,               /* a CUDA runtime call or launch failed */
     MOE_ERR_DEVICE_TIMEOUT = 7      /* device status: a bounded wait inside a kernel ran out */
 } moe_status_t;
@@ -169,6 +169,13 @@ moe_status_t moe_permute(const moe_config_t* cfg, const void* x, const int32_t* 
  * a 16-byte boundary (MOE_ERR_INVALID_ARG otherwise).
  * Contiguous rows outside [0, offsets[E]) and masked rows at or past
  * masked_m[e] are neither read into any stored result nor written.
+ * Group bounds are checked on the device: offsets must start at 0, be
+ * non-decreasing multiples of 128 and stay within M_rows, and each masked_m[e]
+ * must lie in [0, M_rows]. Values outside these bounds are clamped into them
+ * (offsets by a running maximum of the clamped values), so that no read or
+ * write leaves the caller's buffers, and the device status MOE_ERR_CAPACITY is
+ * set (moe_get_device_status); the results of the offending groups are then
+ * unspecified.
  */
 moe_status_t moe_grouped_gemm_fp8(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                                   const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,

@@ -99,9 +99,41 @@ def gpu_forward(cfg: MoeConfig, inp: MoeInputs) -> dict:
     return out
 
 
-def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:
-    if n >= T:
-        return np.arange(T)
+def tile_covering_tokens(layout: str, slot_row: np.ndarray, k: int, seed: int = 0):
+    """Tokens whose kept rows touch every tile the grouped GEMMs schedule.
+
+    Contiguous layout: a tile is a 128-row M tile of the padded, expert-contiguous rows (every
+    group starts on a multiple of 128, so a tile belongs to one expert; its N tiles are all
+    covered by comparing whole rows). Masked layout: a tile is a 32-token slice of an expert's
+    block (the swap-AB kernel's N tile). `slot_row` is the oracle's own slot -> row map. Tiles
+    are visited in a seeded random order; for an uncovered tile one of its rows is picked,
+    preferring the 32-row quadrant i % 4 (i = the tile's visit index) so that every promotion
+    warp's lane quadrant is exercised, and among those the token that reaches the most uncovered
+    tiles; every tile the token reaches is then marked.
+    Returns (sorted tokens, number of tiles, number covered)."""
+    slot_row = np.asarray(slot_row, np.int64)
+    T = slot_row.size // k
+    span = 128 if layout == "contiguous" else 32
+    kept = np.nonzero(slot_row >= 0)[0]
+    rows = slot_row[kept]
+    tiles = rows // span
+    by_tile = {}
+    for r, s_, tl in zip(rows, kept, tiles):
+        by_tile.setdefault(int(tl), []).append((int(r), int(s_ // k)))
     rng = np.random.default_rng(seed)
-    pick = rng.choice(np.arange(1, T - 1), size=n - 2, replace=False)
-    return np.sort(np.concatenate([[0, T - 1], pick]))
+    order = rng.permutation(np.array(sorted(by_tile), dtype=np.int64))
+    per_token = slot_row.reshape(T, k)
+    covered, chosen = set(), []
+    for i, tl in enumerate(order):
+        tl = int(tl)
+        if tl in covered:
+            continue
+        cand = by_tile[tl]
+        quad = [c for c in cand if (c[0] % span) // 32 == i % 4] if span == 128 else []
+        pool = quad or cand
+        # of the candidates, the token whose kept rows reach the most tiles not yet covered
+        gain = [len({int(r) // span for r in per_token[c[1]] if r >= 0} - covered) for c in pool]
+        t = pool[int(np.argmax(gain))][1]
+        chosen.append(t)
+        covered.update(int(r) // span for r in per_token[t] if r >= 0)
+    return np.array(sorted(set(chosen)), dtype=np.int64), len(by_tile), len(covered & set(by_tile))

@@ -5,7 +5,8 @@ the bf16 output within max_rel 2e-2 / mean_rel 2e-3.
 
 Small cases run the oracle on every token; full-size workloads (in the launch
 configuration the benchmark times) run the oracle's routing and dispatch on
-every token and its expert math on a sample of tokens."""
+every token and its expert math on a set of tokens that reaches every tile the
+grouped GEMMs schedule."""
 import numpy as np
 import pytest
 import torch
@@ -14,7 +15,7 @@ import oracle
 from fp8_grouped_gemm_fp32_b200 import api
 from fp8_grouped_gemm_fp32_b200.inputs import CONFIGS, MoeConfig, interleave_w13
 from gpu_helpers import (W_RTOL, assert_close_bf16, ensure_lib, gpu_forward, gpu_inputs, oracle_inputs,
-                         sample_tokens, to_np)
+                         tile_covering_tokens, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -53,15 +54,31 @@ def test_layer_small(name):
     _check_layer(cfg, inp, ref, out, np.arange(cfg.T))
 
 
-@pytest.mark.parametrize("name,n_tokens", [("page", 12), ("prefill", 6), ("decode", 8), ("decode_hash", 24),
-                                           ("skewed", 12)])
-def test_layer_full_size_sampled(name, n_tokens):
+@pytest.mark.parametrize("name", ["page", "prefill", "decode", "decode_hash", "skewed"])
+def test_layer_full_size_tile_covering(name):
+    # Every workload at full size, in the launch configuration the benchmark times: routing, counts and the
+    # slot -> row map (permutation and dropped set) on every token, and y on a set of tokens whose kept rows
+    # reach every tile the two grouped GEMMs schedule (each 128-row M tile of the contiguous layout, each
+    # 32-token slice of an expert's block in the masked layout), chosen from the oracle's own dispatch.
     ensure_lib()
     cfg = CONFIGS[name]
     inp = gpu_inputs(cfg, on_device=True)
     out = gpu_forward(cfg, inp)
-    toks = sample_tokens(cfg.T, n_tokens, seed=cfg.seed)
-    ref = oracle.forward(cfg, oracle_inputs(inp), tokens=toks)
+    o_in = oracle_inputs(inp)
+    idx, _w, _l = oracle.route(cfg, o_in["x"], o_in["Wg"], o_in["bias"], o_in["token_ids"])
+    k = idx.shape[1]
+    c = api.Config.from_moe(cfg)
+    rows_cap = api.moe_rows_capacity(c)
+    cap = oracle.capacity(cfg.T, k, cfg.E, cfg.cap_num, cfg.cap_den)
+    d = oracle.dispatch(idx, cfg.E, cap, 1 if cfg.layout == "masked" else 0, 128, cfg.masked_max_m, rows_cap)
+    toks, n_tiles, n_cov = tile_covering_tokens(cfg.layout, d["slot_row"], k, seed=cfg.seed)
+    assert n_cov == n_tiles and n_tiles > 0                      # the coverage this test claims
+    if cfg.layout == "contiguous":
+        assert n_tiles == d["offsets"][-1] // 128               # = every M tile the kernels schedule
+    else:
+        assert n_tiles == int(np.sum(-(-d["kept"] // 32)))
+    ref = oracle.forward(cfg, o_in, tokens=toks)
+    assert np.array_equal(ref["slot_row"], d["slot_row"])
     _check_layer(cfg, inp, ref, out, toks)
     if cfg.cap_num:
         assert np.count_nonzero(ref["slot_row"] < 0) > 0        # the capacity really drops slots

@@ -260,7 +260,31 @@ GEMM_CASES = [
     (0, 0, 2, 16384, 128, [130, 1], None),
     (1, 0, 2, 256, 16384, [5, 32], 32),
     (1, 1, 2, 256, 16384, [32, 7], 32),
+    # far more tiles than the 148 persistent CTAs (contiguous: 28 M tiles x 16 N tiles = 448; masked: up to
+    # 16 experts x 16 weight tiles x up to 2 token tiles), so every CTA runs several tiles and the stage,
+    # scale and accumulator rings wrap across tile boundaries
+    (0, 0, 8, 4096, 256, [600, 517, 0, 640, 129, 380, 700, 255], None),
+    (0, 1, 8, 4096, 256, [600, 517, 0, 640, 129, 380, 700, 255], None),
+    (1, 0, 16, 2048, 256, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64),
+    (1, 1, 16, 4096, 256, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64),
 ]
+
+MANY_TILES = 296          # two tiles per persistent CTA on a 148-SM part
+
+
+def _tile_count(layout, epi, E, N, groups, M_rows):
+    if layout == 0:
+        return sum(-(-g // 128) for g in groups) * -(-N // 256)
+    return sum(-(-g // 32) for g in groups) * (N // 256 if epi == 1 else N // 128)
+
+
+def test_gemm_cases_include_multi_tile_launches():
+    # the coverage the cases above claim: both layouts and both epilogues have a launch with more tiles
+    # than two per CTA
+    for layout in (0, 1):
+        for epi in (0, 1):
+            assert any(c[0] == layout and c[1] == epi and _tile_count(layout, epi, c[2], c[3], c[5], c[6])
+                       > MANY_TILES for c in GEMM_CASES), (layout, epi)
 
 
 @pytest.mark.parametrize("case", GEMM_CASES)
@@ -294,7 +318,17 @@ W4_CASES = [
     (3, 384, 1024, [1, 31, 64], 64, 0, 3),
     (2, 256, 16384, [5, 32], 32, 0, 4),
     (2, 512, 16384, [32, 9], 32, 1, 5),
+    # more tiles than two per CTA in both epilogues (16 experts x 16 weight tiles x up to 2 token
+    # tiles): the converter warps' stage counter, their barrier phases and the per-tile reload of the row
+    # scales carry across tiles
+    (16, 2048, 1024, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64, 0, 6),
+    (16, 4096, 1024, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64, 1, 7),
 ]
+
+
+def test_w4_cases_include_multi_tile_launches():
+    for epi in (0, 1):
+        assert any(c[5] == epi and _tile_count(1, epi, c[0], c[1], c[3], c[4]) > MANY_TILES for c in W4_CASES)
 
 
 @pytest.mark.parametrize("case", W4_CASES)
@@ -372,6 +406,71 @@ def test_grouped_gemm_writes_nothing_outside_its_groups(layout, epi):
             for e in range(E):
                 assert np.all(Ds[e, :, gi[e]:] == -3.0)
                 assert np.all(Ds[e, :, :gi[e]] > 0)
+
+
+@pytest.mark.parametrize("layout,epi,w4", [(1, 0, False), (1, 1, False), (1, 0, True), (1, 1, True),
+                                           (0, 0, False), (0, 1, False)])
+def test_grouped_gemm_clamps_out_of_bound_groups(layout, epi, w4):
+    # group sizes past the buffers (a masked count above M_rows or below 0; contiguous offsets past M_rows
+    # or not a multiple of 128) are clamped on the device and reported as MOE_ERR_CAPACITY: guard rows past
+    # D and past the scales keep their canary, and the groups within bounds are still exact
+    ensure_lib()
+    E, N, K = 3, 512, 256
+    if layout == 1:
+        M = 32
+        gi = np.array([5, -4, 40], np.int32)                  # expert 2 claims 40 rows of a 32-row block
+        good = [0]
+        rows = E * M
+    else:
+        gi = np.array([0, 128, 128, 1024], np.int32)         # the last group runs past M_rows = 384
+        M = rows = 384
+        good = [0]
+    rng = np.random.default_rng(5)
+    A = _rand_codes(rng, (rows, K))
+    G = K // 128
+    As = rng.uniform(0.002, 0.02, (G, rows) if layout == 0 else (E, G, M)).astype(np.float32)
+    if w4:
+        from fp8_grouped_gemm_fp32_b200.inputs import quantize_weight_int4
+        q, s4 = quantize_weight_int4(torch.from_numpy(rng.standard_normal((E * N, K)).astype(np.float32) * 0.02))
+        B = q.numpy().reshape(E, N, K // 2)
+        Bs = np.ascontiguousarray(s4.numpy().reshape(E, N, K // 128).transpose(0, 2, 1))
+    else:
+        B = _rand_codes(rng, (E, N, K))
+        Bs = rng.uniform(1e-4, 1e-3, (E, N // 128, G)).astype(np.float32)
+    guard = 64
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    width = N if epi == 0 else N // 2
+    dt = torch.int16 if epi == 0 else torch.uint8
+    canary = 0x5A5A if epi == 0 else 0x5A
+    Dfull = torch.full((rows + guard, width), canary, dtype=dt, device="cuda")
+    Gs = N // 256
+    Dsfull = None
+    if epi == 1:
+        Dsfull = torch.full((Gs * M + guard,) if layout == 0 else (E * Gs * M + guard,), -3.0,
+                            dtype=torch.float32, device="cuda")
+    D = Dfull[:rows]
+    fn = api.moe_grouped_gemm_w4 if w4 else api.moe_grouped_gemm_fp8
+    fn(layout, E, N, K, d(A), d(As), d(gi), M, d(B), d(Bs), epi, D, Dsfull)
+    torch.cuda.synchronize()
+    assert api.moe_get_device_status() == api.MOE_ERR_CAPACITY
+    assert api.moe_get_device_status() == api.MOE_OK
+    Dh = to_np(Dfull)
+    assert np.all(Dh[rows:] == canary)                          # nothing past D
+    if epi == 1:
+        assert np.all(to_np(Dsfull)[-guard:] == -3.0)           # nothing past Ds
+    # a group within bounds is unaffected: expert 0's rows match the oracle
+    if layout == 1:
+        gi_ok = np.array([gi[0], 0, 0], np.int32)
+    else:
+        gi_ok = np.array([0, 128, 128, 128], np.int32)
+    Dr, _ = oracle.grouped_gemm(layout, E, N, K, A, As, gi_ok, M, B, Bs, epi, w4=w4)
+    r = np.arange(gi[0]) if layout == 1 else np.arange(128)
+    if epi == 0:
+        assert_close_bf16(Dh[r], Dr[r], "D")
+    else:
+        same = Dh[r] == Dr[r]
+        assert same.mean() > 0.99
+        assert np.all(np.abs(Dh[r].astype(np.int32) - Dr[r].astype(np.int32))[~same] == 1)
 
 
 def test_combine_with_drops():
