@@ -401,6 +401,8 @@ def run_ours(args):
         cfg = cfg.replace(E=args.experts)
     from fp8_grouped_gemm_fp32_b200 import api
     api.lib()                                      # fails loudly if the native library is missing
+    api.moe_set_contig_kernel({"auto": api.CONTIG_AUTO, "single": api.CONTIG_SINGLE,
+                               "pair": api.CONTIG_PAIR}[args.contig])
     layer = Layer(cfg, dev, seed_offset=rank)
     torch.cuda.synchronize()
     for _ in range(args.warmup):
@@ -515,6 +517,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8e4m3 (fp32 accumulate)", "data": "synthetic",
         "config": {"workload": describe(cfg), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "contig_gemm": args.contig,
                    "l2": "no flush: the FP8 weights streamed every step (%.2f GB) exceed the 126 MB L2"
                          % ((work["gemm_up"]["bytes"] + work["gemm_down"]["bytes"]) / 1e9)},
         "roofline": roof,
@@ -586,6 +589,8 @@ def main():
                     help="workload (default: prefill, the largest that fits one GPU)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--contig", default="auto", choices=["auto", "single", "pair"],
+                    help="form of the contiguous grouped GEMM (default: chosen by shape)")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the workload's expert count (reduced cases for profiling captures)")
     args = ap.parse_args()

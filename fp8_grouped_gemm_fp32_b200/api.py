@@ -28,9 +28,12 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_S
 ROUTE_SOFTMAX_TOPK, ROUTE_HASH = 0, 1
 LAYOUT_CONTIGUOUS, LAYOUT_MASKED = 0, 1
 EPI_BF16, EPI_SWIGLU_FP8 = 0, 1
+CONTIG_AUTO, CONTIG_SINGLE, CONTIG_PAIR = 0, 1, 2
 EXPORTS = ("moe_rows_capacity", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_gemm_fp8",
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string",
-           "moe_permute_noalloc", "moe_balance_bias", "moe_grouped_gemm_w4")
+           "moe_permute_noalloc", "moe_balance_bias", "moe_grouped_gemm_w4", "moe_set_contig_kernel",
+           "moe_ep_plan", "moe_ep_workspace_size", "moe_ep_count", "moe_ep_dispatch", "moe_ep_receive",
+           "moe_ep_return")
 
 
 class MoeError(RuntimeError):
@@ -77,10 +80,18 @@ def lib() -> ctypes.CDLL:
         L.moe_balance_bias.argtypes = [I, P, P, P, ctypes.c_float, I, P]
         L.moe_get_device_status.argtypes = [P]
         L.moe_selftest_wait_timeout.argtypes = [I, P]
+        L.moe_set_contig_kernel.argtypes = [I]
+        L.moe_ep_plan.argtypes = [I, I, I, ctypes.c_int64, I, I, I, P, P]
+        L.moe_ep_workspace_size.argtypes = [CP]
+        L.moe_ep_workspace_size.restype = SZ
+        L.moe_ep_count.argtypes = [CP, P, P, P, SZ, P]
+        L.moe_ep_dispatch.argtypes = [CP, P, P, P, P, P, P, SZ, P]
+        L.moe_ep_receive.argtypes = [I, P, I, P, P, P, I, P, P, P]
+        L.moe_ep_return.argtypes = [I, I, P, P, P, P]
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in EXPORTS:
-            if f not in ("moe_rows_capacity", "moe_workspace_size", "moe_status_string"):
+            if f not in ("moe_rows_capacity", "moe_workspace_size", "moe_status_string", "moe_ep_workspace_size"):
                 getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -176,3 +187,36 @@ def moe_get_device_status(stream=None) -> int:
 
 def moe_selftest_wait_timeout(limit_us: int, stream=None):
     _check(lib().moe_selftest_wait_timeout(limit_us, _stream(stream)), "moe_selftest_wait_timeout")
+
+
+def moe_set_contig_kernel(form: int):
+    """Form of the contiguous-layout grouped GEMM for later calls: CONTIG_AUTO, CONTIG_SINGLE or CONTIG_PAIR."""
+    _check(lib().moe_set_contig_kernel(int(form)), "moe_set_contig_kernel")
+
+
+# ---------------------------------------------------------------- expert parallelism (see ep.py)
+def _nbytes(t):
+    return t.numel() * t.element_size() if t is not None else 0
+
+
+def moe_ep_workspace_size(cfg: Config) -> int:
+    return int(lib().moe_ep_workspace_size(ctypes.byref(cfg)))
+
+
+def moe_ep_count(cfg, topk_idx, counts, ws, stream=None):
+    _check(lib().moe_ep_count(ctypes.byref(cfg), _p(topk_idx), _p(counts), _p(ws), _nbytes(ws), _stream(stream)),
+           "moe_ep_count")
+
+
+def moe_ep_dispatch(cfg, x, topk_idx, plan_dev, send, slot_row, ws, stream=None):
+    _check(lib().moe_ep_dispatch(ctypes.byref(cfg), _p(x), _p(topk_idx), _p(plan_dev), _p(send), _p(slot_row), _p(ws),
+                                 _nbytes(ws), _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_receive(H, plan_dev, rows_recv, recv, Aq, As, M_rows, offsets, group_row, stream=None):
+    _check(lib().moe_ep_receive(H, _p(plan_dev), rows_recv, _p(recv) if rows_recv else None, _p(Aq), _p(As), M_rows,
+                                _p(offsets), _p(group_row), _stream(stream)), "moe_ep_receive")
+
+
+def moe_ep_return(H, rows_recv, O, group_row, ret, stream=None):
+    _check(lib().moe_ep_return(H, rows_recv, _p(O), _p(group_row), _p(ret), _stream(stream)), "moe_ep_return")

@@ -31,6 +31,7 @@ cudaError_t launch_grouped_gemm_w4(int E, int N, int K, const uint8_t* A, const 
 cudaError_t launch_combine(const uint16_t* O, const int32_t* slot_row, const float* topk_w, int T, int k, int H,
                            uint16_t* y, cudaStream_t s);
 cudaError_t launch_selftest_wait(int* status, uint64_t wait_ns, cudaStream_t s);
+void set_contig_mode(int mode);
 cudaError_t launch_balance_bias(int E, const int32_t* counts, int64_t* load, float* bias, float gamma, int update,
                                 cudaStream_t s);
 
@@ -160,6 +161,16 @@ inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 int* device_status_word() {
     DeviceInfo* dev;
     return device_info(&dev) == MOE_OK ? dev->status : nullptr;
+}
+
+// The current device's SM count and status word, for entry points defined in other files.
+moe_status_t current_device(int* num_sms, int** status) {
+    DeviceInfo* dev;
+    const moe_status_t st = device_info(&dev);
+    if (st != MOE_OK) return st;
+    *num_sms = dev->num_sms;
+    *status = dev->status;
+    return MOE_OK;
 }
 
 }  // namespace moe
@@ -331,6 +342,12 @@ moe_status_t moe_balance_bias(int E, const int32_t* counts, int64_t* load, float
     DeviceInfo* dev;
     if ((st = device_info(&dev)) != MOE_OK) return st;
     return cuda_status(launch_balance_bias(E, counts, load, bias, gamma, update != 0, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_set_contig_kernel(int form) {
+    if (form != MOE_CONTIG_AUTO && form != MOE_CONTIG_SINGLE && form != MOE_CONTIG_PAIR) return MOE_ERR_INVALID_ARG;
+    set_contig_mode(form);
+    return MOE_OK;
 }
 
 moe_status_t moe_get_device_status(void* stream) {

@@ -60,11 +60,14 @@ constexpr int kOutBox = 32;
 constexpr int kOutBoxBytes = kOutBox * kOutBox * 2;            // 2 KB
 constexpr int kOutStageBytes = 8 * 4 * kOutBoxBytes;           // 64 KB
 
-template <int EPI>
+// PAIR: the two CTAs of a cluster compute one 256-row x 256-column tile with pair MMAs; each holds its
+// 128 A rows and its 128-row half of the B tile, so a stage is 32 KB instead of 48 KB.
+template <int EPI, bool PAIR = false>
 struct SmemC {
-    static constexpr int kStages = EPI == 0 ? 3 : 4;
+    static constexpr int kBStage = PAIR ? kBBytes / 2 : kBBytes;
+    static constexpr int kStages = PAIR ? (EPI == 0 ? 4 : 6) : (EPI == 0 ? 3 : 4);
     uint8_t a[kStages][kABytes];
-    uint8_t b[kStages][kBBytes];
+    uint8_t b[kStages][kBStage];
     uint8_t out[EPI == 0 ? kOutStageBytes : 8 * kOutBoxBytes];
     float sa[kSaSlots][kBM];    // activation scales of one K block for the tile's 128 rows
     float wsc[2][2][kMaxKB];    // weight-block scales of a tile (two tiles in flight): [tile & 1][block][kb]
@@ -81,6 +84,7 @@ struct SmemC {
     uint32_t tmem_base;
     volatile int abort_flag;
     int32_t P[kMaxE + 1];
+    int32_t Q[PAIR ? kMaxE + 1 : 1];     // PAIR: prefix of the pair tiles per expert, ceil(M tiles / 2)
 };
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
@@ -99,6 +103,7 @@ __device__ __forceinline__ int find_group(const int32_t* P, int E, int q) {
 
 struct TileC {
     int e, m0, n0, width;
+    bool store;      // false for the idle half of a lone pair tile: computed, not written
 };
 
 __device__ __forceinline__ TileC decode_tile_c(const int32_t* P, int E, int NT, int N, int tile) {
@@ -111,25 +116,52 @@ __device__ __forceinline__ TileC decode_tile_c(const int32_t* P, int E, int NT, 
     t.m0 = (P[t.e] + local % mt_e) * kBM;
     t.n0 = nt * kBN;
     t.width = min(kBN, N - t.n0);
+    t.store = true;
+    return t;
+}
+
+// Pair tiles: an expert's M tiles are taken two at a time (the leader the first, the other CTA the second);
+// with an odd count the last pair is lone: both CTAs load the leader's rows and only the leader stores.
+// Order: expert -> N tile -> pair, so the pairs running at the same time share a weight tile through L2.
+__device__ __forceinline__ TileC decode_tile_pair(const int32_t* P, const int32_t* Q, int E, int NT, int tile,
+                                                  uint32_t rank) {
+    TileC t;
+    const int q = tile / NT;
+    t.e = find_group(Q, E, q);
+    const int mt_e = P[t.e + 1] - P[t.e];
+    const int pr_e = Q[t.e + 1] - Q[t.e];
+    const int local = tile - NT * Q[t.e];
+    const int nt = local / pr_e;
+    const int pp = local % pr_e;
+    const bool lone = 2 * pp + 1 == mt_e;
+    t.m0 = (P[t.e] + 2 * pp + (lone ? 0 : static_cast<int>(rank))) * kBM;
+    t.n0 = nt * kBN;
+    t.width = kBN;
+    t.store = !(lone && rank == 1);
     return t;
 }
 
 __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
-template <int EPI>
+template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(kThreadsC, 1)
 gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmD, const float* __restrict__ As, const int32_t* __restrict__ offsets, int M_rows,
                  const float* __restrict__ Bs, int E, int N, int K, void* __restrict__ D, float* __restrict__ Ds,
                  int* status, uint64_t wait_ns) {
     extern __shared__ uint8_t smem_raw[];
-    using SC = SmemC<EPI>;
+    using SC = SmemC<EPI, PAIR>;
     constexpr int kStagesC = SC::kStages;
     SC& sm = *reinterpret_cast<SC*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = K / kBK;
     const int NB = N / kBM;                 // 128-wide weight blocks along N
     const int NT = (N + kBN - 1) / kBN;
+    // PAIR: this CTA's rank in its cluster of two (0 = leader, which issues the MMAs), the cluster's index
+    // and count (the persistent tile loop runs over clusters); otherwise each CTA works alone
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0;
+    const int tile0 = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+    const int tstep = PAIR ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
 
     // group prefix in M tiles: P[e] = offsets[e] / 128. Offsets that are not non-decreasing multiples of
     // 128 within [0, M_rows] (P[0] = 0) are forced into that shape by a running maximum of the clamped
@@ -154,6 +186,23 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             carry = __shfl_sync(0xffffffffu, v, 31);
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, kStatusCapacity);
+        if constexpr (PAIR) {
+            // pair tiles per expert: Q[e + 1] - Q[e] = ceil((P[e + 1] - P[e]) / 2)
+            __syncwarp();
+            int qc = 0;
+            if (lane == 0) sm.Q[0] = 0;
+            for (int b = 0; b < E; b += 32) {
+                const int e = b + lane;
+                int v = e < E ? (sm.P[e + 1] - sm.P[e] + 1) >> 1 : 0;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, v, d);
+                    if (lane >= d) v += u;
+                }
+                if (e < E) sm.Q[e + 1] = qc + v;
+                qc += __shfl_sync(0xffffffffu, v, 31);
+            }
+        }
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStagesC; ++s) {
@@ -166,7 +215,8 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.tfull[b], 1);
-            mbar_init(&sm.tempty[b], 8);
+            // PAIR: the leader's accumulator buffer is free when both CTAs' promotion warps have read it
+            mbar_init(&sm.tempty[b], PAIR ? 16 : 8);
             mbar_init(&sm.red_bar[b], 256);
             mbar_init(&sm.wfull[b], 1);
             mbar_init(&sm.wempty[b], 8);
@@ -175,19 +225,30 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, 512);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(&sm.tmem_base, 512);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&sm.tmem_base, 512);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (PAIR) cluster_sync(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int MT = sm.P[E];
-    const int total = MT * NT;
+    const int total = (PAIR ? sm.Q[E] : sm.P[E]) * NT;
+    auto decode = [&](int tile) -> TileC {
+        if constexpr (PAIR) return decode_tile_pair(sm.P, sm.Q, E, NT, tile, rank);
+        else return decode_tile_c(sm.P, E, NT, N, tile);
+    };
 
+    // A wait that runs out stops this CTA and (PAIR) its partner, whose waits on this CTA would otherwise
+    // only end at their own limits.
     auto fail = [&]() {
         set_status(status, kStatusTimeout);
         sm.abort_flag = 1;
+        if constexpr (PAIR) st_shared_cluster_u32(mapa_shared(smem_u32((const void*)&sm.abort_flag), rank ^ 1u), 1u);
     };
 
     // Register split (launch: 384 threads x 168 = 64512): the TMA/MMA warpgroup gives up
@@ -232,33 +293,45 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             return true;
         };
         uint32_t it = 0, ti = 0;
-        TileC t = decode_tile_c(sm.P, E, NT, N, blockIdx.x);
-        if (blockIdx.x < total) {
+        TileC t{};
+        t.e = -1;                                    // no tile (a CTA past the last tile decodes nothing)
+        if (tile0 < total) {
+            t = decode(tile0);
             read_scales(t);
             if (!publish_scales(0)) {
                 if (lane == 0 && !sm.abort_flag) fail();
                 t.e = -1;
             }
         }
-        for (int tile = blockIdx.x; tile < total && t.e >= 0; tile += gridDim.x, ++ti) {
-            const int nxt = tile + gridDim.x;
+        for (int tile = tile0; tile < total && t.e >= 0; tile += tstep, ++ti) {
+            const int nxt = tile + tstep;
             TileC tn = t;
             if (nxt < total) {
-                tn = decode_tile_c(sm.P, E, NT, N, nxt);
+                tn = decode(nxt);
                 read_scales(tn);
             }
             int ok = 1;
             if (lane == 0) {
-                const uint32_t bytes = kABytes + (t.width == kBN ? kBBytes : kBBytes / 2);
+                // PAIR: both CTAs' loads count on the leader's full barrier, which the leader arms with the
+                // bytes of both (its MMA reads both CTAs' stages); each CTA loads its A rows and its half of B
+                const uint32_t bytes = PAIR ? 2u * (kABytes + SC::kBStage)
+                                            : kABytes + (t.width == kBN ? kBBytes : kBBytes / 2);
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % kStagesC;
                     const uint32_t ph = (it / kStagesC) & 1;
                     if (!mbar_wait(&sm.empty[s], ph ^ 1, wait_ns)) { fail(); ok = 0; break; }
-                    mbar_arrive_expect_tx(&sm.full[s], bytes);
-                    tma_load_2d(sm.a[s], &tmA, &sm.full[s], kb * kBK, t.m0);
-                    tma_load_2d(sm.b[s], &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0);
-                    if (t.width == kBN)
-                        tma_load_2d(sm.b[s] + kBBytes / 2, &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0 + 128);
+                    if constexpr (PAIR) {
+                        const uint32_t fb = mapa_shared(smem_u32(&sm.full[s]), 0);
+                        if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], bytes);
+                        tma_load_2d_pair(sm.a[s], &tmA, fb, kb * kBK, t.m0);
+                        tma_load_2d_pair(sm.b[s], &tmB, fb, kb * kBK, t.e * N + t.n0 + static_cast<int>(rank) * 128);
+                    } else {
+                        mbar_arrive_expect_tx(&sm.full[s], bytes);
+                        tma_load_2d(sm.a[s], &tmA, &sm.full[s], kb * kBK, t.m0);
+                        tma_load_2d(sm.b[s], &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0);
+                        if (t.width == kBN)
+                            tma_load_2d(sm.b[s] + kBBytes / 2, &tmB, &sm.full[s], kb * kBK, t.e * N + t.n0 + 128);
+                    }
                     // the 128 activation scales of this K block, into the scale ring
                     const int j = it % kSaSlots;
                     if (!mbar_wait(&sm.sempty[j], ((it / kSaSlots) & 1) ^ 1, wait_ns)) { fail(); ok = 0; break; }
@@ -275,12 +348,12 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             t = tn;
         }
       } else if (warp == 1) {
-        // ---------------- MMA issuer
-        if (lane == 0) {
+        // ---------------- MMA issuer (PAIR: the leader only, for both CTAs)
+        if (lane == 0 && rank == 0) {
             uint32_t it = 0, kbt = 0;
-            for (int tile = blockIdx.x; tile < total && !sm.abort_flag; tile += gridDim.x) {
-                const TileC t = decode_tile_c(sm.P, E, NT, N, tile);
-                const uint32_t idesc = f8_idesc(kBM, t.width);
+            for (int tile = tile0; tile < total && !sm.abort_flag; tile += tstep) {
+                const TileC t = decode(tile);
+                const uint32_t idesc = PAIR ? f8_idesc(2 * kBM, kBN) : f8_idesc(kBM, t.width);
                 for (int kb = 0; kb < KB; ++kb, ++it, ++kbt) {
                     const int s = it % kStagesC;
                     const uint32_t ph = (it / kStagesC) & 1;
@@ -291,11 +364,21 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
                     const uint32_t d = tmem + buf * kBN;
+                    if constexpr (PAIR) {
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 32; ++kk)
-                        umma_f8(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc, kk > 0);
-                    umma_commit(&sm.empty[s]);
-                    umma_commit(&sm.tfull[buf]);
+                        for (int kk = 0; kk < kBK / 32; ++kk)
+                            umma_f8_pair(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc,
+                                         kk > 0);
+                        umma_commit_pair(&sm.empty[s], 0x3);     // both CTAs' stage s is free again
+                        umma_commit_pair(&sm.tfull[buf], 0x3);   // both CTAs' accumulator buffer is ready
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 32; ++kk)
+                            umma_f8(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc,
+                                    kk > 0);
+                        umma_commit(&sm.empty[s]);
+                        umma_commit(&sm.tfull[buf]);
+                    }
                 }
             }
         }
@@ -308,9 +391,11 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int row = q * 32 + lane;          // row within the tile
         uint32_t kbt = 0, ep = 0;
         uint32_t ti = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++ti) {
+        // PAIR: the accumulator buffer is released on the leader's barrier, which counts both CTAs' warps
+        const uint32_t tempty_leader0 = PAIR ? mapa_shared(smem_u32(&sm.tempty[0]), 0) : 0u;
+        for (int tile = tile0; tile < total; tile += tstep, ++ti) {
             if (sm.abort_flag) break;
-            const TileC t = decode_tile_c(sm.P, E, NT, N, tile);
+            const TileC t = decode(tile);
             const bool full = t.width == kBN;
             // the tile's weight-block scales, staged by the producer warp
             const int ws = ti & 1;
@@ -343,7 +428,12 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 auto release = [&]() {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+                    if (lane == 0) {
+                        if (PAIR && rank != 0)
+                            mbar_arrive_cluster(tempty_leader0 + buf * static_cast<uint32_t>(sizeof(uint64_t)));
+                        else
+                            mbar_arrive(&sm.tempty[buf]);
+                    }
                 };
                 auto fold = [&](float2* dst, const float (&v)[32], float f) {
                     const float2 ff = make_float2(f, f);
@@ -373,7 +463,16 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.wempty[ws]);          // the tile's weight scales are no longer read
             const int64_t grow = t.m0 + row;
-            if constexpr (EPI == 0) {
+            if (!t.store) {
+                // the idle half of a lone pair tile: its rows belong to the leader, which stores them; the
+                // SwiGLU epilogue's barrier phase still advances so both halves stay in step
+                if constexpr (EPI == 1) {
+                    const int p = ep & 1;
+                    mbar_arrive(&sm.red_bar[p]);
+                    if (!mbar_wait(&sm.red_bar[p], (ep >> 1) & 1, wait_ns)) { fail(); break; }
+                    ++ep;
+                }
+            } else if constexpr (EPI == 0) {
                 // this warp's 32 rows x 128 columns as four 32 x 32 boxes: box (r, c) holds columns
                 // n0 + r * 128 + half * 64 + c * 32 + [0, 32); 16-byte pieces are placed with the
                 // 64-byte swizzle (piece p of row l at p ^ ((l >> 1) & 3)), which the store undoes
@@ -458,15 +557,20 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
 
     if (warp >= 4 && lane == 0) bulk_wait_all();   // the output stores have completed
-    __syncthreads();
+    tc_fence_before();
+    // PAIR: neither CTA leaves while the leader's MMAs may still read the other's shared memory or write its
+    // tensor memory; after this barrier both abort flags are final
+    if constexpr (PAIR) cluster_sync(); else __syncthreads();
     if (sm.abort_flag) {
         // let TMA copies and MMAs that were already issued land before the memory is released
         const uint64_t t0 = globaltimer_ns();
         while (globaltimer_ns() - t0 < kDrainNs) __nanosleep(1000);
     }
+    if constexpr (PAIR) cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem, 512);
+        else tmem_dealloc(tmem, 512);
     }
 }
 
@@ -889,6 +993,67 @@ static cudaError_t check_reg_split(Kern k) {
     return a.numRegs * kThreadsC >= kRegsSplit ? cudaSuccess : cudaErrorInvalidConfiguration;
 }
 
+// Contiguous kernel in one of its two forms: one CTA per tile, or (PAIR) clusters of two CTAs sharing
+// 256 x 256 tiles, as many clusters as fit on the device at once (queried once per device).
+template <int EPI, bool PAIR>
+static cudaError_t launch_contig(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapD,
+                                 const float* As, const int32_t* offsets, int M_rows, const float* Bs, int E, int N,
+                                 int K, void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms,
+                                 cudaStream_t s) {
+    auto kern = gg_contig_kernel<EPI, PAIR>;
+    const size_t smem = sizeof(SmemC<EPI, PAIR>) + 1024;
+    cudaError_t err = set_smem(kern, smem);
+    if (err == cudaSuccess) err = check_reg_split(kern);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(kThreadsC);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    if constexpr (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        static int clusters[64] = {0};
+        int dev = 0;
+        if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        if (clusters[dev] == 0) {
+            cfg.gridDim = dim3(2 * (num_sms / 2));
+            int n = 0;
+            if ((err = cudaOccupancyMaxActiveClusters(&n, kern, &cfg)) != cudaSuccess) return err;
+            if (n <= 0) return cudaErrorInvalidConfiguration;
+            clusters[dev] = n;
+        }
+        cfg.gridDim = dim3(2 * clusters[dev]);
+    } else {
+        cfg.gridDim = dim3(num_sms);
+        cfg.attrs = nullptr;
+        cfg.numAttrs = 0;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, mapA, mapB, mapD, As, offsets, M_rows, Bs, E, N, K, D, Ds, status, wait_ns);
+}
+
+// Which form of the contiguous kernel runs (moe_set_contig_kernel): 0 chooses by shape, 1 forces single
+// CTAs, 2 forces CTA pairs (where N allows them).
+static int g_contig_mode = 0;
+
+void set_contig_mode(int mode) { __atomic_store_n(&g_contig_mode, mode, __ATOMIC_RELAXED); }
+
+// CTA pairs need whole 256-column tiles. They pay off when most experts fill several 128-row tiles: a
+// group with an odd tile count leaves half of its last pair idle, so the rows the buffer holds per expert
+// (capacity, padding included) must average at least two and a half tiles.
+static bool use_pairs(int E, int N, int M_rows) {
+    if (N % kBN) return false;
+    const int mode = __atomic_load_n(&g_contig_mode, __ATOMIC_RELAXED);
+    if (mode == 1) return false;
+    if (mode == 2) return true;
+    return static_cast<int64_t>(M_rows) * 2 >= static_cast<int64_t>(5) * kBM * E;
+}
+
 cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                                 const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs, int epilogue,
                                 void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s) {
@@ -896,23 +1061,19 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
     if (layout == 0) {
         if (!make_map(&mapA, A, K, static_cast<uint64_t>(M_rows), kBM)) return cudaErrorInvalidValue;
         if (!make_map(&mapB, B, K, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
+        const bool pair = use_pairs(E, N, M_rows);
         if (epilogue == 0) {
             if (!make_out_map(&mapD, D, N, static_cast<uint64_t>(M_rows), 2)) return cudaErrorInvalidValue;
-            const size_t smem = sizeof(SmemC<0>) + 1024;
-            cudaError_t err = set_smem(gg_contig_kernel<0>, smem);
-            if (err == cudaSuccess) err = check_reg_split(gg_contig_kernel<0>);
-            if (err != cudaSuccess) return err;
-            gg_contig_kernel<0><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K,
-                                                                  D, Ds, status, wait_ns);
-        } else {
-            if (!make_out_map(&mapD, D, N / 2, static_cast<uint64_t>(M_rows), 1)) return cudaErrorInvalidValue;
-            const size_t smem = sizeof(SmemC<1>) + 1024;
-            cudaError_t err = set_smem(gg_contig_kernel<1>, smem);
-            if (err == cudaSuccess) err = check_reg_split(gg_contig_kernel<1>);
-            if (err != cudaSuccess) return err;
-            gg_contig_kernel<1><<<num_sms, kThreadsC, smem, s>>>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K,
-                                                                  D, Ds, status, wait_ns);
+            return pair ? launch_contig<0, true>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K, D, Ds, status,
+                                                 wait_ns, num_sms, s)
+                        : launch_contig<0, false>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K, D, Ds, status,
+                                                  wait_ns, num_sms, s);
         }
+        if (!make_out_map(&mapD, D, N / 2, static_cast<uint64_t>(M_rows), 1)) return cudaErrorInvalidValue;
+        return pair ? launch_contig<1, true>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K, D, Ds, status,
+                                             wait_ns, num_sms, s)
+                    : launch_contig<1, false>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K, D, Ds, status,
+                                              wait_ns, num_sms, s);
     } else {
         if (!make_map(&mapA, A, K, static_cast<uint64_t>(E) * M_rows, kBT)) return cudaErrorInvalidValue;
         if (!make_map(&mapB, B, K, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;

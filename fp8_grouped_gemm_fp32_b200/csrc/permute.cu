@@ -88,16 +88,17 @@ __global__ void __launch_bounds__(256) permute_scan_kernel(const int32_t* __rest
     }
 }
 
-// Block-wide exclusive scan of per-expert row counts into off_s[0..E].
-__device__ void group_offsets(const int32_t* __restrict__ kept, int E, int masked_max_m, int32_t* off_s,
+// Block-wide exclusive scan of per-expert row counts, each rounded up to a multiple of `pad` (the tile
+// M, or 1 for unpadded send rows), into off_s[0..E].
+__device__ void group_offsets(const int32_t* __restrict__ kept, int E, int masked_max_m, int pad, int32_t* off_s,
                               int32_t* kept_s) {
     __shared__ int32_t wsum[8];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // each thread owns experts 2*tid, 2*tid+1 (E <= 512)
     int32_t a = 0, b = 0;
     const int e0 = 2 * tid, e1 = 2 * tid + 1;
-    if (e0 < E) { kept_s[e0] = kept[e0]; a = (kept_s[e0] + kGroup - 1) / kGroup * kGroup; }
-    if (e1 < E) { kept_s[e1] = kept[e1]; b = (kept_s[e1] + kGroup - 1) / kGroup * kGroup; }
+    if (e0 < E) { kept_s[e0] = kept[e0]; a = (kept_s[e0] + pad - 1) / pad * pad; }
+    if (e1 < E) { kept_s[e1] = kept[e1]; b = (kept_s[e1] + pad - 1) / pad * pad; }
     const int32_t local = a + b;
     int32_t incl = local;
 #pragma unroll
@@ -190,9 +191,9 @@ __device__ __forceinline__ GroupCodes quantise_group(uint4 raw, float amax) {
 // blockIdx.x >= nchunks (contiguous layout only): the padding rows of one expert, one slice of
 // pad_slices of its 128-groups (codes 0, scale 1, row_src -1). Block 0 also writes offsets.
 __global__ void __launch_bounds__(256) permute_map_kernel(
-    const int32_t* __restrict__ topk_idx, int T, int H, int k, int E, int nchunks, int pad_slices, int masked_max_m,
-    int ld_rows, const int32_t* __restrict__ base, const int32_t* __restrict__ kept, uint8_t* __restrict__ Aq,
-    float* __restrict__ As, int32_t* __restrict__ offsets, int32_t* __restrict__ row_src,
+    const int32_t* __restrict__ topk_idx, int T, int H, int k, int E, int nchunks, int pad, int pad_slices,
+    int masked_max_m, int ld_rows, const int32_t* __restrict__ base, const int32_t* __restrict__ kept,
+    uint8_t* __restrict__ Aq, float* __restrict__ As, int32_t* __restrict__ offsets, int32_t* __restrict__ row_src,
     int32_t* __restrict__ slot_row) {
     extern __shared__ int32_t sm[];
     int32_t* off_s = sm;                    // [E + 1]
@@ -201,8 +202,8 @@ __global__ void __launch_bounds__(256) permute_map_kernel(
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = H / kGroup;
 
-    group_offsets(kept, E, masked_max_m, off_s, kept_s);
-    if (blockIdx.x == 0)
+    group_offsets(kept, E, masked_max_m, pad, off_s, kept_s);
+    if (blockIdx.x == 0 && offsets)
         for (int e = tid; e <= E; e += blockDim.x) offsets[e] = off_s[e];
 
     if (blockIdx.x >= nchunks) {            // padding rows of one expert (contiguous layout)
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(256) permute_map_kernel(
             }
             const int64_t s = static_cast<int64_t>(t_lane) * k + j;
             slot_row[s] = row;
-            if (row >= 0) row_src[row] = static_cast<int32_t>(s);
+            if (row >= 0 && row_src) row_src[row] = static_cast<int32_t>(s);
         }
     }
 }
@@ -255,9 +256,12 @@ __global__ void __launch_bounds__(256) permute_map_kernel(
 // destination row of the token (slot_row). A warp takes one token and up to 8 of its groups, a
 // half-warp per group with 8 values (one 16-byte load) per lane, all four loads of a lane in flight
 // together; warps stride over (token, 8-group slice) items.
+// Scales go to As in the grouped layouts ([G][ld_rows], or [E][G][masked_max_m] when masked), or, with
+// `trailer`, right after the row's codes (row stride row_bytes = H + 4 G: the send rows of expert
+// parallelism, one contiguous record per row).
 __global__ void __launch_bounds__(256, 4) permute_quant_kernel(
-    const uint16_t* __restrict__ x, int T, int H, int k, int masked_max_m, int ld_rows,
-    const int32_t* __restrict__ slot_row, uint8_t* __restrict__ Aq, float* __restrict__ As) {
+    const uint16_t* __restrict__ x, int T, int H, int k, int masked_max_m, int ld_rows, int64_t row_bytes,
+    bool trailer, const int32_t* __restrict__ slot_row, uint8_t* __restrict__ Aq, float* __restrict__ As) {
     constexpr int U = 4;
     const int lane = threadIdx.x & 31, hl = lane & 15, hw = lane >> 4;
     const int G = H / kGroup;
@@ -313,9 +317,11 @@ __global__ void __launch_bounds__(256, 4) permute_quant_kernel(
             for (int u = 0; u < U; ++u) {
                 const int g = g0 + 2 * u + hw;
                 if (g >= G) continue;
-                *reinterpret_cast<uint2*>(Aq + static_cast<int64_t>(row) * H + g * kGroup + hl * 8) = code[u];
+                *reinterpret_cast<uint2*>(Aq + static_cast<int64_t>(row) * row_bytes + g * kGroup + hl * 8) = code[u];
                 if (hl == 0) {
-                    if (masked) {
+                    if (trailer) {
+                        reinterpret_cast<float*>(Aq + static_cast<int64_t>(row) * row_bytes + H)[g] = sc[u];
+                    } else if (masked) {
                         const int e = row / masked_max_m, rr = row - e * masked_max_m;
                         As[(static_cast<int64_t>(e) * G + g) * masked_max_m + rr] = sc[u];
                     } else {
@@ -346,8 +352,8 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, int T, in
     const int pad_slices = masked_max_m > 0 ? 1 : (G + 3) / 4;
     const int gx = nchunks + (masked_max_m > 0 ? 0 : E * pad_slices);
     const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1);
-    permute_map_kernel<<<gx, 256, smem, s>>>(topk_idx, T, H, k, E, nchunks, pad_slices, masked_max_m, ld_rows, base,
-                                             kept, Aq, As, offsets, row_src, slot_row);
+    permute_map_kernel<<<gx, 256, smem, s>>>(topk_idx, T, H, k, E, nchunks, kGroup, pad_slices, masked_max_m, ld_rows,
+                                             base, kept, Aq, As, offsets, row_src, slot_row);
     // one warp per (token, 8-group slice); enough blocks to keep every SM full, striding beyond that
     const int64_t warps = static_cast<int64_t>(T) * ((G + 7) / 8);
     int per_sm = 0;
@@ -357,7 +363,51 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, int T, in
     const int64_t cap_blocks = static_cast<int64_t>(per_sm) * num_sms * 4;
     const int blocks = static_cast<int>(std::min<int64_t>((warps + 7) / 8, cap_blocks));
     if (blocks > 0)
-        permute_quant_kernel<<<blocks, 256, 0, s>>>(x, T, H, k, masked_max_m, ld_rows, slot_row, Aq, As);
+        permute_quant_kernel<<<blocks, 256, 0, s>>>(x, T, H, k, masked_max_m, ld_rows, H, false, slot_row, Aq, As);
+    return cudaGetLastError();
+}
+
+int64_t ep_row_bytes(int H);
+
+// Expert parallelism, first half (before the counts are exchanged): per-chunk masks and the per-expert
+// exclusive scan over chunks, as for moe_permute; counts [E] out, ranks kept in `scratch`.
+cudaError_t launch_ep_count(const int32_t* topk_idx, int T, int k, int E, int32_t* counts, void* scratch,
+                            int* status, cudaStream_t s) {
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    int32_t* cnt = static_cast<int32_t*>(scratch);
+    int32_t* base = cnt + static_cast<size_t>(nchunks) * E;
+    int32_t* unused_kept = base + static_cast<size_t>(nchunks) * E;   // no capacity here: kept = counts
+    permute_count_kernel<<<(nchunks + 7) / 8, 256, 8 * E * sizeof(uint32_t), s>>>(topk_idx, T, k, E, nchunks, cnt);
+    permute_scan_kernel<<<E, 256, 0, s>>>(cnt, nchunks, -1, 0, base, counts, unused_kept, status);
+    return cudaGetLastError();
+}
+
+size_t ep_scratch_bytes(int T, int E) { return permute_scratch_bytes(T, E) + sizeof(int32_t) * static_cast<size_t>(E); }
+
+// Bytes of one send / receive row: H codes, H/128 fp32 scales, padded to 16 bytes.
+int64_t ep_row_bytes(int H) { return (static_cast<int64_t>(H) + 4 * (H / kGroup) + 15) / 16 * 16; }
+
+// Second half: send rows for the kept slots. kept_mine [E] (device, from the plan) bounds each expert's
+// ranks exactly as the capacity does in moe_permute; rows are unpadded (pad 1), in expert order, which
+// is destination-rank order since each rank's experts are contiguous.
+cudaError_t launch_ep_dispatch(const uint16_t* x, const int32_t* topk_idx, int T, int H, int k, int E,
+                               const int32_t* kept_mine, uint8_t* send, int32_t* slot_row, void* scratch,
+                               int num_sms, cudaStream_t s) {
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    int32_t* base = static_cast<int32_t*>(scratch) + static_cast<size_t>(nchunks) * E;
+    const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1);
+    permute_map_kernel<<<nchunks, 256, smem, s>>>(topk_idx, T, H, k, E, nchunks, 1, 1, 0, 0, base, kept_mine,
+                                                  nullptr, nullptr, nullptr, nullptr, slot_row);
+    const int G = H / kGroup;
+    const int64_t warps = static_cast<int64_t>(T) * ((G + 7) / 8);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_quant_kernel, 256, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t cap_blocks = static_cast<int64_t>(per_sm) * num_sms * 4;
+    const int blocks = static_cast<int>(std::min<int64_t>((warps + 7) / 8, cap_blocks));
+    if (blocks > 0)
+        permute_quant_kernel<<<blocks, 256, 0, s>>>(x, T, H, k, 0, 0, ep_row_bytes(H), true, slot_row, send, nullptr);
     return cudaGetLastError();
 }
 

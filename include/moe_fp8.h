@@ -61,6 +61,7 @@ typedef enum {
 typedef enum { MOE_ROUTE_SOFTMAX_TOPK = 0, MOE_ROUTE_HASH = 1 } moe_routing_t;
 typedef enum { MOE_LAYOUT_CONTIGUOUS = 0, MOE_LAYOUT_MASKED = 1 } moe_layout_t;
 typedef enum { MOE_EPI_BF16 = 0, MOE_EPI_SWIGLU_FP8 = 1 } moe_epilogue_t;
+typedef enum { MOE_CONTIG_AUTO = 0, MOE_CONTIG_SINGLE = 1, MOE_CONTIG_PAIR = 2 } moe_contig_kernel_t;
 
 /* Limits checked by every entry point. */
 #define MOE_MAX_EXPERTS 512
@@ -274,6 +275,27 @@ moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const void* x, const i
 moe_status_t moe_balance_bias(int E, const int32_t* counts, int64_t* load, float* bias, float gamma, int update,
                               void* stream);
 
+/*
+ * Chooses how the contiguous-layout grouped GEMM (moe_grouped_gemm_fp8 and
+ * moe_forward) is run, for every later call in this process. The grouped
+ * GEMM of the pages (MegaMoE page, 3.2) is one tile scheduler over the
+ * flattened M of all groups; on B200 it has two forms:
+ *   MOE_CONTIG_SINGLE  one CTA per 128-row x 256-column tile
+ *   MOE_CONTIG_PAIR    clusters of two CTAs, each pair computing a 256-row x
+ *                      256-column tile with paired tensor-core MMAs (each CTA
+ *                      loads its 128 rows and half of the weight tile, which
+ *                      halves the shared-memory traffic per MMA); an expert
+ *                      with an odd number of 128-row tiles computes its last
+ *                      one on one CTA of a pair while the other idles. Needs N
+ *                      a multiple of 256 (otherwise the single form runs).
+ *   MOE_CONTIG_AUTO    (the default) pairs when the buffer holds at least 2.5
+ *                      tiles of rows per expert on average (M_rows >= 320 E),
+ *                      else single CTAs.
+ * Both forms compute the same products and the same fp32 promotion, in the
+ * same order. Returns MOE_ERR_INVALID_ARG for any other value.
+ */
+moe_status_t moe_set_contig_kernel(int form);
+
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: MOE_OK, MOE_ERR_CAPACITY or MOE_ERR_DEVICE_TIMEOUT. */
 moe_status_t moe_get_device_status(void* stream);
@@ -283,6 +305,106 @@ moe_status_t moe_get_device_status(void* stream);
  * barrier that nothing completes; the wait gives up, records
  * MOE_ERR_DEVICE_TIMEOUT in the device status word and the kernel returns. */
 moe_status_t moe_selftest_wait_timeout(int limit_us, void* stream);
+
+/*
+ * ---------------------------------------------------------------- expert parallelism
+ * The layer across G GPUs, one process per GPU, experts split evenly: rank r
+ * holds experts [r E/G, (r+1) E/G) and its own batch of tokens. Sources:
+ * TP-MoE page, section 3.3 (experts placed on several cards; tokens travel to
+ * their expert's card by all-to-all and back) and 4.1 step 3 (each card routes
+ * its own tokens, then sends them by all-to-all); MegaMoE page, section 3.4
+ * (dispatch and combine as the two communication primitives); TP-MoE page,
+ * section 6.2 (the all-to-all payload compressed to FP8) and 5.3 (a send and
+ * a receive buffer of the payload). The layer's result on
+ * every rank equals that of one GPU on the ranks' batches concatenated in rank
+ * order: routing is per token, ranks within an expert (and so the capacity
+ * drop) follow that global token order, and capacity uses the global T.
+ *
+ * One step of rank r:
+ *   moe_route                   its own tokens (all E experts)
+ *   moe_ep_count                counts[E] of its slots per expert
+ *   (collective)                all-gather of counts -> [G][E] on every rank
+ *   moe_ep_plan (host)          the exchange plan below, from the gathered
+ *                               counts; the same counts give every rank a
+ *                               consistent plan
+ *   moe_ep_dispatch             quantises x (1x128, as moe_permute) once per
+ *                               token and writes one send row per kept slot,
+ *                               ordered by destination rank, then expert, then
+ *                               token; slot_row maps slot t*k+j to its send row
+ *                               (-1 if the capacity drops it)
+ *   (collective)                all-to-all of the send rows (send_rows[d] to d)
+ *   moe_ep_receive              places the received rows into the contiguous
+ *                               grouped layout of its E/G experts (padding rows
+ *                               filled) and remembers each row's place
+ *   moe_grouped_gemm_fp8 x 2    the local experts, contiguous layout
+ *   moe_ep_return               gathers each received row's expert output into
+ *                               receive order
+ *   (collective)                all-to-all back (recv_rows[s] to s)
+ *   moe_combine                 y from the returned rows (slot_row into them)
+ *
+ * A send/receive row is H bytes of E4M3 codes followed by H/128 fp32 scales,
+ * padded to a multiple of 16 bytes (row stride MOE_EP_ROW_BYTES(H)).
+ */
+#define MOE_EP_MAX_RANKS 64
+#define MOE_EP_ROW_BYTES(H) (((size_t)(H) + 4u * ((size_t)(H) / 128u) + 15u) / 16u * 16u)
+
+/* The exchange plan of one rank (host memory; the device steps read a device
+ * copy of it, which the caller makes with one copy of sizeof(moe_ep_plan_t)). */
+typedef struct {
+    int32_t G, rank, E, E_local;   /* E_local = E / G experts on each rank */
+    int32_t cap;                   /* per-expert capacity from the global T, -1 if none */
+    int32_t rows_send;             /* rows this rank sends: sum of send_rows */
+    int32_t rows_recv;             /* rows it receives: sum of recv_rows */
+    int32_t rows_group;            /* rows of its grouped layout: offsets[E_local] */
+    int32_t kept_mine[MOE_MAX_EXPERTS];      /* per expert e: this rank's slots of e kept */
+    int32_t send_rows[MOE_EP_MAX_RANKS];     /* rows for each destination rank */
+    int32_t recv_rows[MOE_EP_MAX_RANKS];     /* rows from each source rank */
+    int32_t recv_start[MOE_MAX_EXPERTS + 1]; /* block b = s * E_local + e_loc: first receive row */
+    int32_t group_start[MOE_MAX_EXPERTS];    /* block b: its first row in the grouped layout */
+    int32_t offsets[MOE_MAX_EXPERTS + 1];    /* grouped layout of the local experts, multiples of 128 */
+    int32_t kept[MOE_MAX_EXPERTS];           /* rows of each local expert (all sources) */
+} moe_ep_plan_t;
+
+/* Host-only, no GPU needed. counts_all [G][E] int32 (host): counts_all[s][e] =
+ * slots of rank s routed to expert e (moe_ep_count on rank s). T_total = the
+ * tokens of all ranks; k, cap_num and cap_den as in moe_config_t (0/0 =
+ * dropless). Capacity C = floor(ceil(T_total k / E) * cap_num / cap_den)
+ * (DeepSeek MoE page, 2.5); expert e keeps its first C slots in global token
+ * order, so rank s keeps clamp(C - sum_{s' < s} counts_all[s'][e], 0,
+ * counts_all[s][e]). Errors: G outside 1..MOE_EP_MAX_RANKS, E not a multiple
+ * of G or above MOE_MAX_EXPERTS, rank outside [0, G), negative counts,
+ * MOE_ERR_UNSUPPORTED_SHAPE when a row count would pass 2^31 / 128. */
+moe_status_t moe_ep_plan(int G, int rank, int E, int64_t T_total, int k, int cap_num, int cap_den,
+                         const int32_t* counts_all, moe_ep_plan_t* plan);
+
+/* Per-expert counts of this rank's slots: counts [E] int32 out. cfg as for
+ * moe_route on this rank's batch (cfg->T its tokens; capacity fields unused
+ * here). ws: moe_ep_workspace_size(cfg) bytes; it must be passed unchanged to
+ * the moe_ep_dispatch of the same step (it holds the slots' ranks). */
+size_t moe_ep_workspace_size(const moe_config_t* cfg);
+moe_status_t moe_ep_count(const moe_config_t* cfg, const int32_t* topk_idx, int32_t* counts, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* Send rows of this rank: send [plan.rows_send rows x MOE_EP_ROW_BYTES(H)] u8
+ * out; slot_row [T*k] out: the send row of each slot, -1 if dropped. x [T, H]
+ * bf16; plan_dev: device copy of this rank's plan; ws as moe_ep_count left it.
+ * Codes and scales are moe_permute's, bit for bit. */
+moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                             const moe_ep_plan_t* plan_dev, uint8_t* send, int32_t* slot_row, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Received rows (recv: plan.rows_recv rows x MOE_EP_ROW_BYTES(H), ordered by
+ * source rank, then local expert, then token) into the grouped layout of the
+ * local experts: Aq [M_rows, H] u8 and As [H/128][M_rows] fp32 (moe_permute's
+ * contiguous layout; padding rows code 0, scale 1), offsets [E_local + 1] out
+ * (the plan's), group_row [plan.rows_recv] int32 out: the grouped row of each
+ * received row. M_rows >= plan.rows_group, a multiple of 4. */
+moe_status_t moe_ep_receive(int H, const moe_ep_plan_t* plan_dev, int rows_recv, const uint8_t* recv, uint8_t* Aq,
+                            float* As, int M_rows, int32_t* offsets, int32_t* group_row, void* stream);
+
+/* ret [rows_recv, H] bf16 out: row i = O [group_row[i]] (the local experts'
+ * output rows, moe_grouped_gemm_fp8's bf16 epilogue) in receive order. */
+moe_status_t moe_ep_return(int H, int rows_recv, const void* O, const int32_t* group_row, void* ret, void* stream);
 
 const char* moe_status_string(moe_status_t status);
 

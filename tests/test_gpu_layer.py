@@ -54,16 +54,25 @@ def test_layer_small(name):
     _check_layer(cfg, inp, ref, out, np.arange(cfg.T))
 
 
-@pytest.mark.parametrize("name", ["page", "prefill", "decode", "decode_hash", "skewed"])
-def test_layer_full_size_tile_covering(name):
+@pytest.mark.parametrize("name,form", [("page", api.CONTIG_AUTO), ("page", api.CONTIG_PAIR),
+                                       ("prefill", api.CONTIG_AUTO), ("decode", api.CONTIG_AUTO),
+                                       ("decode_hash", api.CONTIG_AUTO), ("skewed", api.CONTIG_AUTO)])
+def test_layer_full_size_tile_covering(name, form):
     # Every workload at full size, in the launch configuration the benchmark times: routing, counts and the
     # slot -> row map (permutation and dropped set) on every token, and y on a set of tokens whose kept rows
     # reach every tile the two grouped GEMMs schedule (each 128-row M tile of the contiguous layout, each
     # 32-token slice of an expert's block in the masked layout), chosen from the oracle's own dispatch.
+    # The default kernel choice runs on every workload (CTA pairs for prefill and skewed, single CTAs for
+    # page); the page workload also runs with CTA pairs forced, where most experts fill one or two 128-row
+    # tiles, so many pair tiles are lone (one CTA of the pair idle).
     ensure_lib()
     cfg = CONFIGS[name]
     inp = gpu_inputs(cfg, on_device=True)
-    out = gpu_forward(cfg, inp)
+    api.moe_set_contig_kernel(form)
+    try:
+        out = gpu_forward(cfg, inp)
+    finally:
+        api.moe_set_contig_kernel(api.CONTIG_AUTO)
     o_in = oracle_inputs(inp)
     idx, _w, _l = oracle.route(cfg, o_in["x"], o_in["Wg"], o_in["bias"], o_in["token_ids"])
     k = idx.shape[1]

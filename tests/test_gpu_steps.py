@@ -287,12 +287,31 @@ def test_gemm_cases_include_multi_tile_launches():
                        > MANY_TILES for c in GEMM_CASES), (layout, epi)
 
 
-@pytest.mark.parametrize("case", GEMM_CASES)
-def test_grouped_gemm(case):
+class contig_form:
+    """Runs the enclosed calls with the contiguous GEMM forced to one form, then restores the default."""
+
+    def __init__(self, form):
+        self.form = form
+
+    def __enter__(self):
+        api.moe_set_contig_kernel(self.form)
+
+    def __exit__(self, *exc):
+        api.moe_set_contig_kernel(api.CONTIG_AUTO)
+
+
+# contiguous cases run in both forms of the kernel (single CTAs, CTA pairs: the pair form needs N a
+# multiple of 256 and otherwise runs single CTAs); masked cases have one form
+GEMM_RUNS = [(c, f) for c in GEMM_CASES for f in ((1, 2) if c[0] == 0 else (0,))]
+
+
+@pytest.mark.parametrize("case,form", GEMM_RUNS)
+def test_grouped_gemm(case, form):
     ensure_lib()
     layout, epi, E, N, K, groups, Mr = case
     A, As, gi, M, B, Bs = _gemm_case(layout, epi, E, N, K, groups, Mr, seed=sum(groups) + N)
-    D, Ds = _gemm_gpu(layout, epi, E, N, K, A, As, gi, M, B, Bs)
+    with contig_form(form):
+        D, Ds = _gemm_gpu(layout, epi, E, N, K, A, As, gi, M, B, Bs)
     Dr, Dsr = oracle.grouped_gemm(layout, E, N, K, A, As, gi, M, B, Bs, epi)
     rows = _valid_rows(layout, gi, M, E)
     if epi == 0:
@@ -369,8 +388,8 @@ def test_grouped_gemm_w4(case):
         assert np.allclose(s, sr, rtol=1e-5, atol=0)
 
 
-@pytest.mark.parametrize("layout,epi", [(0, 0), (0, 1), (1, 0), (1, 1)])
-def test_grouped_gemm_writes_nothing_outside_its_groups(layout, epi):
+@pytest.mark.parametrize("layout,epi,form", [(0, 0, 1), (0, 1, 1), (0, 0, 2), (0, 1, 2), (1, 0, 0), (1, 1, 0)])
+def test_grouped_gemm_writes_nothing_outside_its_groups(layout, epi, form):
     # canary-filled outputs with guard rows past the end: rows outside every group (contiguous) or at
     # and past a block's count (masked) keep the canary, as do the guard rows and their scales
     ensure_lib()
@@ -388,8 +407,9 @@ def test_grouped_gemm_writes_nothing_outside_its_groups(layout, epi):
         G = N // 256
         Dsfull = torch.full(((G, M) if layout == 0 else (E, G, M)), -3.0, dtype=torch.float32, device="cuda")
     D = Dfull[:rows]
-    api.moe_grouped_gemm_fp8(layout, E, N, K, d(A), d(As), d(gi), M, d(B), d(Bs), epi, D, Dsfull)
-    torch.cuda.synchronize()
+    with contig_form(form):
+        api.moe_grouped_gemm_fp8(layout, E, N, K, d(A), d(As), d(gi), M, d(B), d(Bs), epi, D, Dsfull)
+        torch.cuda.synchronize()
     assert api.moe_get_device_status() == api.MOE_OK
     Dh = to_np(Dfull)
     canary = 0x5A5A if epi == 0 else 0x5A
@@ -408,9 +428,10 @@ def test_grouped_gemm_writes_nothing_outside_its_groups(layout, epi):
                 assert np.all(Ds[e, :, :gi[e]] > 0)
 
 
-@pytest.mark.parametrize("layout,epi,w4", [(1, 0, False), (1, 1, False), (1, 0, True), (1, 1, True),
-                                           (0, 0, False), (0, 1, False)])
-def test_grouped_gemm_clamps_out_of_bound_groups(layout, epi, w4):
+@pytest.mark.parametrize("layout,epi,w4,form", [(1, 0, False, 0), (1, 1, False, 0), (1, 0, True, 0), (1, 1, True, 0),
+                                                (0, 0, False, 1), (0, 1, False, 1), (0, 0, False, 2),
+                                                (0, 1, False, 2)])
+def test_grouped_gemm_clamps_out_of_bound_groups(layout, epi, w4, form):
     # group sizes past the buffers (a masked count above M_rows or below 0; contiguous offsets past M_rows
     # or not a multiple of 128) are clamped on the device and reported as MOE_ERR_CAPACITY: guard rows past
     # D and past the scales keep their canary, and the groups within bounds are still exact
@@ -450,8 +471,9 @@ def test_grouped_gemm_clamps_out_of_bound_groups(layout, epi, w4):
                             dtype=torch.float32, device="cuda")
     D = Dfull[:rows]
     fn = api.moe_grouped_gemm_w4 if w4 else api.moe_grouped_gemm_fp8
-    fn(layout, E, N, K, d(A), d(As), d(gi), M, d(B), d(Bs), epi, D, Dsfull)
-    torch.cuda.synchronize()
+    with contig_form(form):
+        fn(layout, E, N, K, d(A), d(As), d(gi), M, d(B), d(Bs), epi, D, Dsfull)
+        torch.cuda.synchronize()
     assert api.moe_get_device_status() == api.MOE_ERR_CAPACITY
     assert api.moe_get_device_status() == api.MOE_OK
     Dh = to_np(Dfull)
