@@ -32,7 +32,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from fp8_grouped_gemm_fp32_b200.inputs import CONFIGS, MoeConfig, interleave_w13, make_inputs  # noqa: E402
+from fp8_grouped_gemm_fp32_b200.inputs import (CONFIGS, MoeConfig, interleave_w13, interleave_w13_w4,  # noqa: E402
+                                                make_inputs)
 
 METRIC = "MoE layer tokens/s; grouped FP8 GEMM TFLOPS and % of B200 roofline"
 FP8_PER_BF16 = 2.0          # nominal dense FP8 : BF16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
@@ -43,6 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def describe(cfg: MoeConfig) -> str:
     s = (f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} I={cfg.I} "
          f"{'hash k=1' if cfg.routing == 'hash' else f'top-{cfg.k} softmax'} {cfg.layout} layout")
+    if cfg.weights == "w4":
+        s += " 4-bit weights (row scales)"
     if cfg.cap_num:
         s += f" capacity ceil(T*k/E)*{cfg.cap_num}/{cfg.cap_den}"
     return s + f" bias={cfg.bias} seed={cfg.seed}"
@@ -173,8 +176,12 @@ def algorithmic_work(cfg: MoeConfig, kept: np.ndarray):
     Rk = int(kept.sum())
     touched = int(np.count_nonzero(kept))
     G = lambda n: n // 128
-    w13 = touched * (2 * I * H + 4 * G(2 * I) * G(H))
-    w2 = touched * (H * I + 4 * G(H) * G(I))
+    if cfg.weights == "w4":       # packed levels (half a byte each) and one fp32 scale per row per K block
+        w13 = touched * (2 * I * H // 2 + 4 * 2 * I * G(H))
+        w2 = touched * (H * I // 2 + 4 * H * G(I))
+    else:
+        w13 = touched * (2 * I * H + 4 * G(2 * I) * G(H))
+        w2 = touched * (H * I + 4 * G(H) * G(I))
     work = {
         "router": dict(bytes=(T * H * 2 + E * H * 4 + T * k * 8) if cfg.routing != "hash" else T * 4 + T * k * 8,
                        flops=2.0 * T * E * H if cfg.routing != "hash" else 0.0),
@@ -195,7 +202,8 @@ class Layer:
         self.api = api
         self.cfg = cfg
         self.inp = make_inputs(cfg.replace(seed=cfg.seed + seed_offset), device=dev)
-        self.W13, self.S13 = interleave_w13(self.inp.W1q, self.inp.S1, self.inp.W3q, self.inp.S3)
+        inter = interleave_w13_w4 if cfg.weights == "w4" else interleave_w13
+        self.W13, self.S13 = inter(self.inp.W1q, self.inp.S1, self.inp.W3q, self.inp.S3)
         self.c = api.Config.from_moe(cfg)
         T, k, H, E, I = cfg.T, cfg.k, cfg.H, cfg.E, cfg.I
         z = lambda *s, dt: torch.empty(*s, dtype=dt, device=dev)
@@ -239,11 +247,11 @@ class Layer:
         a.moe_permute(self.c, i.x, self.topk_idx, self.Aq, self.As, self.counts, self.kept, self.offsets,
                       self.row_src, self.slot_row, self.step_ws)
         ev[2].record()
-        a.moe_grouped_gemm_fp8(int(masked), cfg.E, 2 * cfg.I, cfg.H, self.Aq, self.As, group,
-                               self.M_rows, self.W13, self.S13, a.EPI_SWIGLU_FP8, self.Hq, self.Hs)
+        gemm = a.moe_grouped_gemm_w4 if cfg.weights == "w4" else a.moe_grouped_gemm_fp8
+        gemm(int(masked), cfg.E, 2 * cfg.I, cfg.H, self.Aq, self.As, group, self.M_rows, self.W13, self.S13,
+             a.EPI_SWIGLU_FP8, self.Hq, self.Hs)
         ev[3].record()
-        a.moe_grouped_gemm_fp8(int(masked), cfg.E, cfg.H, cfg.I, self.Hq, self.Hs, group, self.M_rows,
-                               i.W2q, i.S2, a.EPI_BF16, self.O)
+        gemm(int(masked), cfg.E, cfg.H, cfg.I, self.Hq, self.Hs, group, self.M_rows, i.W2q, i.S2, a.EPI_BF16, self.O)
         ev[4].record()
         a.moe_combine(self.c, self.O, self.slot_row, self.topk_w, self.y)
         ev[5].record()
@@ -399,6 +407,9 @@ def run_ours(args):
     cfg = CONFIGS[args.config]
     if args.experts:
         cfg = cfg.replace(E=args.experts)
+    if args.tokens:
+        cfg = cfg.replace(T=args.tokens, masked_max_m=(-(-args.tokens // 32) * 32 if cfg.layout == "masked"
+                                                       else cfg.masked_max_m))
     from fp8_grouped_gemm_fp32_b200 import api
     api.lib()                                      # fails loudly if the native library is missing
     api.moe_set_contig_kernel({"auto": api.CONTIG_AUTO, "single": api.CONTIG_SINGLE,
@@ -515,7 +526,9 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp8e4m3 (fp32 accumulate)", "data": "synthetic",
+        "vs_baseline": None, "data": "synthetic",
+        "dtype": ("4-bit weight levels (as e4m3) x fp8e4m3 activations, fp32 accumulate" if cfg.weights == "w4"
+                  else "fp8e4m3 (fp32 accumulate)"),
         "config": {"workload": describe(cfg), "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "contig_gemm": args.contig,
                    "l2": "no flush: the FP8 weights streamed every step (%.2f GB) exceed the 126 MB L2"
@@ -593,6 +606,8 @@ def main():
                     help="form of the contiguous grouped GEMM (default: chosen by shape)")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the workload's expert count (reduced cases for profiling captures)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (reduced cases for profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

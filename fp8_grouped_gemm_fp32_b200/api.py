@@ -29,6 +29,7 @@ ROUTE_SOFTMAX_TOPK, ROUTE_HASH = 0, 1
 LAYOUT_CONTIGUOUS, LAYOUT_MASKED = 0, 1
 EPI_BF16, EPI_SWIGLU_FP8 = 0, 1
 CONTIG_AUTO, CONTIG_SINGLE, CONTIG_PAIR = 0, 1, 2
+WEIGHTS_FP8, WEIGHTS_W4 = 0, 1
 EXPORTS = ("moe_rows_capacity", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_gemm_fp8",
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string",
            "moe_permute_noalloc", "moe_balance_bias", "moe_grouped_gemm_w4", "moe_set_contig_kernel",
@@ -44,7 +45,7 @@ class MoeError(RuntimeError):
 
 class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("T", "H", "E", "I", "k", "routing", "cap_num", "cap_den",
-                                            "layout", "masked_max_m")]
+                                            "layout", "masked_max_m", "weights")]
 
     @classmethod
     def from_moe(cls, cfg) -> "Config":
@@ -53,7 +54,7 @@ class Config(ctypes.Structure):
                    ROUTE_HASH if cfg.routing == "hash" else ROUTE_SOFTMAX_TOPK,
                    cfg.cap_num, cfg.cap_den,
                    LAYOUT_MASKED if cfg.layout == "masked" else LAYOUT_CONTIGUOUS,
-                   cfg.masked_max_m)
+                   cfg.masked_max_m, WEIGHTS_W4 if getattr(cfg, "weights", "fp8") == "w4" else WEIGHTS_FP8)
 
 
 _lib = None

@@ -51,6 +51,7 @@ moe_status_t check_cfg(const moe_config_t* c) {
     if (c->cap_num < 0 || c->cap_den < 0 || ((c->cap_num == 0) != (c->cap_den == 0))) return MOE_ERR_INVALID_ARG;
     if (c->layout != MOE_LAYOUT_CONTIGUOUS && c->layout != MOE_LAYOUT_MASKED) return MOE_ERR_INVALID_ARG;
     if (c->layout == MOE_LAYOUT_MASKED && (c->masked_max_m <= 0 || c->masked_max_m % 32)) return MOE_ERR_INVALID_ARG;
+    if (c->weights != MOE_WEIGHTS_FP8 && c->weights != MOE_WEIGHTS_W4) return MOE_ERR_INVALID_ARG;
     const int64_t rows = c->layout == MOE_LAYOUT_MASKED
                              ? static_cast<int64_t>(c->E) * c->masked_max_m
                              : static_cast<int64_t>(c->T) * c->k + static_cast<int64_t>(c->E) * (kGroup - 1);
@@ -304,6 +305,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
     if (cfg->routing == MOE_ROUTE_SOFTMAX_TOPK && (!ptr_ok(Wg) || (bias && !aligned16(bias))))
         return MOE_ERR_INVALID_ARG;
     if (cfg->routing == MOE_ROUTE_HASH && !ptr_ok(token_ids)) return MOE_ERR_INVALID_ARG;
+    if (cfg->weights == MOE_WEIGHTS_W4 && cfg->layout != MOE_LAYOUT_MASKED) return MOE_ERR_UNSUPPORTED_SHAPE;
     const FwdWs w = carve(cfg, ws);
     if (ws_bytes < w.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (cfg->T == 0) return MOE_OK;
@@ -323,11 +325,19 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
                        masked ? cfg->masked_max_m : 0, rows, w.Aq, w.As, counts, w.kept, w.offsets, w.row_src,
                        slot_row, w.step, dev->status, dev->num_sms, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_grouped_gemm(cfg->layout, cfg->E, 2 * cfg->I, cfg->H, w.Aq, w.As, group, M_rows, W13, S13,
-                            MOE_EPI_SWIGLU_FP8, w.Hq, w.Hs, dev->status, kWaitNs, dev->num_sms, s);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_grouped_gemm(cfg->layout, cfg->E, cfg->H, cfg->I, w.Hq, w.Hs, group, M_rows, W2, S2, MOE_EPI_BF16,
-                            w.O, nullptr, dev->status, kWaitNs, dev->num_sms, s);
+    if (cfg->weights == MOE_WEIGHTS_W4) {
+        e = launch_grouped_gemm_w4(cfg->E, 2 * cfg->I, cfg->H, w.Aq, w.As, group, M_rows, W13, S13, MOE_EPI_SWIGLU_FP8,
+                                   w.Hq, w.Hs, dev->status, kWaitNs, dev->num_sms, s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = launch_grouped_gemm_w4(cfg->E, cfg->H, cfg->I, w.Hq, w.Hs, group, M_rows, W2, S2, MOE_EPI_BF16, w.O,
+                                   nullptr, dev->status, kWaitNs, dev->num_sms, s);
+    } else {
+        e = launch_grouped_gemm(cfg->layout, cfg->E, 2 * cfg->I, cfg->H, w.Aq, w.As, group, M_rows, W13, S13,
+                                MOE_EPI_SWIGLU_FP8, w.Hq, w.Hs, dev->status, kWaitNs, dev->num_sms, s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = launch_grouped_gemm(cfg->layout, cfg->E, cfg->H, cfg->I, w.Hq, w.Hs, group, M_rows, W2, S2, MOE_EPI_BF16,
+                                w.O, nullptr, dev->status, kWaitNs, dev->num_sms, s);
+    }
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_combine(w.O, slot_row, topk_w, cfg->T, cfg->k, cfg->H, static_cast<uint16_t*>(y), s);
     return cuda_status(e);

@@ -31,9 +31,11 @@
 //   tiny; experts with no tokens produce no tiles. A second weight format,
 //   4-bit levels -7..7 with one fp32 scale per weight row per 128-wide K
 //   block (DeepSeek-V4 lecture page, 3.1), runs through the same kernel:
-//   TMA brings the packed levels, four converter warps expand them to E4M3
-//   codes (every level is exact in E4M3) in the swizzled layout the MMA
-//   reads, and each promotion thread applies its own row's scale.
+//   TMA brings the packed levels into a deep ring, four converter warps
+//   expand them to E4M3 codes (every level is exact in E4M3) and write them
+//   into tensor memory, from where the MMA reads its A operand (no expanded
+//   copy passes through shared memory), and each promotion thread applies its
+//   own row's scale.
 //
 // Every wait on an mbarrier is bounded; a wait that runs out records
 // MOE_ERR_DEVICE_TIMEOUT, the CTA stops issuing work, lets copies and MMAs in
@@ -581,43 +583,51 @@ constexpr int kWBlk = kBM * kBK;              // 16 KB: 128 weight rows x 128 K 
 // threads: warp 0 TMA, warp 1 MMA, then the promotion warps: four for SwiGLU (a thread holds a weight
 // row's 32 gate and 32 up columns), eight for the bf16 output (two warps per lane quadrant, 16 token
 // columns each, so two warps share each scheduler's promotion work)
-// With 4-bit weights (W4) four more warps expand each stage's packed levels to E4M3 codes.
+// With 4-bit weights (W4) four more warps, one per tensor-memory lane quadrant, expand each stage's packed
+// levels to E4M3 codes and write them into tensor memory, where the MMA reads its A operand.
 template <int EPI, bool W4 = false>
 __host__ __device__ constexpr int masked_threads() { return (EPI == 1 ? 192 : 320) + (W4 ? 128 : 0); }
 
-// 4-bit weight levels, four per 16 bits in k order (4-bit two's complement), to four E4M3 codes: one
-// byte permute reads the codes of 0..7, one the codes of -8..-1, and one in sign-replicate mode builds
-// the byte mask of the negative levels.
 __device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
 }
-__device__ __forceinline__ uint32_t w4x4_to_e4m3x4(uint32_t h) {
-    const uint32_t sel = h & 0x7777u;
-    const uint32_t pos = prmt_b32(0x44403800u, 0x4e4c4a48u, sel);
-    const uint32_t neg = prmt_b32(0xcaccced0u, 0xb8c0c4c8u, sel);
-    const uint32_t sg = h & 0x8888u;
-    const uint32_t mask = prmt_b32(0x00008000u, 0u, sg | (sg >> 3));
-    return (pos & ~mask) | (neg & mask);
+
+// Eight 4-bit weight levels of consecutive k (one 32-bit word of the packed row: level i < 4 has its
+// magnitude in bits 4i..4i+2 and its sign in bit 8i+7, level 4+i its magnitude in bits 16+4i..16+4i+2
+// and its sign in bit 8i+3) to eight E4M3 codes, k order, two words. A byte permute looks the magnitudes'
+// codes up (0..7 are exact in E4M3: 0x00 38 40 44 48 4a 4c 4e) and the sign bits, already at bit 7 of
+// their bytes (after a 4-bit shift for the upper four), are or-ed in: E4M3's sign is its top bit.
+__device__ __forceinline__ void w4x8_to_e4m3x8(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    lo = prmt_b32(0x44403800u, 0x4e4c4a48u, w & 0x7777u) | (w & 0x80808080u);
+    hi = prmt_b32(0x44403800u, 0x4e4c4a48u, (w >> 16) & 0x7777u) | ((w << 4) & 0x80808080u);
 }
 
 template <int EPI, bool W4 = false>
 struct SmemM {
-    static constexpr int kW = EPI == 1 ? 2 * kWBlk : kWBlk;    // weight rows per stage: 256 (a|b) or 128
-    static constexpr int kStages = W4 ? (EPI == 1 ? 3 : 6) : (EPI == 1 ? 4 : 10);
-    static constexpr int kWP = W4 ? kW / 2 : 16;               // packed 4-bit levels per stage
-    static constexpr int kCols = EPI == 1 ? 2 * kBT : kBT;     // tensor-memory columns per buffer
+    static constexpr int kW = EPI == 1 ? 2 * kWBlk : kWBlk;    // weight bytes per stage: 256 rows (a|b) or 128
+    // W4: a deep ring of packed stages (8 or 16 KB of levels + the 4 KB token tile each); the expanded
+    // codes live in tensor memory (kA slots) instead of shared memory
+    static constexpr int kStages = W4 ? (EPI == 1 ? 8 : 16) : (EPI == 1 ? 4 : 10);
+    static constexpr int kWS = W4 ? 16 : kW;                   // expanded codes in shared memory (FP8 only)
+    static constexpr int kWP = W4 ? kW / 2 : 16;               // packed 4-bit levels per stage (W4 only)
+    static constexpr int kCols = EPI == 1 ? 2 * kBT : kBT;     // tensor-memory columns per accumulator buffer
     static constexpr int kBufs = 4;                            // MMA runs up to 3 K blocks ahead of promotion
     static constexpr int kSaSlots = 16;                        // scale ring deeper than the stage ring
-    uint8_t w[kStages][kW];
-    uint8_t x[kStages][kXBytes];
-    uint8_t wp[kStages][kWP];                                   // packed levels (W4), 64 bytes per row
+    static constexpr int kACols = kW / kBM / 4;                // W4: tensor-memory columns of one A slot (32 or 64)
+    static constexpr int kA = W4 ? (EPI == 1 ? 4 : 8) : 1;     // W4: A slots after the accumulators
+    static constexpr uint32_t kTmemCols = W4 ? 512u : static_cast<uint32_t>(kBufs * kCols);
+    static_assert(!W4 || kBufs * kCols + kA * kACols <= 512, "tensor memory holds the accumulators and A slots");
+    alignas(1024) uint8_t x[kStages][kXBytes];                  // 128-byte swizzled tiles: 1024-byte aligned
+    alignas(1024) uint8_t w[kStages][kWS];
+    alignas(1024) uint8_t wp[kStages][kWP];                     // packed levels (W4), 64 bytes per row, 64-byte swizzle
     float hs[EPI == 1 ? 2 : 1][EPI == 1 ? kBT : 1][kBM];       // SwiGLU output staged for the requant
     float sa[kSaSlots][kBT];                                    // activation scales of one K block, 32 tokens
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t conv[kStages];                                     // W4: the stage's levels are expanded
+    uint64_t afull[kA];                                         // W4: A slot written by the converter warps
+    uint64_t aempty[kA];                                        // W4: A slot read by the MMA
     uint64_t sfull[kSaSlots];
     uint64_t sempty[kSaSlots];
     uint64_t tfull[kBufs];
@@ -628,6 +638,15 @@ struct SmemM {
     int32_t P[kMaxE + 1];
     int32_t M[kMaxE];                                           // tokens per expert (masked_m)
 };
+
+// every layout, plus the 1 KB the kernels spend aligning it, within the 227 KB a CTA may use
+constexpr size_t kSmemLimit = 232448;
+static_assert(sizeof(SmemC<0, false>) + 1024 <= kSmemLimit && sizeof(SmemC<1, false>) + 1024 <= kSmemLimit &&
+              sizeof(SmemC<0, true>) + 1024 <= kSmemLimit && sizeof(SmemC<1, true>) + 1024 <= kSmemLimit,
+              "contiguous kernel shared memory");
+static_assert(sizeof(SmemM<0, false>) + 1024 <= kSmemLimit && sizeof(SmemM<1, false>) + 1024 <= kSmemLimit &&
+              sizeof(SmemM<0, true>) + 1024 <= kSmemLimit && sizeof(SmemM<1, true>) + 1024 <= kSmemLimit,
+              "masked kernel shared memory");
 
 template <int EPI, bool W4>
 __global__ void __launch_bounds__(masked_threads<EPI, W4>(), 1)
@@ -644,7 +663,8 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     const int KB = K / kBK;
     const int NB = N / kBM;                          // 128-row weight blocks per expert
     const int NBt = EPI == 1 ? NB / 2 : NB;          // weight tiles per expert
-    constexpr uint32_t kTmemCols = S::kBufs * S::kCols;        // 256 (SwiGLU) or 128 columns
+    constexpr uint32_t kTmemCols = S::kTmemCols;
+    constexpr uint32_t kA0 = S::kBufs * S::kCols;              // W4: first column of the A slots
 
     if (warp == 0) {
         // tile prefix over experts: tiles_e = NBt * ceil(m_e / 32)
@@ -671,8 +691,12 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     if (threadIdx.x == 32) {
         for (int s = 0; s < S::kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 1);
-            if (W4) mbar_init(&sm.conv[s], 4);
+            // W4: a stage is free once the MMA has read its token tile and the four converter warps its levels
+            mbar_init(&sm.empty[s], W4 ? 5 : 1);
+        }
+        for (int a = 0; a < S::kA; ++a) {
+            mbar_init(&sm.afull[a], 4);
+            mbar_init(&sm.aempty[a], 1);
         }
         for (int j = 0; j < S::kSaSlots; ++j) {
             mbar_init(&sm.sfull[j], 1);
@@ -752,16 +776,30 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     const int buf = kbt % S::kBufs;
                     const uint32_t bph = (kbt / S::kBufs) & 1;
                     if (!mbar_wait(&sm.full[s], ph, wait_ns)) { fail(); break; }
-                    if (W4 && !mbar_wait(&sm.conv[s], ph, wait_ns)) { fail(); break; }
+                    const int a = it % S::kA;
+                    if (W4 && !mbar_wait(&sm.afull[a], (it / S::kA) & 1, wait_ns)) { fail(); break; }
                     if (!mbar_wait(&sm.tempty[buf], bph ^ 1, wait_ns)) { fail(); break; }
                     tc_fence_after();
-                    const uint32_t w0 = smem_u32(sm.w[s]), x0 = smem_u32(sm.x[s]);
+                    const uint32_t x0 = smem_u32(sm.x[s]);
                     const uint32_t d = tmem + buf * S::kCols;
+                    if constexpr (W4) {
+                        // A (the expanded weight rows) from tensor memory: 8 columns per 32-wide K slice
+                        const uint32_t a0 = tmem + kA0 + a * S::kACols;
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 32; ++kk) {
-                        const uint64_t xd = sw128_kmajor_desc(x0 + kk * 32);
-                        umma_f8(d, sw128_kmajor_desc(w0 + kk * 32), xd, idesc, kk > 0);
-                        if (EPI == 1) umma_f8(d + kBT, sw128_kmajor_desc(w0 + kWBlk + kk * 32), xd, idesc, kk > 0);
+                        for (int kk = 0; kk < kBK / 32; ++kk) {
+                            const uint64_t xd = sw128_kmajor_desc(x0 + kk * 32);
+                            umma_f8_ta(d, a0 + kk * 8, xd, idesc, kk > 0);
+                            if (EPI == 1) umma_f8_ta(d + kBT, a0 + 32 + kk * 8, xd, idesc, kk > 0);
+                        }
+                        umma_commit(&sm.aempty[a]);
+                    } else {
+                        const uint32_t w0 = smem_u32(sm.w[s]);
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 32; ++kk) {
+                            const uint64_t xd = sw128_kmajor_desc(x0 + kk * 32);
+                            umma_f8(d, sw128_kmajor_desc(w0 + kk * 32), xd, idesc, kk > 0);
+                            if (EPI == 1) umma_f8(d + kBT, sw128_kmajor_desc(w0 + kWBlk + kk * 32), xd, idesc, kk > 0);
+                        }
                     }
                     umma_commit(&sm.empty[s]);
                     umma_commit(&sm.tfull[buf]);
@@ -769,11 +807,14 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
         }
     } else if (W4 && warp >= kConvWarp0) {
-        // expansion of each stage's packed levels: thread ct takes 16-byte chunk cc of rows cr + 16 j, so
-        // a warp reads four whole packed rows and writes four whole 128-byte rows in the 128-byte
-        // swizzled layout the MMA descriptor reads (chunk c of row r at c ^ (r & 7))
-        const int ct = threadIdx.x - kConvWarp0 * 32;
-        const int cr = ct >> 3, cc = ct & 7;
+        // Expansion: thread = tensor-memory lane = weight row r of the tile (warp % 4 is the lane quadrant
+        // it may write). The row's packed levels of a K block (64 bytes per 128-row block, 64-byte
+        // swizzled by TMA: 16-byte piece c of row r at c ^ ((r >> 1) & 3), conflict-free across eight
+        // rows) go to registers, which frees the stage's levels; the 128 codes go to the row's 32 columns
+        // of an A slot (64 for the gate and up blocks), whose completion the MMA waits on.
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         uint32_t it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
@@ -781,22 +822,34 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 if (sm.abort_flag) { ok = false; break; }
                 const int s = it % S::kStages;
                 const uint32_t ph = (it / S::kStages) & 1;
+                const int a = it % S::kA;
                 if (!mbar_wait(&sm.full[s], ph, wait_ns)) { fail(); ok = false; break; }
+                uint4 pk[EPI == 1 ? 2 : 1][4];
+#pragma unroll
+                for (int b = 0; b < (EPI == 1 ? 2 : 1); ++b)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        pk[b][c] = *reinterpret_cast<const uint4*>(sm.wp[s] + b * (kWBlk / 2) + r * (kBK / 2) +
+                                                                   ((c ^ ((r >> 1) & 3)) << 4));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.empty[s]);
+                if (!mbar_wait(&sm.aempty[a], ((it / S::kA) & 1) ^ 1, wait_ns)) { fail(); ok = false; break; }
+                tc_fence_after();
 #pragma unroll
                 for (int b = 0; b < (EPI == 1 ? 2 : 1); ++b) {
-                    const uint8_t* src = sm.wp[s] + b * (kWBlk / 2);
-                    const uint32_t dst = smem_u32(sm.w[s] + b * kWBlk);
+                    uint32_t codes[32];
 #pragma unroll
-                    for (int j = 0; j < kBM / 16; ++j) {
-                        const int r = cr + 16 * j;
-                        const uint2 p = *reinterpret_cast<const uint2*>(src + r * (kBK / 2) + cc * 8);
-                        st_shared_v4(dst + r * kBK + ((cc ^ (r & 7)) << 4), w4x4_to_e4m3x4(p.x),
-                                     w4x4_to_e4m3x4(p.x >> 16), w4x4_to_e4m3x4(p.y), w4x4_to_e4m3x4(p.y >> 16));
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t wv[4] = {pk[b][c].x, pk[b][c].y, pk[b][c].z, pk[b][c].w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) w4x8_to_e4m3x8(wv[j], codes[8 * c + 2 * j], codes[8 * c + 2 * j + 1]);
                     }
+                    tmem_st32(tmem + lane_base + kA0 + a * S::kACols + b * 32, codes);
                 }
-                fence_proxy_async_smem();
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.conv[s]);
+                if (lane == 0) mbar_arrive(&sm.afull[a]);
             }
         }
     } else {
@@ -1043,15 +1096,13 @@ static int g_contig_mode = 0;
 
 void set_contig_mode(int mode) { __atomic_store_n(&g_contig_mode, mode, __ATOMIC_RELAXED); }
 
-// CTA pairs need whole 256-column tiles. They pay off when most experts fill several 128-row tiles: a
-// group with an odd tile count leaves half of its last pair idle, so the rows the buffer holds per expert
-// (capacity, padding included) must average at least two and a half tiles.
+// CTA pairs need whole 256-column tiles; they run only when asked for (the default is single CTAs, the
+// faster form as measured on the prefill and skewed workloads).
 static bool use_pairs(int E, int N, int M_rows) {
+    (void)E;
+    (void)M_rows;
     if (N % kBN) return false;
-    const int mode = __atomic_load_n(&g_contig_mode, __ATOMIC_RELAXED);
-    if (mode == 1) return false;
-    if (mode == 2) return true;
-    return static_cast<int64_t>(M_rows) * 2 >= static_cast<int64_t>(5) * kBM * E;
+    return __atomic_load_n(&g_contig_mode, __ATOMIC_RELAXED) == 2;
 }
 
 cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
@@ -1094,8 +1145,9 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
     return cudaGetLastError();
 }
 
-// 2-D map over a row-major byte matrix [rows, cols] read in boxes of 64 bytes x box_rows, unswizzled
-// (4-bit weights: 64 bytes hold a row's 128 levels of one K block).
+// 2-D map over a row-major byte matrix [rows, cols] read in boxes of 64 bytes x box_rows with the 64-byte
+// swizzle (4-bit weights: 64 bytes hold a row's 128 levels of one K block; 16-byte piece c of row r lands
+// at c ^ ((r >> 1) & 3), so eight consecutive rows read at the same piece hit distinct banks).
 static bool make_packed_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
     EncodeTiledFn fn = tensor_map_encoder();
     if (!fn) return false;
@@ -1104,7 +1156,7 @@ static bool make_packed_map(CUtensorMap* m, const void* base, uint64_t cols, uin
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK / 2), box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -18,6 +18,8 @@
 // cores: the fixed order rules out the tensor cores). Logits go to scratch,
 // and a warp-per-token kernel selects the top-k and computes the weights in
 // fp64. W_g (7.3 MB at the largest size) stays L2-resident across token tiles.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -54,20 +56,28 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     const int lane = threadIdx.x & 31;
     const int warp = (threadIdx.x >> 5) - (DP ? 1 : 0);             // compute warp index; -1: producer warp
     const int wt = warp / WE, we = warp % WE;
-    const int t_base = blockIdx.x * C::TT, e_base = blockIdx.y * C::EC;
     const int nst = H / kRouterHS;
     const bool producer = threadIdx.x == 0;
+    // Persistent: the CTA takes tiles blockIdx.x, blockIdx.x + gridDim.x, ... of (token tile, expert tile),
+    // the expert tile varying fastest so that the CTAs running together share each x tile through L2.
+    // The stage ring runs on across tiles: global stage g = (the CTA's i-th tile) * nst + stage in tile.
+    const int ET = (E + C::EC - 1) / C::EC;
+    const int tiles = ((T + C::TT - 1) / C::TT) * ET;
+    const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int64_t stages_total = static_cast<int64_t>(my_tiles) * nst;
 
     auto fail = [&]() {
         set_status(status, kStatusTimeout);
         *abort_flag = 1;
     };
-    auto issue = [&](int st) {      // stage st into slot st % kStages
-        const int s = st % C::kStages;
+    auto issue = [&](int64_t g) {      // global stage g into slot g % kStages
+        const int s = static_cast<int>(g % C::kStages);
+        const int tile = blockIdx.x + static_cast<int>(g / nst) * gridDim.x;
+        const int st = static_cast<int>(g % nst);
         uint8_t* stage = smem + s * C::kStageBytes;
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-        tma_load_2d(stage, &tmX, &full[s], st * kRouterHS, t_base);
-        tma_load_2d(stage + C::kXBytes, &tmW, &full[s], st * kRouterHS, e_base);
+        tma_load_2d(stage, &tmX, &full[s], st * kRouterHS, (tile / ET) * C::TT);
+        tma_load_2d(stage + C::kXBytes, &tmW, &full[s], st * kRouterHS, (tile % ET) * C::EC);
     };
     if (producer) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -78,35 +88,49 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         fence_mbar_init();
         prefetch_tensormap(&tmX);
         prefetch_tensormap(&tmW);
-        for (int st = 0; st < C::kStages && st < nst; ++st) issue(st);
+        for (int64_t g = 0; g < C::kStages && g < stages_total; ++g) issue(g);
     }
     __syncthreads();
 
     if (DP && warp < 0) {
         // dedicated producer: refill each slot as soon as every compute warp has finished with it
         if (producer)
-            for (int st = C::kStages; st < nst && !*abort_flag; ++st) {
-                const int u = st / C::kStages - 1;
-                if (!mbar_wait(&empty[st % C::kStages], u & 1, wait_ns)) { fail(); break; }
-                issue(st);
+            for (int64_t g = C::kStages; g < stages_total && !*abort_flag; ++g) {
+                const int64_t u = g / C::kStages - 1;
+                if (!mbar_wait(&empty[g % C::kStages], static_cast<uint32_t>(u & 1), wait_ns)) { fail(); break; }
+                issue(g);
             }
         __syncthreads();
+        if (*abort_flag) {
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < 200000) __nanosleep(1000);
+        }
         return;
     }
+    bool ok = true;
+    int64_t g = 0;
+    for (int it = 0; it < my_tiles && ok; ++it) {
+    const int tile = blockIdx.x + it * gridDim.x;
+    const int t_base = (tile / ET) * C::TT, e_base = (tile % ET) * C::EC;
     float acc[TR][ER];
 #pragma unroll
     for (int i = 0; i < TR; ++i)
 #pragma unroll
         for (int q = 0; q < ER; ++q) acc[i][q] = 0.0f;
-    bool ok = true;
-    for (int st = 0; st < nst; ++st) {
-        // the slot of stage st - 1 takes stage st - 1 + kStages once every warp has finished with it
-        if (!DP && producer && st > 0 && st - 1 + C::kStages < nst) {
-            if (!mbar_wait(&empty[(st - 1) % C::kStages], ((st - 1) / C::kStages) & 1, wait_ns)) fail();
-            else issue(st - 1 + C::kStages);
+    for (int st = 0; st < nst; ++st, ++g) {
+        // the slot of stage g - 1 takes stage g - 1 + kStages once every warp has finished with it
+        if (!DP && producer && g > 0 && g - 1 + C::kStages < stages_total) {
+            if (!mbar_wait(&empty[(g - 1) % C::kStages], static_cast<uint32_t>(((g - 1) / C::kStages) & 1), wait_ns))
+                fail();
+            else
+                issue(g - 1 + C::kStages);
         }
-        const int s = st % C::kStages;
-        if (*abort_flag || !mbar_wait(&full[s], (st / C::kStages) & 1, wait_ns)) { fail(); ok = false; break; }
+        const int s = static_cast<int>(g % C::kStages);
+        if (*abort_flag || !mbar_wait(&full[s], static_cast<uint32_t>((g / C::kStages) & 1), wait_ns)) {
+            fail();
+            ok = false;
+            break;
+        }
         const uint8_t* stage = smem + s * C::kStageBytes;
         const uint16_t* xs = reinterpret_cast<const uint16_t*>(stage) + (wt * TR) * kRouterHS + 4 * lane;
         const float* ws = reinterpret_cast<const float*>(stage + C::kXBytes) + (we * ER) * kRouterHS + 4 * lane;
@@ -163,6 +187,7 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
             const int t = t_base + wt * TR + n / ER, e = e_base + we * ER + n % ER;
             if (t < T && e < E) logits[static_cast<int64_t>(t) * E + e] = bias ? v[m] + bias[e] : v[m];
         }
+    }
     }
     __syncthreads();
     if (*abort_flag) {
@@ -258,7 +283,7 @@ static bool make_router_map(CUtensorMap* m, CUtensorMapDataType dt, int elem_byt
 
 template <int TR, int ER, int WT, int WE, bool DP>
 static cudaError_t launch_logits(const uint16_t* x, const float* Wg, const float* bias, float* logits, int T, int H,
-                                 int E, int* status, uint64_t wait_ns, cudaStream_t s) {
+                                 int E, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s) {
     using C = RouterCfg<TR, ER, WT, WE, DP>;
     CUtensorMap mx, mw;
     if (!make_router_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, H, T, C::TT) ||
@@ -267,7 +292,8 @@ static cudaError_t launch_logits(const uint16_t* x, const float* Wg, const float
     auto kern = router_logits_kernel<TR, ER, WT, WE, DP>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (err != cudaSuccess) return err;
-    dim3 grid((T + C::TT - 1) / C::TT, (E + C::EC - 1) / C::EC);
+    const long tiles = static_cast<long>((T + C::TT - 1) / C::TT) * ((E + C::EC - 1) / C::EC);
+    const int grid = static_cast<int>(std::min<long>(tiles, num_sms));     // one CTA per SM, persistent
     kern<<<grid, C::kThreads, C::kSmem, s>>>(mx, mw, bias, logits, T, H, E, status, wait_ns);
     return cudaGetLastError();
 }
@@ -280,11 +306,11 @@ cudaError_t launch_router_softmax(const uint16_t* x, const float* Wg, const floa
     const long ctas_big = static_cast<long>((T + 31) / 32) * ((E + 31) / 32);
     const long ctas_mid = static_cast<long>((T + 15) / 16) * ((E + 15) / 16);
     if (ctas_big >= num_sms)
-        err = launch_logits<8, 8, 4, 4, false>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);  // 32 tokens x 32 experts
+        err = launch_logits<8, 8, 4, 4, false>(x, Wg, bias, logits, T, H, E, status, wait_ns, num_sms, s);  // 32 tokens x 32 experts
     else if (ctas_mid >= num_sms)
-        err = launch_logits<8, 4, 2, 4, true>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);   // 16 tokens x 16 experts
+        err = launch_logits<8, 4, 2, 4, true>(x, Wg, bias, logits, T, H, E, status, wait_ns, num_sms, s);   // 16 tokens x 16 experts
     else
-        err = launch_logits<8, 4, 1, 4, true>(x, Wg, bias, logits, T, H, E, status, wait_ns, s);   // 8 tokens x 16 experts
+        err = launch_logits<8, 4, 1, 4, true>(x, Wg, bias, logits, T, H, E, status, wait_ns, num_sms, s);   // 8 tokens x 16 experts
     if (err != cudaSuccess) return err;
     const int blocks = (T + 7) / 8;
     if (E <= 64)

@@ -58,6 +58,7 @@ class MoeConfig:
     cap_den: int = 0
     masked_max_m: int = 0
     seed: int = 0
+    weights: str = "fp8"              # "fp8" (E4M3, 128x128 block scales) | "w4" (4-bit levels, row scales)
 
     def replace(self, **kw) -> "MoeConfig":
         return dataclasses.replace(self, **kw)
@@ -73,6 +74,9 @@ CONFIGS = {
                              layout="masked", masked_max_m=128, seed=3),
     "skewed": MoeConfig("skewed", T=16384, H=4096, E=64, I=1408, k=2, bias="zipf",
                         cap_num=5, cap_den=4, seed=4),
+    # the decode workload with 4-bit expert weights (DeepSeek-V4 lecture page, 3.1)
+    "decode_w4": MoeConfig("decode_w4", T=128, H=7168, E=256, I=2048, k=8, bias="uniform",
+                           layout="masked", masked_max_m=128, seed=3, weights="w4"),
 }
 
 
@@ -83,12 +87,12 @@ class MoeInputs:
     Wg: torch.Tensor           # [E, H] fp32
     bias: torch.Tensor         # [E] fp32
     token_ids: torch.Tensor    # [T] int32
-    W1q: torch.Tensor          # [E, I, H] uint8 (E4M3 codes), K(=H)-major
-    S1: torch.Tensor           # [E, I/128, H/128] fp32
-    W3q: torch.Tensor          # [E, I, H] uint8
-    S3: torch.Tensor           # [E, I/128, H/128] fp32
-    W2q: torch.Tensor          # [E, H, I] uint8, K(=I)-major
-    S2: torch.Tensor           # [E, H/128, I/128] fp32
+    W1q: torch.Tensor          # [E, I, H] uint8 (E4M3 codes), K(=H)-major; w4: [E, I, H/2] packed levels
+    S1: torch.Tensor           # [E, I/128, H/128] fp32; w4: [E, H/128, I] (K-block-major row scales)
+    W3q: torch.Tensor          # [E, I, H] uint8; w4: [E, I, H/2]
+    S3: torch.Tensor           # [E, I/128, H/128] fp32; w4: [E, H/128, I]
+    W2q: torch.Tensor          # [E, H, I] uint8, K(=I)-major; w4: [E, H, I/2]
+    S2: torch.Tensor           # [E, H/128, I/128] fp32; w4: [E, I/128, H]
 
     def to(self, device) -> "MoeInputs":
         kw = {f.name: getattr(self, f.name) for f in dataclasses.fields(self)}
@@ -116,15 +120,24 @@ def quantize_weight_int4(w: torch.Tensor):
     each scaled by its max-abs, levels round((w / max|w|) * (2^3 - 1))): [N, K] fp32 ->
     (codes uint8 [N, K/2], fp32 scales [N, K/128]). A block is one row by 128 consecutive k; the level
     is rounded half to even (torch.round) from the exact ratio (float64); the stored scale is
-    max-abs / 7 in fp32 (1.0 for an all-zero block), so a weight dequantises to level * scale. Two
-    levels per byte, the even k in the low nibble, as 4-bit two's-complement integers."""
+    max-abs / 7 in fp32 (1.0 for an all-zero block), so a weight dequantises to level * scale.
+    Levels are stored as a sign and a 3-bit magnitude, eight consecutive k per little-endian 32-bit
+    word: level i (i = 0..3) has its magnitude in bits 4i..4i+2 and its sign in bit 8i+7, level 4+i
+    its magnitude in bits 16+4i..16+4i+2 and its sign in bit 8i+3 (a pure bit layout)."""
     N, K = w.shape
     blk = w.reshape(N, K // BLOCK, BLOCK)
     amax = blk.abs().amax(dim=2)
     lev = torch.where(amax[..., None] > 0, (blk.double() * 7.0 / amax.double()[..., None]).round(),
                       torch.zeros_like(blk, dtype=torch.float64))
-    lev = lev.to(torch.int16).reshape(N, K // 2, 2) & 15
-    codes = (lev[..., 0] | (lev[..., 1] << 4)).to(torch.uint8)
+    lev = lev.to(torch.int64).reshape(N, K // 8, 8)
+    mag, neg = lev.abs(), (lev < 0).to(torch.int64)
+    word = torch.zeros(N, K // 8, dtype=torch.int64, device=w.device)
+    for i in range(4):
+        word |= mag[..., i] << (4 * i)
+        word |= neg[..., i] << (8 * i + 7)
+        word |= mag[..., 4 + i] << (16 + 4 * i)
+        word |= neg[..., 4 + i] << (8 * i + 3)
+    codes = torch.stack([(word >> (8 * b)) & 255 for b in range(4)], dim=-1).to(torch.uint8).reshape(N, K // 2)
     scale = torch.where(amax > 0, amax / 7.0, torch.ones_like(amax))
     return codes.contiguous(), scale.contiguous()
 
@@ -158,19 +171,40 @@ def make_inputs(cfg: MoeConfig, device="cpu", T: Optional[int] = None) -> MoeInp
     Wg = torch.randn(E, H, generator=g, device=dev, dtype=torch.float32) * 0.02
     bias = _bias(cfg, g, dev)
     token_ids = torch.randint(0, 102400, (Tn,), generator=g, device=dev, dtype=torch.int32)
-    W1q = torch.empty(E, I, H, dtype=torch.uint8, device=dev)
-    W3q = torch.empty(E, I, H, dtype=torch.uint8, device=dev)
-    W2q = torch.empty(E, H, I, dtype=torch.uint8, device=dev)
-    S1 = torch.empty(E, I // BLOCK, H // BLOCK, dtype=torch.float32, device=dev)
+    w4 = cfg.weights == "w4"
+    cols = (lambda K: K // 2) if w4 else (lambda K: K)
+    W1q = torch.empty(E, I, cols(H), dtype=torch.uint8, device=dev)
+    W3q = torch.empty(E, I, cols(H), dtype=torch.uint8, device=dev)
+    W2q = torch.empty(E, H, cols(I), dtype=torch.uint8, device=dev)
+    if w4:
+        S1 = torch.empty(E, H // BLOCK, I, dtype=torch.float32, device=dev)
+        S2 = torch.empty(E, I // BLOCK, H, dtype=torch.float32, device=dev)
+    else:
+        S1 = torch.empty(E, I // BLOCK, H // BLOCK, dtype=torch.float32, device=dev)
+        S2 = torch.empty(E, H // BLOCK, I // BLOCK, dtype=torch.float32, device=dev)
     S3 = torch.empty_like(S1)
-    S2 = torch.empty(E, H // BLOCK, I // BLOCK, dtype=torch.float32, device=dev)
     for e in range(E):
         for (wq, ws, shape) in ((W1q, S1, (I, H)), (W3q, S3, (I, H)), (W2q, S2, (H, I))):
             w = torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * 0.02
-            q, s = quantize_weight_blocks(w)
+            if w4:
+                q, s = quantize_weight_int4(w)
+                s = s.t()                                   # row scales, K-block-major
+            else:
+                q, s = quantize_weight_blocks(w)
             wq[e].copy_(q)
             ws[e].copy_(s)
     return MoeInputs(cfg, x, Wg, bias, token_ids, W1q, S1, W3q, S3, W2q, S2)
+
+
+def make_router_inputs(cfg: MoeConfig, device="cpu"):
+    """x, W_g and bias exactly as make_inputs draws them on `device` (they come first in its draw
+    order), without drawing the expert weights: (x [T, H] bf16, W_g [E, H] fp32, bias [E] fp32)."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed)
+    x = torch.randn(cfg.T, cfg.H, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    Wg = torch.randn(cfg.E, cfg.H, generator=g, device=dev, dtype=torch.float32) * 0.02
+    return x, Wg, _bias(cfg, g, dev)
 
 
 def interleave_w13(W1q: torch.Tensor, S1: torch.Tensor, W3q: torch.Tensor, S3: torch.Tensor):
@@ -183,6 +217,18 @@ def interleave_w13(W1q: torch.Tensor, S1: torch.Tensor, W3q: torch.Tensor, S3: t
     w = torch.stack((W1q.reshape(E, nb, BLOCK, H), W3q.reshape(E, nb, BLOCK, H)), dim=2)
     s = torch.stack((S1, S3), dim=2)
     return w.reshape(E, 2 * I, H).contiguous(), s.reshape(E, 2 * nb, H // BLOCK).contiguous()
+
+
+def interleave_w13_w4(W1q: torch.Tensor, S1: torch.Tensor, W3q: torch.Tensor, S3: torch.Tensor):
+    """interleave_w13 for 4-bit weights: the packed rows [E, I, H/2] alternate in 128-row blocks (W1 block
+    j, W3 block j) as for E4M3, and the K-block-major row scales [E, H/128, I] follow the same row order
+    along their last axis. Pure layout."""
+    E, I, Hp = W1q.shape
+    nb = I // BLOCK
+    w = torch.stack((W1q.reshape(E, nb, BLOCK, Hp), W3q.reshape(E, nb, BLOCK, Hp)), dim=2)
+    KB = S1.shape[1]
+    s = torch.stack((S1.reshape(E, KB, nb, BLOCK), S3.reshape(E, KB, nb, BLOCK)), dim=3)
+    return w.reshape(E, 2 * I, Hp).contiguous(), s.reshape(E, KB, 2 * I).contiguous()
 
 
 def capacity_rows_bound(cfg: MoeConfig, pad: int = BLOCK) -> int:

@@ -62,6 +62,9 @@ typedef enum { MOE_ROUTE_SOFTMAX_TOPK = 0, MOE_ROUTE_HASH = 1 } moe_routing_t;
 typedef enum { MOE_LAYOUT_CONTIGUOUS = 0, MOE_LAYOUT_MASKED = 1 } moe_layout_t;
 typedef enum { MOE_EPI_BF16 = 0, MOE_EPI_SWIGLU_FP8 = 1 } moe_epilogue_t;
 typedef enum { MOE_CONTIG_AUTO = 0, MOE_CONTIG_SINGLE = 1, MOE_CONTIG_PAIR = 2 } moe_contig_kernel_t;
+/* Expert weights: E4M3 with one fp32 scale per 128x128 block, or 4-bit levels with one fp32 scale per
+ * weight row per 128-wide K block (moe_grouped_gemm_w4; masked layout only). */
+typedef enum { MOE_WEIGHTS_FP8 = 0, MOE_WEIGHTS_W4 = 1 } moe_weights_t;
 
 /* Limits checked by every entry point. */
 #define MOE_MAX_EXPERTS 512
@@ -79,6 +82,7 @@ typedef struct {
     int cap_den;
     int layout;         /* moe_layout_t */
     int masked_max_m;   /* rows per expert in the masked layout (ignored when contiguous) */
+    int weights;        /* moe_weights_t: the expert weights' format (moe_forward) */
 } moe_config_t;
 
 /* Rows of the permuted buffers (Aq, As, Hq, Hs, O, row_src) for `cfg`:
@@ -190,8 +194,11 @@ moe_status_t moe_grouped_gemm_fp8(int layout, int E, int N, int K, const uint8_t
  *   layout      MOE_LAYOUT_MASKED only (MOE_ERR_UNSUPPORTED_SHAPE otherwise);
  *               A, As, group_info (masked_m), M_rows, epilogue, D and Ds as in
  *               moe_grouped_gemm_fp8
- *   B           [E, N, K/2] u8: two levels per byte, the even k in the low
- *               nibble, each a 4-bit two's-complement integer in -7..7
+ *   B           [E, N, K/2] u8: levels -7..7 as a sign and a 3-bit magnitude,
+ *               eight consecutive k per little-endian 32-bit word; level i
+ *               (i = 0..3) of a word has its magnitude in bits 4i..4i+2 and
+ *               its sign in bit 8i+7, level 4+i its magnitude in bits
+ *               16+4i..16+4i+2 and its sign in bit 8i+3
  *   Bs          [E, K/128, N] fp32 (K-block-major): the scale of weight row n
  *               for K block kb, max-abs / 7 of its 128 weights; a weight is
  *               level * scale
@@ -218,9 +225,14 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* O, const int32_t* 
 /*
  * The whole layer on one stream: route -> permute -> grouped GEMM with W13
  * (SwiGLU + FP8 requant epilogue) -> grouped GEMM with W2 (bf16) -> combine.
+ * cfg->weights = MOE_WEIGHTS_FP8:
  *   W13 [E, 2I, H] u8 with 128-row blocks alternating W1 block j, W3 block j
  *   S13 [E, 2I/128, H/128] fp32 in the same block order
  *   W2  [E, H, I] u8, S2 [E, H/128, I/128] fp32
+ * cfg->weights = MOE_WEIGHTS_W4 (masked layout only; MOE_ERR_UNSUPPORTED_SHAPE
+ * otherwise), the 4-bit format of moe_grouped_gemm_w4:
+ *   W13 [E, 2I, H/2] u8, rows in the same W1/W3 block alternation
+ *   S13 [E, H/128, 2I] fp32, W2 [E, H, I/2] u8, S2 [E, I/128, H] fp32
  *   y [T, H] bf16 out; topk_idx, topk_w, counts, slot_row as in the calls above
  *   ws  scratch of at least moe_workspace_size(cfg, 1) bytes, 256-byte aligned
  */
@@ -288,9 +300,8 @@ moe_status_t moe_balance_bias(int E, const int32_t* counts, int64_t* load, float
  *                      with an odd number of 128-row tiles computes its last
  *                      one on one CTA of a pair while the other idles. Needs N
  *                      a multiple of 256 (otherwise the single form runs).
- *   MOE_CONTIG_AUTO    (the default) pairs when the buffer holds at least 2.5
- *                      tiles of rows per expert on average (M_rows >= 320 E),
- *                      else single CTAs.
+ *   MOE_CONTIG_AUTO    (the default) the faster form as measured on this
+ *                      build's workloads: single CTAs.
  * Both forms compute the same products and the same fp32 promotion, in the
  * same order. Returns MOE_ERR_INVALID_ARG for any other value.
  */

@@ -88,7 +88,7 @@ def _declare(L):
     L.orc_combine.argtypes = [_i, _i, _i, _p, _p, _p, _p]
     L.orc_balance_bias.argtypes = [_i, _p, _p, _p, ctypes.c_float, _i]
     L.orc_grouped_gemm_w4.argtypes = [_i, _i, _i, _i, _p, _p, _p, _i, _p, _p, _i, _p, _p, _i]
-    L.orc_w4_decode.argtypes = [ctypes.c_uint8, _i]
+    L.orc_w4_decode.argtypes = [_p, _i]
     L.orc_w4_decode.restype = _i
 
 
@@ -211,9 +211,11 @@ def expert_rows(xq, xs, W1q, S1, W3q, S3, W2q, S2, nthreads: Optional[int] = Non
     return hq, hs, o
 
 
-def w4_decode(byte: int, high: bool) -> int:
-    """One 4-bit weight code (DeepSeek-V4 lecture page, 3.1): nibble `high` of `byte`, sign-extended."""
-    return int(lib().orc_w4_decode(byte, int(bool(high))))
+def w4_decode(row: np.ndarray, k: int) -> int:
+    """The 4-bit weight level of element k of a packed row (DeepSeek-V4 lecture page, 3.1): sign and 3-bit
+    magnitude, eight consecutive k per little-endian 32-bit word (moe_oracle.c, orc_w4_decode)."""
+    r = _c(row, np.uint8)
+    return int(lib().orc_w4_decode(_ptr(r), int(k)))
 
 
 def grouped_gemm(layout: int, E: int, N: int, K: int, A, As, group_info, M_rows: int, B, Bs,
@@ -301,14 +303,41 @@ def permute(cfg, x_bits, topk_idx, rows_cap: int, pad: int = GROUP):
     return d
 
 
-def expert_outputs_for_rows(inp, rows_by_expert, xq, xs, nthreads=None):
-    """{expert: (token list)} -> {expert: o bf16 [n, H]} through orc_expert_rows."""
+def expert_rows_w4(xq, xs, W1q, S1, W3q, S3, W2q, S2, nthreads: Optional[int] = None):
+    """The expert function with 4-bit weights (DeepSeek-V4 lecture page, 3.1) for n rows: the 4-bit grouped
+    GEMM (orc_grouped_gemm_w4) with W1/W3 rows alternating in 128-row blocks and the SwiGLU + 1x128
+    requantisation epilogue, then with W2 and the bf16 epilogue, one expert in the masked layout.
+    W1q, W3q [I, H/2] and W2q [H, I/2] packed levels; S1, S3 [H/128, I] and S2 [I/128, H] row scales
+    (K-block-major). Returns o bf16 bits [n, H]."""
+    xq = _c(xq, np.uint8)
+    n, H = xq.shape
+    I = W1q.shape[0]
+    M = max(32, -(-n // 32) * 32)
+    A = np.zeros((M, H), np.uint8)
+    A[:n] = xq
+    As = np.ones((1, H // GROUP, M), np.float32)
+    As[0, :, :n] = np.asarray(xs, np.float32).T
+    nb = I // GROUP
+    W13 = np.stack((np.asarray(W1q).reshape(nb, GROUP, -1), np.asarray(W3q).reshape(nb, GROUP, -1)),
+                   axis=1).reshape(2 * I, -1)
+    S13 = np.stack((np.asarray(S1).reshape(H // GROUP, nb, GROUP), np.asarray(S3).reshape(H // GROUP, nb, GROUP)),
+                   axis=2).reshape(H // GROUP, 2 * I)
+    gi = np.array([n], np.int32)
+    hq, hs = grouped_gemm(1, 1, 2 * I, H, A, As, gi, M, W13[None], S13[None], 1, nthreads, w4=True)
+    o, _ = grouped_gemm(1, 1, H, I, hq, hs, gi, M, np.asarray(W2q)[None], np.asarray(S2)[None], 0, nthreads,
+                        w4=True)
+    return o[:n]
+
+
+def expert_outputs_for_rows(inp, rows_by_expert, xq, xs, nthreads=None, w4: bool = False):
+    """{expert: (token list)} -> {expert: o bf16 [n, H]} through orc_expert_rows (E4M3 weights) or the
+    4-bit grouped GEMMs (w4)."""
     out = {}
+    fn = expert_rows_w4 if w4 else (lambda *a: expert_rows(*a)[2])
     for e, toks in rows_by_expert.items():
         toks = np.asarray(toks, dtype=np.int64)
-        _, _, o = expert_rows(xq[toks], xs[toks], inp["W1q"][e], inp["S1"][e], inp["W3q"][e], inp["S3"][e],
-                              inp["W2q"][e], inp["S2"][e], nthreads)
-        out[e] = o
+        out[e] = fn(xq[toks], xs[toks], inp["W1q"][e], inp["S1"][e], inp["W3q"][e], inp["S3"][e],
+                    inp["W2q"][e], inp["S2"][e], nthreads)
     return out
 
 
@@ -332,7 +361,7 @@ def forward(cfg, inp: dict, tokens: Optional[np.ndarray] = None, rows_cap: Optio
         for j in range(k):
             if d["slot_row"][t * k + j] >= 0:
                 by_e.setdefault(int(idx[t, j]), []).append(int(t))
-    outs = expert_outputs_for_rows(inp, by_e, d["xq"], d["xs"], nthreads)
+    outs = expert_outputs_for_rows(inp, by_e, d["xq"], d["xs"], nthreads, w4=getattr(cfg, "weights", "fp8") == "w4")
     H = inp["x"].shape[1]
     O = np.zeros((rows_cap, H), dtype=np.uint16)
     for e, toks in by_e.items():

@@ -291,11 +291,24 @@ static double dot_row(int K, const uint8_t* a, const float* a_s, const uint8_t* 
 }
 
 /* 4-bit weight codes ([P3] 3.1): the integer levels -7..7 of a block scaled by
- * its max-abs, round((w / max|w|) * (2^3 - 1)). Two codes per byte, the even k
- * in the low nibble, each a 4-bit two's-complement integer. */
-int orc_w4_decode(uint8_t byte, int high) {
-    int v = high ? (byte >> 4) : (byte & 15);
-    return v >= 8 ? v - 16 : v;
+ * its max-abs, round((w / max|w|) * (2^3 - 1)), stored as a sign and a 3-bit
+ * magnitude. A row holds K/8 little-endian 32-bit words, each with the levels
+ * of eight consecutive k (k = 8 q + i): the magnitude of level i (i = 0..3) in
+ * bits 4i..4i+2 and its sign in bit 8i+7; the magnitude of level 4+i in bits
+ * 16+4i..16+4i+2 and its sign in bit 8i+3. Returns the level of element k. */
+int orc_w4_decode(const uint8_t* row, int k) {
+    const uint8_t* b = row + 4 * (k / 8);
+    const uint32_t w = (uint32_t)b[0] | ((uint32_t)b[1] << 8) | ((uint32_t)b[2] << 16) | ((uint32_t)b[3] << 24);
+    const int i = k % 8;
+    int mag, neg;
+    if (i < 4) {
+        mag = (int)((w >> (4 * i)) & 7u);
+        neg = (int)((w >> (8 * i + 7)) & 1u);
+    } else {
+        mag = (int)((w >> (16 + 4 * (i - 4))) & 7u);
+        neg = (int)((w >> (8 * (i - 4) + 3)) & 1u);
+    }
+    return neg ? -mag : mag;
 }
 
 /* As dot_row, with a row of 4-bit weight codes and the row's K/128 scales
@@ -306,7 +319,7 @@ static double dot_row_w4(int K, const uint8_t* a, const float* a_s, const uint8_
     double acc = 0.0;
     int kk;
     for (kk = 0; kk < K; ++kk) {
-        float wd = (float)orc_w4_decode(w[kk >> 1], kk & 1) * w_s[(int64_t)(kk / GROUP) * ws_stride];
+        float wd = (float)orc_w4_decode(w, kk) * w_s[(int64_t)(kk / GROUP) * ws_stride];
         acc += (double)deq(a[kk], a_s[kk / GROUP]) * (double)wd;
     }
     return acc;

@@ -103,8 +103,11 @@ void orc_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const f
 void orc_grouped_gemm_w4(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                          const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs,
                          int epilogue, void* D, float* Ds, int nthreads);
-/* One 4-bit weight code: nibble `high` (0 = low) of `byte`, sign-extended. */
-int orc_w4_decode(uint8_t byte, int high);
+/* The 4-bit weight level (-7..7) of element k of a packed row: sign and 3-bit
+ * magnitude, eight consecutive k per little-endian 32-bit word; level i of a
+ * word (i = 0..3): magnitude in bits 4i..4i+2, sign in bit 8i+7; level 4+i:
+ * magnitude in bits 16+4i..16+4i+2, sign in bit 8i+3. */
+int orc_w4_decode(const uint8_t* row, int k);
 /* Combine: y[t,:] = sum_j [kept] w[t,j] * O[slot_row[t*k+j], :], fp64, -> bf16. */
 void orc_combine(int T, int k, int H, const int32_t* slot_row, const float* topk_w,
                  const uint16_t* O, uint16_t* y);

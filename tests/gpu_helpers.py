@@ -8,7 +8,7 @@ import torch
 import oracle
 from fp8_grouped_gemm_fp32_b200 import api
 from fp8_grouped_gemm_fp32_b200.build import build
-from fp8_grouped_gemm_fp32_b200.inputs import MoeConfig, MoeInputs, interleave_w13, make_inputs
+from fp8_grouped_gemm_fp32_b200.inputs import MoeConfig, MoeInputs, interleave_w13, interleave_w13_w4, make_inputs
 
 # Tolerances on bf16 outputs (the layer's stated bar): max_i |y_i - r_i| / max(|r_i|, rms(r))
 # and sum |y - r| / sum |r|. The denominator floor rms(r) keeps the element-wise ratio finite
@@ -82,7 +82,7 @@ def gpu_inputs(cfg: MoeConfig, T=None, on_device: bool = False) -> MoeInputs:
 def gpu_forward(cfg: MoeConfig, inp: MoeInputs) -> dict:
     c = api.Config.from_moe(cfg)
     dev = inp.x.device
-    W13, S13 = interleave_w13(inp.W1q, inp.S1, inp.W3q, inp.S3)
+    W13, S13 = (interleave_w13_w4 if cfg.weights == "w4" else interleave_w13)(inp.W1q, inp.S1, inp.W3q, inp.S3)
     T, k, H, E = cfg.T, cfg.k, cfg.H, cfg.E
     out = dict(
         y=torch.empty(T, H, dtype=torch.bfloat16, device=dev),

@@ -29,6 +29,8 @@ SMALL = {
     "hash_small": (MoeConfig("hash_small", T=96, H=256, E=16, I=128, k=1, routing="hash",
                              layout="masked", masked_max_m=96, seed=13), None),
     "one_expert": (MoeConfig("one_expert", T=200, H=256, E=1, I=256, k=1, bias="zero", seed=14), None),
+    "w4_masked": (MoeConfig("w4_masked", T=80, H=384, E=16, I=256, k=4, bias="uniform", layout="masked",
+                            masked_max_m=64, seed=15, weights="w4"), None),
 }
 
 
@@ -55,16 +57,18 @@ def test_layer_small(name):
 
 
 @pytest.mark.parametrize("name,form", [("page", api.CONTIG_AUTO), ("page", api.CONTIG_PAIR),
-                                       ("prefill", api.CONTIG_AUTO), ("decode", api.CONTIG_AUTO),
-                                       ("decode_hash", api.CONTIG_AUTO), ("skewed", api.CONTIG_AUTO)])
+                                       ("prefill", api.CONTIG_AUTO), ("prefill", api.CONTIG_PAIR),
+                                       ("decode", api.CONTIG_AUTO),
+                                       ("decode_hash", api.CONTIG_AUTO), ("skewed", api.CONTIG_AUTO),
+                                       ("decode_w4", api.CONTIG_AUTO)])
 def test_layer_full_size_tile_covering(name, form):
     # Every workload at full size, in the launch configuration the benchmark times: routing, counts and the
     # slot -> row map (permutation and dropped set) on every token, and y on a set of tokens whose kept rows
     # reach every tile the two grouped GEMMs schedule (each 128-row M tile of the contiguous layout, each
     # 32-token slice of an expert's block in the masked layout), chosen from the oracle's own dispatch.
-    # The default kernel choice runs on every workload (CTA pairs for prefill and skewed, single CTAs for
-    # page); the page workload also runs with CTA pairs forced, where most experts fill one or two 128-row
-    # tiles, so many pair tiles are lone (one CTA of the pair idle).
+    # The default kernel choice runs on every workload; the page workload also runs with CTA pairs forced,
+    # where most experts fill one or two 128-row tiles, so many pair tiles are lone (one CTA of the pair
+    # idle), and prefill with CTA pairs forced, where most experts fill two or three.
     ensure_lib()
     cfg = CONFIGS[name]
     inp = gpu_inputs(cfg, on_device=True)

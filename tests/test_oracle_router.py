@@ -137,3 +137,17 @@ def test_hash_golden_and_histogram():
     for t in tids.tolist():
         tally[((t * 2654435761) & 0xFFFFFFFF) % 256] += 1
     assert np.array_equal(np.bincount(idx[:, 0], minlength=256), tally)
+
+
+def test_fixed_fp32_order_selects_as_exact_arithmetic_on_the_page_workload():
+    # the fixed fp32 logit order (a reading: the pages give none) against fp64 logits on the page workload's
+    # router inputs: no token's top-k set differs, and any token whose top-k could differ has a margin within
+    # the fp32 error bound of the canonical order
+    from fp8_grouped_gemm_fp32_b200.inputs import CONFIGS, make_router_inputs
+    from oracle.router_fp64_diagnostic import diagnose
+    cfg = CONFIGS["page"]
+    x, Wg, bias = make_router_inputs(cfg)
+    d = diagnose(cfg, x.view(torch.int16).numpy().view(np.uint16), Wg.numpy(), bias.numpy())
+    assert d["differ"] == 0
+    assert d["differ_within_near"]
+    assert 0 < d["near_ties"] < 0.01 * cfg.T

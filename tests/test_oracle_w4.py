@@ -46,11 +46,20 @@ def golden_cases():
 
 
 def _unpack(codes):
-    """uint8 [..., K/2] -> int levels [..., K]: low nibble first, 4-bit two's complement."""
-    c = codes.astype(np.int16)
-    lo, hi = c & 15, c >> 4
-    lev = np.stack([lo, hi], axis=-1).reshape(*codes.shape[:-1], codes.shape[-1] * 2)
-    return np.where(lev >= 8, lev - 16, lev)
+    """uint8 [..., K/2] -> int levels [..., K]: per little-endian 32-bit word, eight consecutive k;
+    level i < 4: magnitude bits 4i..4i+2, sign bit 8i+7; level 4+i: magnitude bits 16+4i..16+4i+2,
+    sign bit 8i+3."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    w = c.reshape(*c.shape[:-1], c.shape[-1] // 4, 4).astype(np.int64)
+    word = w[..., 0] | (w[..., 1] << 8) | (w[..., 2] << 16) | (w[..., 3] << 24)
+    lev = []
+    for i in range(8):
+        if i < 4:
+            mag, neg = (word >> (4 * i)) & 7, (word >> (8 * i + 7)) & 1
+        else:
+            mag, neg = (word >> (16 + 4 * (i - 4))) & 7, (word >> (8 * (i - 4) + 3)) & 1
+        lev.append(np.where(neg == 1, -mag, mag))
+    return np.stack(lev, axis=-1).reshape(*c.shape[:-1], c.shape[-1] * 2)
 
 
 def test_quantiser_golden_blocks():
@@ -72,10 +81,22 @@ def test_quantiser_golden_blocks():
         assert scale.numpy()[0, 0] == np.float32(c["scale"]), c["name"]
 
 
-def test_every_code_decodes_as_twos_complement():
-    for b in range(256):
-        assert oracle.w4_decode(b, False) == ((b & 15) ^ 8) - 8
-        assert oracle.w4_decode(b, True) == ((b >> 4) ^ 8) - 8
+def test_every_level_at_every_position_decodes():
+    # a word holding one level at one of its eight places, every level -7..7 at every place, and words of
+    # random levels: the oracle's decode returns exactly the levels placed
+    for i in range(8):
+        for L in range(-7, 8):
+            word = abs(L) << (4 * i if i < 4 else 16 + 4 * (i - 4))
+            if L < 0:
+                word |= 1 << (8 * i + 7 if i < 4 else 8 * (i - 4) + 3)
+            row = np.frombuffer(int(word).to_bytes(4, "little"), np.uint8)
+            assert [oracle.w4_decode(row, k) for k in range(8)] == [L if k == i else 0 for k in range(8)], (i, L)
+    rng = np.random.default_rng(3)
+    lev = rng.integers(-7, 8, (16, 128))
+    codes, _ = quantize_weight_int4(torch.from_numpy(lev.astype(np.float32) * 7 / np.where(
+        np.abs(lev).reshape(16, 1, 128).max(-1) > 0, np.abs(lev).reshape(16, 1, 128).max(-1), 1).repeat(128, 1)))
+    got = np.array([[oracle.w4_decode(codes.numpy()[r], k) for k in range(128)] for r in range(16)])
+    assert np.array_equal(got, _unpack(codes.numpy()))
 
 
 def test_level_grids_round_trip_and_error_bound():
@@ -178,3 +199,34 @@ def test_w4_grouped_gemm_equals_dense_fp64(layout):
         assert np.all(np.abs(Dq[rows].astype(np.int32) - hq.astype(np.int32))[~same] == 1)
         ds = Ds[:, rows].T if layout == 0 else Ds[e][:, :len(rows)].T
         assert np.allclose(ds, hs, rtol=1e-6, atol=0)
+
+
+def test_w4_expert_rows_equal_fp64_expert_function():
+    # E_i(x) = W2 (silu(W1 x) * W3 x) with 4-bit weights, h requantised per 1x128 group and o rounded to
+    # bf16: the oracle's composition of its 4-bit grouped GEMMs against numpy fp64 matmuls over weights
+    # unpacked and dequantised here (a gate/up mix-up, a scale transposed or the wrong interleave fails it)
+    rng = np.random.default_rng(11)
+    n, H, I = 37, 256, 384
+    x = rng.standard_normal((n, H)).astype(np.float32)
+    xq, xs = oracle.quant_rows(x)
+    wts = {}
+    for name, (N, K) in (("W1", (I, H)), ("W3", (I, H)), ("W2", (H, I))):
+        q, s = quantize_weight_int4(torch.from_numpy(rng.standard_normal((N, K)).astype(np.float32) * 0.02))
+        wts[name] = (q.numpy(), np.ascontiguousarray(s.numpy().T))        # scales K-block-major [K/128, N]
+    o = oracle.expert_rows_w4(xq, xs, wts["W1"][0], wts["W1"][1], wts["W3"][0], wts["W3"][1], wts["W2"][0],
+                              wts["W2"][1])
+
+    def deq_w(q, s_kb_major):
+        return _unpack(q).astype(np.float64) * np.repeat(s_kb_major.T.astype(np.float64), 128, axis=1)
+
+    def deq_rows(codes, scales):
+        return oracle.e4m3_decode_array(codes) * np.repeat(scales.astype(np.float64), 128, axis=1)
+
+    xd = deq_rows(xq, xs).astype(np.float32).astype(np.float64)       # dequantised values are fp32
+    a = xd @ deq_w(*wts["W1"]).astype(np.float32).astype(np.float64).T
+    b = xd @ deq_w(*wts["W3"]).astype(np.float32).astype(np.float64).T
+    h = (a / (1.0 + np.exp(-a)) * b).astype(np.float32)
+    hq, hs = oracle.quant_rows(h)
+    hd = deq_rows(hq, hs).astype(np.float32).astype(np.float64)
+    ref = oracle.f64_to_bf16_bits(hd @ deq_w(*wts["W2"]).astype(np.float32).astype(np.float64).T)
+    assert np.array_equal(o, ref)
