@@ -198,6 +198,7 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* Wg, 
     if (st != MOE_OK) return st;
     DeviceInfo* dev;
     if ((st = device_info(&dev)) != MOE_OK) return st;
+    if (cfg->T == 0) return MOE_OK;                       // no tokens: nothing is read or written
     if (!ptr_ok(topk_idx) || !ptr_ok(topk_w)) return MOE_ERR_INVALID_ARG;
     if (cfg->routing == MOE_ROUTE_HASH) {
         if (!ptr_ok(token_ids)) return MOE_ERR_INVALID_ARG;
@@ -285,8 +286,8 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* O, const int32_t* 
     if (st != MOE_OK) return st;
     DeviceInfo* dev;
     if ((st = device_info(&dev)) != MOE_OK) return st;
+    if (cfg->T == 0) return MOE_OK;                       // no tokens: nothing is read or written
     if (!ptr_ok(O) || !ptr_ok(slot_row) || !ptr_ok(topk_w) || !ptr_ok(y)) return MOE_ERR_INVALID_ARG;
-    if (cfg->T == 0) return MOE_OK;
     return cuda_status(launch_combine(static_cast<const uint16_t*>(O), slot_row, topk_w, cfg->T, cfg->k, cfg->H,
                                       static_cast<uint16_t*>(y), static_cast<cudaStream_t>(stream)));
 }

@@ -271,9 +271,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {
     return r;
 }
 
-// Arrives (release, cluster scope) on an mbarrier given by its shared::cluster address.
+// Arrives on an mbarrier given by its shared::cluster address (possibly in the peer CTA). Default
+// semantics (release at CTA scope): a cluster-scope release would fence all of the thread's memory
+// operations on every call; what the arrival orders here are tensor-memory reads, which
+// tcgen05.fence::before_thread_sync already orders before it.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {

@@ -199,10 +199,11 @@ moe_status_t moe_ep_count(const moe_config_t* cfg, const int32_t* topk_idx, int3
     int num_sms = 0;
     int* status = nullptr;
     if ((st = current_device(&num_sms, &status)) != MOE_OK) return st;
-    if (!ptr16(topk_idx) || !ptr16(counts) || !ptr16(ws)) return MOE_ERR_INVALID_ARG;
-    if (ws_bytes < ep_scratch_bytes(cfg->T, cfg->E)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!ptr16(counts)) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cfg->T == 0) return cuda_status(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->E, s));
+    if (cfg->T == 0) return cuda_status(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->E, s));   // all zero
+    if (!ptr16(topk_idx) || !ptr16(ws)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < ep_scratch_bytes(cfg->T, cfg->E)) return MOE_ERR_WORKSPACE_TOO_SMALL;
     return cuda_status(launch_ep_count(topk_idx, cfg->T, cfg->k, cfg->E, counts, ws, status, s));
 }
 
@@ -214,10 +215,10 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const void* x, const int32
     int num_sms = 0;
     int* status = nullptr;
     if ((st = current_device(&num_sms, &status)) != MOE_OK) return st;
+    if (cfg->T == 0) return MOE_OK;                       // no tokens: no send rows, no slots
     if (!ptr16(x) || !ptr16(topk_idx) || !ptr16(plan_dev) || !ptr16(slot_row) || !ptr16(ws)) return MOE_ERR_INVALID_ARG;
     if (send && !ptr16(send)) return MOE_ERR_INVALID_ARG;
     if (ws_bytes < ep_scratch_bytes(cfg->T, cfg->E)) return MOE_ERR_WORKSPACE_TOO_SMALL;
-    if (cfg->T == 0) return MOE_OK;
     const int32_t* kept_mine = reinterpret_cast<const int32_t*>(reinterpret_cast<const uint8_t*>(plan_dev) +
                                                                 offsetof(moe_ep_plan_t, kept_mine));
     return cuda_status(launch_ep_dispatch(static_cast<const uint16_t*>(x), topk_idx, cfg->T, cfg->H, cfg->k, cfg->E,

@@ -624,6 +624,9 @@ struct SmemM {
     alignas(1024) uint8_t wp[kStages][kWP];                     // packed levels (W4), 64 bytes per row, 64-byte swizzle
     float hs[EPI == 1 ? 2 : 1][EPI == 1 ? kBT : 1][kBM];       // SwiGLU output staged for the requant
     float sa[kSaSlots][kBT];                                    // activation scales of one K block, 32 tokens
+    // W4: the tile's weight-row scales of the same K block (128 rows, or the 256 gate and up rows), copied
+    // with the activation scales and released with them, so the promotion warps read no global memory
+    float wrs[W4 ? kSaSlots : 1][W4 ? kW / kBK : 1];
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t afull[kA];                                         // W4: A slot written by the converter warps
@@ -759,9 +762,13 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     // the token tile's 32 activation scales of this K block, into the scale ring
                     const int j = it % S::kSaSlots;
                     if (!mbar_wait(&sm.sempty[j], ((it / S::kSaSlots) & 1) ^ 1, wait_ns)) { fail(); break; }
-                    mbar_arrive_expect_tx(&sm.sfull[j], kBT * sizeof(float));
+                    constexpr uint32_t kWrsBytes = W4 ? static_cast<uint32_t>(sizeof(sm.wrs[0])) : 0u;
+                    mbar_arrive_expect_tx(&sm.sfull[j], kBT * sizeof(float) + kWrsBytes);
                     bulk_load(sm.sa[j], As + (static_cast<int64_t>(e) * KB + kb) * Mmax + tt * kBT, kBT * sizeof(float),
                               &sm.sfull[j]);
+                    if constexpr (W4)       // row scales [E, K/128, N]: the tile's rows are consecutive
+                        bulk_load(sm.wrs[j], Bs + (static_cast<int64_t>(e) * KB + kb) * N + (wrow - e * N), kWrsBytes,
+                                  &sm.sfull[j]);
                 }
             }
         }
@@ -887,13 +894,6 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const float wta[4] = {wa[0], wa[1], wa[2], wa[3]};
             const float wtb[4] = {wb[0], wb[1], wb[2], wb[3]};
             if constexpr (!W4) load_w(tile + gridDim.x);
-            // W4: this thread's weight row(s) carry their own scale per K block, [E, K/128, N]
-            const float* wsr = Bs + static_cast<int64_t>(e) * KB * N + (EPI == 1 ? 2 * nb : nb) * kBM + r;
-            float nsa = 0.0f, nsb = 0.0f;
-            if constexpr (W4) {
-                nsa = wsr[0];
-                if (EPI == 1) nsb = wsr[kBM];
-            }
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb, ++kbt) {
                 const int buf = kbt % S::kBufs;
@@ -907,17 +907,14 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     const float4 v4 = *reinterpret_cast<const float4*>(&sm.sa[j][cof + 4 * i]);
                     sa[4 * i] = v4.x; sa[4 * i + 1] = v4.y; sa[4 * i + 2] = v4.z; sa[4 * i + 3] = v4.w;
                 }
+                float swa, swb;
+                if constexpr (W4) {            // this thread's weight row (and its up row) scale for the K block
+                    swa = sm.wrs[j][r];
+                    swb = EPI == 1 ? sm.wrs[j][kBM + r] : 0.0f;
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.sempty[j]);
-                float swa, swb;
-                if constexpr (W4) {
-                    swa = nsa;
-                    swb = nsb;
-                    if (kb + 1 < KB) {
-                        nsa = wsr[static_cast<int64_t>(kb + 1) * N];
-                        if (EPI == 1) nsb = wsr[static_cast<int64_t>(kb + 1) * N + kBM];
-                    }
-                } else {
+                if constexpr (!W4) {
                     const int wi = kb >> 5;
                     swa = __shfl_sync(0xffffffffu, wi == 0 ? wta[0] : wi == 1 ? wta[1] : wi == 2 ? wta[2] : wta[3],
                                       kb & 31);

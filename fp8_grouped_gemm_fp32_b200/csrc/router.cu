@@ -63,21 +63,32 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     // The stage ring runs on across tiles: global stage g = (the CTA's i-th tile) * nst + stage in tile.
     const int ET = (E + C::EC - 1) / C::EC;
     const int tiles = ((T + C::TT - 1) / C::TT) * ET;
-    const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int64_t stages_total = static_cast<int64_t>(my_tiles) * nst;
+    const int my_tiles = static_cast<int>(blockIdx.x) < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const uint32_t stages_total = static_cast<uint32_t>(my_tiles) * nst;
 
     auto fail = [&]() {
         set_status(status, kStatusTimeout);
         *abort_flag = 1;
     };
-    auto issue = [&](int64_t g) {      // global stage g into slot g % kStages
+    // Stages are issued strictly in order (only thread 0 issues): the next one's tile (the CTA's pf_it-th)
+    // and stage within it are kept as running counters, so issuing costs no division by the stage count.
+    int pf_it = 0, pf_st = 0, pf_t0 = 0, pf_e0 = 0;
+    auto pf_tile = [&]() {
+        const int tile = blockIdx.x + pf_it * gridDim.x;
+        pf_t0 = (tile / ET) * C::TT;
+        pf_e0 = (tile % ET) * C::EC;
+    };
+    auto issue = [&](uint32_t g) {      // global stage g (the next in order) into slot g % kStages
         const int s = static_cast<int>(g % C::kStages);
-        const int tile = blockIdx.x + static_cast<int>(g / nst) * gridDim.x;
-        const int st = static_cast<int>(g % nst);
         uint8_t* stage = smem + s * C::kStageBytes;
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-        tma_load_2d(stage, &tmX, &full[s], st * kRouterHS, (tile / ET) * C::TT);
-        tma_load_2d(stage + C::kXBytes, &tmW, &full[s], st * kRouterHS, (tile % ET) * C::EC);
+        tma_load_2d(stage, &tmX, &full[s], pf_st * kRouterHS, pf_t0);
+        tma_load_2d(stage + C::kXBytes, &tmW, &full[s], pf_st * kRouterHS, pf_e0);
+        if (++pf_st == nst) {
+            pf_st = 0;
+            ++pf_it;
+            pf_tile();
+        }
     };
     if (producer) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -88,16 +99,17 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         fence_mbar_init();
         prefetch_tensormap(&tmX);
         prefetch_tensormap(&tmW);
-        for (int64_t g = 0; g < C::kStages && g < stages_total; ++g) issue(g);
+        pf_tile();
+        for (uint32_t g = 0; g < C::kStages && g < stages_total; ++g) issue(g);
     }
     __syncthreads();
 
     if (DP && warp < 0) {
         // dedicated producer: refill each slot as soon as every compute warp has finished with it
         if (producer)
-            for (int64_t g = C::kStages; g < stages_total && !*abort_flag; ++g) {
-                const int64_t u = g / C::kStages - 1;
-                if (!mbar_wait(&empty[g % C::kStages], static_cast<uint32_t>(u & 1), wait_ns)) { fail(); break; }
+            for (uint32_t g = C::kStages; g < stages_total && !*abort_flag; ++g) {
+                const uint32_t u = g / C::kStages - 1;
+                if (!mbar_wait(&empty[g % C::kStages], u & 1, wait_ns)) { fail(); break; }
                 issue(g);
             }
         __syncthreads();
@@ -108,25 +120,28 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         return;
     }
     bool ok = true;
-    int64_t g = 0;
+    uint32_t g = 0;
     for (int it = 0; it < my_tiles && ok; ++it) {
     const int tile = blockIdx.x + it * gridDim.x;
     const int t_base = (tile / ET) * C::TT, e_base = (tile % ET) * C::EC;
-    float acc[TR][ER];
+    // acc2[p][q] holds the chains of tokens 2p and 2p + 1 with expert q: one packed fp32x2 multiply-add
+    // advances both (each half rounds exactly as a scalar fused multiply-add) for half the issue slots
+    static_assert(TR % 2 == 0, "tokens are paired");
+    float2 acc2[TR / 2][ER];
 #pragma unroll
-    for (int i = 0; i < TR; ++i)
+    for (int i = 0; i < TR / 2; ++i)
 #pragma unroll
-        for (int q = 0; q < ER; ++q) acc[i][q] = 0.0f;
+        for (int q = 0; q < ER; ++q) acc2[i][q] = make_float2(0.0f, 0.0f);
     for (int st = 0; st < nst; ++st, ++g) {
         // the slot of stage g - 1 takes stage g - 1 + kStages once every warp has finished with it
         if (!DP && producer && g > 0 && g - 1 + C::kStages < stages_total) {
-            if (!mbar_wait(&empty[(g - 1) % C::kStages], static_cast<uint32_t>(((g - 1) / C::kStages) & 1), wait_ns))
+            if (!mbar_wait(&empty[(g - 1) % C::kStages], ((g - 1) / C::kStages) & 1, wait_ns))
                 fail();
             else
                 issue(g - 1 + C::kStages);
         }
         const int s = static_cast<int>(g % C::kStages);
-        if (*abort_flag || !mbar_wait(&full[s], static_cast<uint32_t>((g / C::kStages) & 1), wait_ns)) {
+        if (*abort_flag || !mbar_wait(&full[s], (g / C::kStages) & 1, wait_ns)) {
             fail();
             ok = false;
             break;
@@ -138,17 +153,20 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 #pragma unroll
         for (int q = 0; q < ER; ++q) wv[q] = *reinterpret_cast<const float4*>(ws + q * kRouterHS);
 #pragma unroll
-        for (int i = 0; i < TR; ++i) {
-            const uint2 xr = *reinterpret_cast<const uint2*>(xs + i * kRouterHS);
-            const float x0 = __uint_as_float(xr.x << 16), x1 = __uint_as_float(xr.x & 0xffff0000u);
-            const float x2 = __uint_as_float(xr.y << 16), x3 = __uint_as_float(xr.y & 0xffff0000u);
+        for (int i = 0; i < TR / 2; ++i) {
+            const uint2 xa = *reinterpret_cast<const uint2*>(xs + (2 * i) * kRouterHS);
+            const uint2 xb = *reinterpret_cast<const uint2*>(xs + (2 * i + 1) * kRouterHS);
+            const float2 x0 = make_float2(__uint_as_float(xa.x << 16), __uint_as_float(xb.x << 16));
+            const float2 x1 = make_float2(__uint_as_float(xa.x & 0xffff0000u), __uint_as_float(xb.x & 0xffff0000u));
+            const float2 x2 = make_float2(__uint_as_float(xa.y << 16), __uint_as_float(xb.y << 16));
+            const float2 x3 = make_float2(__uint_as_float(xa.y & 0xffff0000u), __uint_as_float(xb.y & 0xffff0000u));
             // lane j's chain for (token, expert) runs over h = 4j, 4j+1, 4j+2, 4j+3 of this block in order
 #pragma unroll
             for (int q = 0; q < ER; ++q) {
-                acc[i][q] = fmaf(x0, wv[q].x, acc[i][q]);
-                acc[i][q] = fmaf(x1, wv[q].y, acc[i][q]);
-                acc[i][q] = fmaf(x2, wv[q].z, acc[i][q]);
-                acc[i][q] = fmaf(x3, wv[q].w, acc[i][q]);
+                acc2[i][q] = __ffma2_rn(x0, make_float2(wv[q].x, wv[q].x), acc2[i][q]);
+                acc2[i][q] = __ffma2_rn(x1, make_float2(wv[q].y, wv[q].y), acc2[i][q]);
+                acc2[i][q] = __ffma2_rn(x2, make_float2(wv[q].z, wv[q].z), acc2[i][q]);
+                acc2[i][q] = __ffma2_rn(x3, make_float2(wv[q].w, wv[q].w), acc2[i][q]);
             }
         }
         __syncwarp();
@@ -163,7 +181,7 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         // TR * ER / 32 finished logits.
         constexpr int NV = TR * ER;
         static_assert(NV % 32 == 0, "the register tile must spread evenly over the lanes");
-        float* v = &acc[0][0];
+        float* v = &acc2[0][0].x;             // value n: token 2 (n / (2 ER)) + (n & 1), expert (n / 2) % ER
         int base = 0;
 #pragma unroll
         for (int lvl = 0; lvl < 5; ++lvl) {
@@ -184,7 +202,7 @@ router_logits_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 #pragma unroll
         for (int m = 0; m < NV / 32; ++m) {
             const int n = base + m;
-            const int t = t_base + wt * TR + n / ER, e = e_base + we * ER + n % ER;
+            const int t = t_base + wt * TR + 2 * (n / (2 * ER)) + (n & 1), e = e_base + we * ER + (n >> 1) % ER;
             if (t < T && e < E) logits[static_cast<int64_t>(t) * E + e] = bias ? v[m] + bias[e] : v[m];
         }
     }

@@ -72,7 +72,8 @@ typedef enum { MOE_WEIGHTS_FP8 = 0, MOE_WEIGHTS_W4 = 1 } moe_weights_t;
 #define MOE_TILE_M 128
 
 typedef struct {
-    int T;              /* tokens (0 allowed: nothing is launched) */
+    int T;              /* tokens (0 allowed: nothing is launched and the per-token buffers may be
+                           empty; moe_ep_count still zeroes its counts) */
     int H;              /* hidden size, multiple of 128 */
     int E;              /* experts, 1..MOE_MAX_EXPERTS */
     int I;              /* expert intermediate size, multiple of 128 */
