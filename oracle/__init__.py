@@ -90,6 +90,7 @@ def _declare(L):
     L.orc_grouped_gemm_w4.argtypes = [_i, _i, _i, _i, _p, _p, _p, _i, _p, _p, _i, _p, _p, _i]
     L.orc_w4_decode.argtypes = [_p, _i]
     L.orc_w4_decode.restype = _i
+    L.orc_quant_group.argtypes = [_i64, _p, _p, _p]
 
 
 def _ptr(a: Optional[np.ndarray]):
@@ -385,3 +386,176 @@ def moe_inputs_to_numpy(inp) -> dict:
         W1q=inp.W1q.detach().cpu().numpy(), S1=inp.S1.detach().cpu().numpy(),
         W3q=inp.W3q.detach().cpu().numpy(), S3=inp.S3.detach().cpu().numpy(),
         W2q=inp.W2q.detach().cpu().numpy(), S2=inp.S2.detach().cpu().numpy())
+
+
+# ---------------------------------------------------------------- backward pass
+# The layer's backward (TP-MoE page, 4.1 step 5: gradients go back along the dispatch path and the gate
+# network is updated too). The pages fix no precision for it; the readings this oracle follows:
+#  * the quantisation steps of the forward pass count as the identity (their gradient passes straight
+#    through), and top-k selection, capacity and routing are held fixed;
+#  * every operand of a backward grouped GEMM is FP8 with fp32 scales, like the forward's: a gradient
+#    operand in 1x128 groups along the contraction, the other operand of a weight-gradient GEMM in
+#    128x128 blocks (the forward's weight granularity); sums in fp64; GEMM outputs bf16 (RNE);
+#  * intermediates stored between steps: dO = w * dy in fp32, then FP8; dh, a, b and g in bf16.
+def quant_group(v: np.ndarray):
+    """One scale for all of v: (codes like v's shape, scale)."""
+    v = _c(v, np.float32)
+    q = np.empty(v.shape, dtype=np.uint8)
+    s = np.empty(1, dtype=np.float32)
+    lib().orc_quant_group(v.size, _ptr(v), _ptr(q), _ptr(s))
+    return q, float(s[0])
+
+
+def tile_transpose_quant(V: np.ndarray, offsets: np.ndarray, kept: np.ndarray, mode: str):
+    """The weight-gradient operand of one activation-like matrix V [rows, C] (fp32) in the contiguous
+    grouped layout (expert e's rows at offsets[e] .. offsets[e] + kept[e]; other rows count as 0): for
+    every 128-row tile m of that layout, the transposed block V[128 m : 128 m + 128]^T [C, 128]
+    quantised. mode "row": each of the C rows of 128 values one 1x128 group (scales [tiles, C]);
+    mode "block": each 128 x 128 block one scale (scales [tiles, C / 128]). Returns codes
+    [tiles, C, 128], scales."""
+    tiles = int(offsets[-1]) // GROUP
+    C = V.shape[1]
+    W = np.zeros((tiles * GROUP, C), np.float32)
+    for e in range(len(kept)):
+        a, n = int(offsets[e]), int(kept[e])
+        W[a:a + n] = V[a:a + n]
+    Tt = np.ascontiguousarray(W.reshape(tiles, GROUP, C).transpose(0, 2, 1))
+    if mode == "row":
+        q, s = quant_rows(Tt.reshape(tiles * C, GROUP))
+        return q.reshape(tiles, C, GROUP), s.reshape(tiles, C)
+    q = np.empty((tiles, C, GROUP), np.uint8)
+    s = np.empty((tiles, C // GROUP), np.float32)
+    for m in range(tiles):
+        for cb in range(C // GROUP):
+            q[m, cb * GROUP:(cb + 1) * GROUP], s[m, cb] = quant_group(Tt[m, cb * GROUP:(cb + 1) * GROUP])
+    return q, s
+
+
+def _deq_tiles(q, s):
+    """codes [tiles, C, 128] with scales [tiles, C] or [tiles, C/128] -> fp32 values."""
+    v = e4m3_decode_array(q).astype(np.float32)
+    if s.shape[1] == q.shape[1]:
+        return (v * s[:, :, None]).astype(np.float32)
+    return (v * np.repeat(s, GROUP, axis=1)[:, :, None]).astype(np.float32)
+
+
+def swiglu_backward(a: np.ndarray, b: np.ndarray, dh: np.ndarray):
+    """h = silu(a) * b: (da, db) in fp64 from a, b, dh (any float arrays)."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    dh = np.asarray(dh, np.float64)
+    sg = 1.0 / (1.0 + np.exp(-a))
+    return dh * b * sg * (1.0 + a * (1.0 - sg)), dh * a * sg
+
+
+def router_backward(w: np.ndarray, dw: np.ndarray):
+    """w_j = exp(l_j - m) / sum_{top-k} exp(l_i - m): dl_j = w_j (dw_j - sum_i w_i dw_i), fp64."""
+    w = np.asarray(w, np.float64)
+    dw = np.asarray(dw, np.float64)
+    return w * (dw - np.sum(w * dw, axis=1, keepdims=True))
+
+
+def backward(cfg, inp: dict, dy_bits: np.ndarray, nthreads=None):
+    """The layer's backward for a gradient dy [T, H] (bf16 bits) of its output. `inp` as for forward.
+    Returns dx [T, H] (bf16 bits), dWg [E, H] and db [E] (fp32), dW13 [E, 2I, H] (bf16 bits; rows in
+    the W1/W3 128-row block alternation of the forward's up operand) and dW2 [E, H, I] (bf16 bits),
+    with the intermediates."""
+    f = forward(cfg, inp, nthreads=nthreads)
+    idx, w, slot_row = f["topk_idx"], f["topk_w"], f["slot_row"]
+    offsets, kept, row_src = f["offsets"], f["kept"], f["row_src"]
+    T, k = idx.shape
+    H = inp["x"].shape[1]
+    E = cfg.E
+    I = inp["W1q"][0].shape[0]
+    G = H // GROUP
+    rows_cap = row_src.shape[0]
+    x32 = bf16_bits_to_f32(inp["x"])
+    dy = bf16_bits_to_f32(dy_bits)
+    # per-row data of the forward in its contiguous layout: x codes/scales, h codes/scales, o
+    Aq = f["Aq"]
+    As = f["As"]                                   # [G][rows_cap]
+    hq = np.zeros((rows_cap, I), np.uint8)
+    hs = np.ones((rows_cap, I // GROUP), np.float32)
+    O = np.zeros((rows_cap, H), np.uint16)
+    for e in range(E):
+        a0, n = int(offsets[e]), int(kept[e])
+        if n == 0:
+            continue
+        toks = row_src[a0:a0 + n] // k
+        q_, s_, o_ = expert_rows(f["xq"][toks], f["xs"][toks], inp["W1q"][e], inp["S1"][e], inp["W3q"][e],
+                                 inp["S3"][e], inp["W2q"][e], inp["S2"][e], nthreads)
+        hq[a0:a0 + n], hs[a0:a0 + n], O[a0:a0 + n] = q_, s_, o_
+    # router: dw, dl, the gate's gradients and the gate's share of dx
+    Of = bf16_bits_to_f32(O).astype(np.float64)
+    dw = np.zeros((T, k), np.float64)
+    for s in range(T * k):
+        if slot_row[s] >= 0:
+            dw[s // k, s % k] = np.dot(dy[s // k].astype(np.float64), Of[slot_row[s]])
+    dw = dw.astype(np.float32)
+    dl = router_backward(w, dw).astype(np.float32)
+    dWg = np.zeros((E, H), np.float64)
+    db = np.zeros(E, np.float64)
+    Wg = np.asarray(inp["Wg"], np.float64)
+    dx_router = np.zeros((T, H), np.float64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            dWg[e] += float(dl[t, j]) * x32[t].astype(np.float64)
+            db[e] += float(dl[t, j])
+            dx_router[t] += float(dl[t, j]) * Wg[e]
+    # dO = w * dy (fp32) on kept rows, 1x128 FP8 along H
+    dO = np.zeros((rows_cap, H), np.float32)
+    for s in range(T * k):
+        r = slot_row[s]
+        if r >= 0:
+            dO[r] = np.float32(w[s // k, s % k]) * dy[s // k]
+    dOq, dOs = quant_rows(dO)
+    # transposed weights (layout only): W2^T [E, I, H] with S2^T, W13^T [E, H, 2I] with S13^T
+    W13 = np.stack([np.stack((np.asarray(inp["W1q"][e]).reshape(I // GROUP, GROUP, H),
+                              np.asarray(inp["W3q"][e]).reshape(I // GROUP, GROUP, H)), axis=1).reshape(2 * I, H)
+                    for e in range(E)])
+    S13 = np.stack([np.stack((np.asarray(inp["S1"][e]), np.asarray(inp["S3"][e])), axis=1).reshape(2 * I // GROUP, G)
+                    for e in range(E)])
+    W2 = np.stack([np.asarray(inp["W2q"][e]) for e in range(E)])
+    S2 = np.stack([np.asarray(inp["S2"][e]) for e in range(E)])
+    W2T, S2T = np.ascontiguousarray(W2.transpose(0, 2, 1)), np.ascontiguousarray(S2.transpose(0, 2, 1))
+    W13T, S13T = np.ascontiguousarray(W13.transpose(0, 2, 1)), np.ascontiguousarray(S13.transpose(0, 2, 1))
+    # dh = dO W2 (bf16), a|b recomputed (bf16), g = SwiGLU backward (bf16), dx rows = g W13 (bf16)
+    dh, _ = grouped_gemm(0, E, I, H, dOq, np.ascontiguousarray(dOs.T), offsets, rows_cap, W2T, S2T, 0, nthreads)
+    ab, _ = grouped_gemm(0, E, 2 * I, H, Aq, As, offsets, rows_cap, W13, S13, 0, nthreads)
+    abf = bf16_bits_to_f32(ab).reshape(rows_cap, I // GROUP, 2, GROUP)
+    dhf = bf16_bits_to_f32(dh).reshape(rows_cap, I // GROUP, GROUP)
+    da, dbb = swiglu_backward(abf[:, :, 0], abf[:, :, 1], dhf)
+    g = f64_to_bf16_bits(np.stack((da, dbb), axis=2).reshape(rows_cap, 2 * I))
+    valid = row_src >= 0
+    g[~valid] = 0
+    gf = bf16_bits_to_f32(g)
+    gq, gs = quant_rows(gf)
+    dxr, _ = grouped_gemm(0, E, H, 2 * I, gq, np.ascontiguousarray(gs.T), offsets, rows_cap, W13T, S13T, 0, nthreads)
+    dxrf = bf16_bits_to_f32(dxr).astype(np.float64)
+    dx64 = dx_router.copy()
+    for s in range(T * k):
+        if slot_row[s] >= 0:
+            dx64[s // k] += dxrf[slot_row[s]]
+    dx = f64_to_bf16_bits(dx64)
+    # weight gradients over each expert's 128-row tiles
+    hf = (e4m3_decode_array(hq).astype(np.float32) * np.repeat(hs, GROUP, axis=1)).astype(np.float32)
+    xf = (e4m3_decode_array(Aq).astype(np.float32) * np.repeat(np.ascontiguousarray(As.T), GROUP, axis=1)
+          ).astype(np.float32)
+    A2 = _deq_tiles(*tile_transpose_quant(dO, offsets, kept, "row"))        # [tiles, H, 128]
+    B2 = _deq_tiles(*tile_transpose_quant(hf, offsets, kept, "block"))      # [tiles, I, 128]
+    A13 = _deq_tiles(*tile_transpose_quant(gf, offsets, kept, "row"))       # [tiles, 2I, 128]
+    B13 = _deq_tiles(*tile_transpose_quant(xf, offsets, kept, "block"))     # [tiles, H, 128]
+    dW2 = np.zeros((E, H, I), np.uint16)
+    dW13 = np.zeros((E, 2 * I, H), np.uint16)
+    for e in range(E):
+        m0, m1 = int(offsets[e]) // GROUP, int(offsets[e + 1]) // GROUP
+        acc2 = np.zeros((H, I), np.float64)
+        acc13 = np.zeros((2 * I, H), np.float64)
+        for m in range(m0, m1):
+            acc2 += A2[m].astype(np.float64) @ B2[m].astype(np.float64).T
+            acc13 += A13[m].astype(np.float64) @ B13[m].astype(np.float64).T
+        dW2[e] = f64_to_bf16_bits(acc2)
+        dW13[e] = f64_to_bf16_bits(acc13)
+    return dict(dx=dx, dWg=dWg.astype(np.float32), db=db.astype(np.float32), dW13=dW13, dW2=dW2, dw=dw, dl=dl,
+                dOq=dOq, dOs=dOs, dh=dh, ab=ab, g=g, gq=gq, gs=gs, dx_rows=dxr, forward=f)

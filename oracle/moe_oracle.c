@@ -271,6 +271,24 @@ void orc_quant_rows(int64_t rows, int K, const float* v, uint8_t* q, float* s) {
     }
 }
 
+/* One quantisation group of n values with one scale (the same rule as a
+ * 1x128 group: scale = max|v| / 448 in fp32, 1 for an all-zero group; code =
+ * E4M3 of v / scale). Used for the 128x128 blocks of the weight-gradient
+ * operands of the backward pass. */
+void orc_quant_group(int64_t n, const float* v, uint8_t* q, float* s) {
+    int64_t i;
+    float amax = 0.0f, sc;
+    for (i = 0; i < n; ++i) if (fabsf(v[i]) > amax) amax = fabsf(v[i]);
+    if (amax == 0.0f) {
+        sc = 1.0f;
+        for (i = 0; i < n; ++i) q[i] = orc_e4m3_encode(v[i]);
+    } else {
+        sc = amax / 448.0f;
+        for (i = 0; i < n; ++i) q[i] = orc_e4m3_encode(v[i] / sc);
+    }
+    *s = sc;
+}
+
 /* ------------------------------------------------------------------ */
 /* Expert math (SwiGLU FFN E_i(x) = W2 (silu(W1 x) * W3 x))              */
 /* ------------------------------------------------------------------ */

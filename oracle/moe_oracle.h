@@ -108,6 +108,9 @@ void orc_grouped_gemm_w4(int layout, int E, int N, int K, const uint8_t* A, cons
  * word (i = 0..3): magnitude in bits 4i..4i+2, sign in bit 8i+7; level 4+i:
  * magnitude in bits 16+4i..16+4i+2, sign in bit 8i+3. */
 int orc_w4_decode(const uint8_t* row, int k);
+/* One group of n values quantised with one scale: max|v| / 448 (1 for all
+ * zeros), codes E4M3 of v / scale (the 1x128 rule applied to any group). */
+void orc_quant_group(int64_t n, const float* v, uint8_t* q, float* s);
 /* Combine: y[t,:] = sum_j [kept] w[t,j] * O[slot_row[t*k+j], :], fp64, -> bf16. */
 void orc_combine(int T, int k, int H, const int32_t* slot_row, const float* topk_w,
                  const uint16_t* O, uint16_t* y);
