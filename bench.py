@@ -257,6 +257,48 @@ class Layer:
         ev[5].record()
 
 
+def time_backward(layer, cfg, steps):
+    """The layer's backward (moe_backward) after one forward, timed over `steps` calls with CUDA events:
+    the training side of the layer, reported beside the forward. Contiguous layout, E4M3 weights, softmax
+    routing only."""
+    if cfg.layout != "contiguous" or cfg.weights != "fp8" or cfg.routing != "softmax":
+        return None
+    from fp8_grouped_gemm_fp32_b200.inputs import transpose_weights
+    api, i = layer.api, layer.inp
+    dev = layer.y.device
+    W13T, S13T, W2T, S2T = transpose_weights(layer.W13, layer.S13, i.W2q, i.S2)
+    g = torch.Generator(device=dev).manual_seed(17)
+    dy = (torch.randn(cfg.T, cfg.H, generator=g, device=dev) * 0.1).to(torch.bfloat16)
+    z = lambda *s_, dt: torch.empty(*s_, dtype=dt, device=dev)
+    dx, dWg, db = z(cfg.T, cfg.H, dt=torch.bfloat16), z(cfg.E, cfg.H, dt=torch.float32), z(cfg.E, dt=torch.float32)
+    dW13, dW2 = z(cfg.E, 2 * cfg.I, cfg.H, dt=torch.bfloat16), z(cfg.E, cfg.H, cfg.I, dt=torch.bfloat16)
+    bws = z(api.moe_backward_workspace_size(layer.c), dt=torch.uint8)
+    layer.forward()
+
+    def call():
+        api.moe_backward(layer.c, i.x, i.Wg, layer.W13, layer.S13, W13T, S13T, W2T, S2T, layer.topk_idx, layer.topk_w,
+                         layer.slot_row, layer.ws, dy, dx, dWg, db, dW13, dW2, bws)
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    assert api.moe_get_device_status() == api.MOE_OK
+    ms = e0.elapsed_time(e1) / steps
+    Rk = int(layer.kept.sum().item()) if hasattr(layer.kept, "sum") else 0
+    # FP8 tensor work: dh (H x I), a|b recomputed (2I x H), dx rows (H x 2I), dW2 (H x I), dW13 (2I x H),
+    # each 2 FLOP per multiply-add over the kept rows
+    flops = 2.0 * Rk * cfg.H * cfg.I * (1 + 2 + 2 + 1 + 2)
+    del bws, dW13, dW2
+    return {"ms": ms, "tokens_per_s": cfg.T / (ms / 1e3), "calls": steps, "gemm_tflops_lower_bound": flops / (ms / 1e3) / 1e12,
+            "what": "moe_backward: dx, dW_g, db, dW13, dW2 of one step (five FP8 grouped GEMMs, two of them "
+                    "K-grouped weight gradients), after one forward"}
+
+
 def run_e2e(layer, cfg, steps, world):
     dev = layer.inp.x.device
     hash_routing = cfg.routing == "hash"
@@ -486,6 +528,8 @@ def run_ours(args):
     balance = {"us_per_call": 1e3 * b0.elapsed_time(b1) / 200, "calls": 200, "timing": "CUDA graph replay",
                "bytes_per_call": 28 * cfg.E, "bound": "launch latency (one block, 28 B per expert)"}
 
+    backward = time_backward(layer, cfg, max(3, min(args.steps, 20))) if args.backward else None
+
     peaks, peak_src = load_peaks()
     hbm = float(peaks["hbm_gbs"])
     # The per-kernel events time each GEMM as a burst of a few milliseconds, so the tensor roofline takes
@@ -544,6 +588,7 @@ def run_ours(args):
         "kernels_ms": per,
         "routing": routing_stats(layer.counts.cpu().numpy(), kept),
         "balance_bias": balance,
+        "backward": backward,
         "e2e": {"value": job_tokens_per_s(cfg.T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": layer.launches_per_step * args.steps,
@@ -602,6 +647,8 @@ def main():
                     help="workload (default: prefill, the largest that fits one GPU)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time the layer's backward pass (contiguous FP8 workloads)")
     ap.add_argument("--contig", default="auto", choices=["auto", "single", "pair"],
                     help="form of the contiguous grouped GEMM (default: chosen by shape)")
     ap.add_argument("--experts", type=int, default=0,

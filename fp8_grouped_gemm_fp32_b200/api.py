@@ -34,7 +34,7 @@ EXPORTS = ("moe_rows_capacity", "moe_workspace_size", "moe_route", "moe_permute"
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string",
            "moe_permute_noalloc", "moe_balance_bias", "moe_grouped_gemm_w4", "moe_set_contig_kernel",
            "moe_ep_plan", "moe_ep_workspace_size", "moe_ep_count", "moe_ep_dispatch", "moe_ep_receive",
-           "moe_ep_return")
+           "moe_ep_return", "moe_backward_workspace_size", "moe_backward")
 
 
 class MoeError(RuntimeError):
@@ -89,10 +89,14 @@ def lib() -> ctypes.CDLL:
         L.moe_ep_dispatch.argtypes = [CP, P, P, P, P, P, P, SZ, P]
         L.moe_ep_receive.argtypes = [I, P, I, P, P, P, I, P, P, P]
         L.moe_ep_return.argtypes = [I, I, P, P, P, P]
+        L.moe_backward_workspace_size.argtypes = [CP]
+        L.moe_backward_workspace_size.restype = SZ
+        L.moe_backward.argtypes = [CP] + [P] * 18 + [SZ, P]
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in EXPORTS:
-            if f not in ("moe_rows_capacity", "moe_workspace_size", "moe_status_string", "moe_ep_workspace_size"):
+            if f not in ("moe_rows_capacity", "moe_workspace_size", "moe_status_string", "moe_ep_workspace_size",
+                         "moe_backward_workspace_size"):
                 getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -221,3 +225,15 @@ def moe_ep_receive(H, plan_dev, rows_recv, recv, Aq, As, M_rows, offsets, group_
 
 def moe_ep_return(H, rows_recv, O, group_row, ret, stream=None):
     _check(lib().moe_ep_return(H, rows_recv, _p(O), _p(group_row), _p(ret), _stream(stream)), "moe_ep_return")
+
+
+# ---------------------------------------------------------------- backward pass
+def moe_backward_workspace_size(cfg: Config) -> int:
+    return int(lib().moe_backward_workspace_size(ctypes.byref(cfg)))
+
+
+def moe_backward(cfg, x, Wg, W13, S13, W13T, S13T, W2T, S2T, topk_idx, topk_w, slot_row, fwd_ws, dy, dx, dWg, db,
+                 dW13, dW2, ws, stream=None):
+    _check(lib().moe_backward(ctypes.byref(cfg), _p(x), _p(Wg), _p(W13), _p(S13), _p(W13T), _p(S13T), _p(W2T),
+                              _p(S2T), _p(topk_idx), _p(topk_w), _p(slot_row), _p(fwd_ws), _p(dy), _p(dx), _p(dWg),
+                              _p(db), _p(dW13), _p(dW2), _p(ws), _nbytes(ws), _stream(stream)), "moe_backward")

@@ -32,6 +32,32 @@ cudaError_t launch_combine(const uint16_t* O, const int32_t* slot_row, const flo
                            uint16_t* y, cudaStream_t s);
 cudaError_t launch_selftest_wait(int* status, uint64_t wait_ns, cudaStream_t s);
 void set_contig_mode(int mode);
+cudaError_t launch_grouped_gemm_kgroup(int E, int M, int N, const uint8_t* A, const float* As, const int32_t* offsets,
+                                       int rows_fwd, const uint8_t* B, const float* Bs, void* D, int* status,
+                                       uint64_t wait_ns, int num_sms, cudaStream_t s);
+cudaError_t launch_slot_lists(const int32_t* topk_idx, int T, int k, int E, int32_t* counts, int32_t* offsets,
+                              int32_t* list, int32_t* slot_tmp, void* scratch, int* status, cudaStream_t s);
+size_t ep_scratch_bytes(int T, int E);
+struct TqArgs {
+    const uint16_t* dy;
+    const float* topk_w;
+    const uint8_t* codes;
+    const float* scales;
+    const uint16_t* bf;
+    const int32_t* row_src;
+    int rows, k, C;
+};
+cudaError_t launch_bwd_dl(const uint16_t* dy, const uint16_t* O, const int32_t* slot_row, const float* topk_w, int T,
+                          int k, int H, float* dl, cudaStream_t s);
+cudaError_t launch_bwd_dout(const uint16_t* dy, const float* topk_w, const int32_t* row_src, int rows, int k, int H,
+                            uint8_t* q, float* sc, cudaStream_t s);
+cudaError_t launch_bwd_swiglu(const uint16_t* ab, const uint16_t* dh, const int32_t* row_src, int rows, int I,
+                              uint16_t* g, uint8_t* gq, float* gs, cudaStream_t s);
+cudaError_t launch_bwd_tquant(int src, bool rows_mode, const TqArgs& a, uint8_t* out, float* os, cudaStream_t s);
+cudaError_t launch_bwd_dx(const uint16_t* dxr, const int32_t* slot_row, const int32_t* topk_idx, const float* dl,
+                          const float* Wg, int T, int k, int H, uint16_t* dx, cudaStream_t s);
+cudaError_t launch_bwd_gate(const uint16_t* x, const float* dl, const int32_t* offsets, const int32_t* list, int E, int k,
+                            int H, float* dWg, float* db, cudaStream_t s);
 cudaError_t launch_balance_bias(int E, const int32_t* counts, int64_t* load, float* bias, float gamma, int update,
                                 cudaStream_t s);
 
@@ -43,7 +69,7 @@ __device__ int g_status;
 moe_status_t check_cfg(const moe_config_t* c) {
     if (!c) return MOE_ERR_INVALID_ARG;
     if (c->T < 0 || c->H <= 0 || c->I <= 0 || c->E <= 0 || c->k <= 0) return MOE_ERR_INVALID_ARG;
-    if (c->H % kGroup || c->I % kGroup || c->H > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->H % kGroup || c->I % kGroup || c->H > 16384 || c->I > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->E > MOE_MAX_EXPERTS || c->k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->k > c->E) return MOE_ERR_INVALID_ARG;
     if (c->routing != MOE_ROUTE_SOFTMAX_TOPK && c->routing != MOE_ROUTE_HASH) return MOE_ERR_INVALID_ARG;
@@ -155,6 +181,56 @@ FwdWs carve(const moe_config_t* c, void* base) {
 }
 
 inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// moe_backward's scratch, in carving order (rows = the forward's contiguous rows, tiles = rows / 128)
+struct BwdWs {
+    uint8_t* dOq; float* dOs;             // w * dy on kept rows, 1x128 FP8 along H
+    uint16_t* dh;                         // dO W2, bf16 [rows, I]
+    uint16_t* ab;                         // x W13^T recomputed, bf16 [rows, 2I]
+    uint16_t* g; uint8_t* gq; float* gs;  // SwiGLU backward, bf16 and 1x128 FP8 along 2I
+    uint16_t* dxr;                        // g W13, bf16 [rows, H]
+    float* dl;                            // [T k]
+    uint8_t* A2; float* A2s; uint8_t* B2; float* B2s;        // weight-gradient operands of W2
+    uint8_t* A13; float* A13s; uint8_t* B13; float* B13s;    // ... and of W13
+    int32_t* counts; int32_t* offs; int32_t* list; int32_t* slot_tmp; void* scratch;
+    size_t total;
+};
+
+BwdWs carve_bwd(const moe_config_t* c, void* base) {
+    BwdWs w;
+    const size_t rows = rows_of(c), tiles = rows / kGroup, H = c->H, I = c->I, R = static_cast<size_t>(c->T) * c->k;
+    uint8_t* p = static_cast<uint8_t*>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* q = p ? p + off : nullptr;
+        off += align_up(bytes);
+        return q;
+    };
+    w.dOq = take(rows * H);
+    w.dOs = reinterpret_cast<float*>(take(4 * rows * (H / kGroup)));
+    w.dh = reinterpret_cast<uint16_t*>(take(2 * rows * I));
+    w.ab = reinterpret_cast<uint16_t*>(take(2 * rows * 2 * I));
+    w.g = reinterpret_cast<uint16_t*>(take(2 * rows * 2 * I));
+    w.gq = take(rows * 2 * I);
+    w.gs = reinterpret_cast<float*>(take(4 * rows * (2 * I / kGroup)));
+    w.dxr = reinterpret_cast<uint16_t*>(take(2 * rows * H));
+    w.dl = reinterpret_cast<float*>(take(4 * R));
+    w.A2 = take(rows * H);
+    w.A2s = reinterpret_cast<float*>(take(4 * tiles * H));
+    w.B2 = take(rows * I);
+    w.B2s = reinterpret_cast<float*>(take(4 * tiles * (I / kGroup)));
+    w.A13 = take(rows * 2 * I);
+    w.A13s = reinterpret_cast<float*>(take(4 * tiles * 2 * I));
+    w.B13 = take(rows * H);
+    w.B13s = reinterpret_cast<float*>(take(4 * tiles * (H / kGroup)));
+    w.counts = reinterpret_cast<int32_t*>(take(4 * static_cast<size_t>(c->E)));
+    w.offs = reinterpret_cast<int32_t*>(take(4 * (static_cast<size_t>(c->E) + 1)));
+    w.list = reinterpret_cast<int32_t*>(take(4 * R));
+    w.slot_tmp = reinterpret_cast<int32_t*>(take(4 * R));
+    w.scratch = take(ep_scratch_bytes(c->T, c->E));
+    w.total = off;
+    return w;
+}
 
 }  // namespace
 
@@ -342,6 +418,78 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_combine(w.O, slot_row, topk_w, cfg->T, cfg->k, cfg->H, static_cast<uint16_t*>(y), s);
     return cuda_status(e);
+}
+
+size_t moe_backward_workspace_size(const moe_config_t* cfg) {
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    return carve_bwd(cfg, nullptr).total;
+}
+
+moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const float* Wg, const uint8_t* W13, const float* S13,
+                          const uint8_t* W13T, const float* S13T, const uint8_t* W2T, const float* S2T,
+                          const int32_t* topk_idx, const float* topk_w, const int32_t* slot_row, const void* fwd_ws,
+                          const void* dy, void* dx, float* dWg, float* db, void* dW13, void* dW2, void* ws,
+                          size_t ws_bytes, void* stream) {
+    moe_status_t st = check_cfg(cfg);
+    if (st != MOE_OK) return st;
+    if (cfg->layout != MOE_LAYOUT_CONTIGUOUS || cfg->weights != MOE_WEIGHTS_FP8 ||
+        cfg->routing != MOE_ROUTE_SOFTMAX_TOPK)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    // the weight-gradient GEMM stages at most 128 K blocks per expert: 16384 rows
+    const int64_t most = cfg->cap_num ? std::min<int64_t>(cfg->T, capacity_of(cfg)) : cfg->T;
+    if (most > 16384 || 2 * cfg->I > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;   // K of g W13 is 2I
+    DeviceInfo* dev;
+    if ((st = device_info(&dev)) != MOE_OK) return st;
+    if (cfg->T == 0) return MOE_OK;
+    if (!ptr_ok(x) || !ptr_ok(Wg) || !ptr_ok(W13) || !ptr_ok(S13) || !ptr_ok(W13T) || !ptr_ok(S13T) || !ptr_ok(W2T) ||
+        !ptr_ok(S2T) || !ptr_ok(topk_idx) || !ptr_ok(topk_w) || !ptr_ok(slot_row) || !ptr_ok(fwd_ws) || !ptr_ok(dy) ||
+        !ptr_ok(dx) || !ptr_ok(dWg) || !ptr_ok(db) || !ptr_ok(dW13) || !ptr_ok(dW2) || !ptr_ok(ws) ||
+        (reinterpret_cast<uintptr_t>(ws) % kAlign) || (reinterpret_cast<uintptr_t>(fwd_ws) % kAlign))
+        return MOE_ERR_INVALID_ARG;
+    const BwdWs b = carve_bwd(cfg, ws);
+    if (ws_bytes < b.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    const FwdWs f = carve(cfg, const_cast<void*>(fwd_ws));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int T = cfg->T, k = cfg->k, H = cfg->H, I = cfg->I, E = cfg->E;
+    const int rows = static_cast<int>(rows_of(cfg));
+    const uint16_t* dy16 = static_cast<const uint16_t*>(dy);
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    // gate: dw, dl; expert path: dO, dh, a|b, g, dx rows, dx
+    if (!ok(launch_bwd_dl(dy16, f.O, slot_row, topk_w, T, k, H, b.dl, s))) return MOE_ERR_CUDA;
+    if (!ok(launch_bwd_dout(dy16, topk_w, f.row_src, rows, k, H, b.dOq, b.dOs, s))) return MOE_ERR_CUDA;
+    if (!ok(launch_grouped_gemm(MOE_LAYOUT_CONTIGUOUS, E, I, H, b.dOq, b.dOs, f.offsets, rows, W2T, S2T, MOE_EPI_BF16,
+                                b.dh, nullptr, dev->status, kWaitNs, dev->num_sms, s)))
+        return MOE_ERR_CUDA;
+    if (!ok(launch_grouped_gemm(MOE_LAYOUT_CONTIGUOUS, E, 2 * I, H, f.Aq, f.As, f.offsets, rows, W13, S13, MOE_EPI_BF16,
+                                b.ab, nullptr, dev->status, kWaitNs, dev->num_sms, s)))
+        return MOE_ERR_CUDA;
+    if (!ok(launch_bwd_swiglu(b.ab, b.dh, f.row_src, rows, I, b.g, b.gq, b.gs, s))) return MOE_ERR_CUDA;
+    if (!ok(launch_grouped_gemm(MOE_LAYOUT_CONTIGUOUS, E, H, 2 * I, b.gq, b.gs, f.offsets, rows, W13T, S13T,
+                                MOE_EPI_BF16, b.dxr, nullptr, dev->status, kWaitNs, dev->num_sms, s)))
+        return MOE_ERR_CUDA;
+    if (!ok(launch_bwd_dx(b.dxr, slot_row, topk_idx, b.dl, Wg, T, k, H, static_cast<uint16_t*>(dx), s)))
+        return MOE_ERR_CUDA;
+    // gate gradients over every slot of each expert, in token order
+    if (!ok(launch_slot_lists(topk_idx, T, k, E, b.counts, b.offs, b.list, b.slot_tmp, b.scratch, dev->status, s)))
+        return MOE_ERR_CUDA;
+    if (!ok(launch_bwd_gate(static_cast<const uint16_t*>(x), b.dl, b.offs, b.list, E, k, H, dWg, db, s)))
+        return MOE_ERR_CUDA;
+    // weight gradients: per forward row tile, the transposed operands, then the K-grouped GEMMs
+    TqArgs a{dy16, topk_w, nullptr, nullptr, nullptr, f.row_src, rows, k, H};
+    if (!ok(launch_bwd_tquant(0, true, a, b.A2, b.A2s, s))) return MOE_ERR_CUDA;
+    a.codes = f.Hq; a.scales = f.Hs; a.C = I;
+    if (!ok(launch_bwd_tquant(1, false, a, b.B2, b.B2s, s))) return MOE_ERR_CUDA;
+    a.bf = b.g; a.C = 2 * I;
+    if (!ok(launch_bwd_tquant(2, true, a, b.A13, b.A13s, s))) return MOE_ERR_CUDA;
+    a.codes = f.Aq; a.scales = f.As; a.C = H;
+    if (!ok(launch_bwd_tquant(1, false, a, b.B13, b.B13s, s))) return MOE_ERR_CUDA;
+    if (!ok(launch_grouped_gemm_kgroup(E, H, I, b.A2, b.A2s, f.offsets, rows, b.B2, b.B2s, dW2, dev->status, kWaitNs,
+                                       dev->num_sms, s)))
+        return MOE_ERR_CUDA;
+    if (!ok(launch_grouped_gemm_kgroup(E, 2 * I, H, b.A13, b.A13s, f.offsets, rows, b.B13, b.B13s, dW13, dev->status,
+                                       kWaitNs, dev->num_sms, s)))
+        return MOE_ERR_CUDA;
+    return MOE_OK;
 }
 
 moe_status_t moe_balance_bias(int E, const int32_t* counts, int64_t* load, float* bias, float gamma, int update,

@@ -106,6 +106,8 @@ __device__ __forceinline__ int find_group(const int32_t* P, int E, int q) {
 struct TileC {
     int e, m0, n0, width;
     bool store;      // false for the idle half of a lone pair tile: computed, not written
+    int kb0, nkb;    // the tile's K blocks: kb0 .. kb0 + nkb - 1 (K-grouped: the expert's forward row tiles)
+    int am0;         // K-grouped: the tile's first row within each K block's operand block
 };
 
 __device__ __forceinline__ TileC decode_tile_c(const int32_t* P, int E, int NT, int N, int tile) {
@@ -145,12 +147,18 @@ __device__ __forceinline__ TileC decode_tile_pair(const int32_t* P, const int32_
 
 __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
-template <int EPI, bool PAIR>
+// KG (K-grouped, the weight gradients of the backward pass): expert e's output is its own M_rows x N
+// matrix (rows e * M_rows ...); its K blocks are the expert's 128-row tiles of a forward contiguous layout
+// (offsets, kg_rows rows in all), and K block m of the A operand is the [M_rows, 128] block at rows
+// m * M_rows of A (of B: rows m * N); A's scales are [tiles][M_rows] (one per row per K block), B's
+// [tiles][N / 128] (one per 128-row block per K block).
+template <int EPI, bool PAIR, bool KG = false>
 __global__ void __launch_bounds__(kThreadsC, 1)
 gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmD, const float* __restrict__ As, const int32_t* __restrict__ offsets, int M_rows,
                  const float* __restrict__ Bs, int E, int N, int K, void* __restrict__ D, float* __restrict__ Ds,
-                 int* status, uint64_t wait_ns) {
+                 int* status, uint64_t wait_ns, int kg_rows) {
+    static_assert(!KG || (EPI == 0 && !PAIR), "K-grouped tiles run on single CTAs with the bf16 epilogue");
     extern __shared__ uint8_t smem_raw[];
     using SC = SmemC<EPI, PAIR>;
     constexpr int kStagesC = SC::kStages;
@@ -174,7 +182,7 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         for (int b = 0; b <= E; b += 32) {
             const int e = b + lane;
             const int o = e <= E ? offsets[e] : 0;
-            int v = e == 0 ? 0 : min(max(o, 0), M_rows) / kBM;
+            int v = e == 0 ? 0 : min(max(o, 0), KG ? kg_rows : M_rows) / kBM;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
                 const int u = __shfl_up_sync(0xffffffffu, v, d);
@@ -188,6 +196,13 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             carry = __shfl_sync(0xffffffffu, v, 31);
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, kStatusCapacity);
+        if constexpr (KG) {
+            // a K-grouped tile stages at most kMaxKB weight-block scales: longer experts are reported
+            __syncwarp();
+            bool longk = false;
+            for (int e = lane; e < E; e += 32) longk |= sm.P[e + 1] - sm.P[e] > kMaxKB;
+            if (__any_sync(0xffffffffu, longk) && lane == 0) set_status(status, kStatusCapacity);
+        }
         if constexpr (PAIR) {
             // pair tiles per expert: Q[e + 1] - Q[e] = ceil((P[e + 1] - P[e]) / 2)
             __syncwarp();
@@ -239,10 +254,31 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if constexpr (PAIR) cluster_sync(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int total = (PAIR ? sm.Q[E] : sm.P[E]) * NT;
+    const int MTd = M_rows / kBM;             // K-grouped: M tiles of each expert's output
+    const int total = KG ? E * MTd * NT : (PAIR ? sm.Q[E] : sm.P[E]) * NT;
     auto decode = [&](int tile) -> TileC {
-        if constexpr (PAIR) return decode_tile_pair(sm.P, sm.Q, E, NT, tile, rank);
-        else return decode_tile_c(sm.P, E, NT, N, tile);
+        TileC t;
+        if constexpr (KG) {
+            // expert -> N tile -> M tile: the tiles running together share the expert's B blocks
+            t.e = tile / (NT * MTd);
+            const int rem = tile - t.e * NT * MTd;
+            const int nt = rem / MTd;
+            t.am0 = (rem - nt * MTd) * kBM;
+            t.m0 = t.e * M_rows + t.am0;
+            t.n0 = nt * kBN;
+            t.width = min(kBN, N - t.n0);
+            t.store = true;
+            t.kb0 = sm.P[t.e];
+            t.nkb = min(sm.P[t.e + 1] - sm.P[t.e], kMaxKB);
+            return t;
+        } else {
+            if constexpr (PAIR) t = decode_tile_pair(sm.P, sm.Q, E, NT, tile, rank);
+            else t = decode_tile_c(sm.P, E, NT, N, tile);
+            t.kb0 = 0;
+            t.nkb = KB;
+            t.am0 = t.m0;
+            return t;
+        }
     };
 
     // A wait that runs out stops this CTA and (PAIR) its partner, whose waits on this CTA would otherwise
@@ -268,13 +304,25 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // loads are issued, so their latency stays off the TMA stream.
         float wr0[4], wr1[4];
         auto read_scales = [&](const TileC& u) {
-            const float* b0 = Bs + (static_cast<int64_t>(u.e) * NB + u.n0 / kBM) * KB;
-            const float* b1 = u.width == kBN ? b0 + KB : b0;
+            if constexpr (KG) {
+                // K block kb of the tile is forward row tile u.kb0 + kb; B's scales are [tiles][N / 128]
+                const float* b0 = Bs + static_cast<int64_t>(u.kb0) * NB + u.n0 / kBM;
+                const int d1 = u.width == kBN ? 1 : 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int kb = lane + 32 * i;
-                wr0[i] = kb < KB ? b0[kb] : 0.0f;
-                wr1[i] = kb < KB ? b1[kb] : 0.0f;
+                for (int i = 0; i < 4; ++i) {
+                    const int kb = lane + 32 * i;
+                    wr0[i] = kb < u.nkb ? b0[static_cast<int64_t>(kb) * NB] : 0.0f;
+                    wr1[i] = kb < u.nkb ? b0[static_cast<int64_t>(kb) * NB + d1] : 0.0f;
+                }
+            } else {
+                const float* b0 = Bs + (static_cast<int64_t>(u.e) * NB + u.n0 / kBM) * KB;
+                const float* b1 = u.width == kBN ? b0 + KB : b0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int kb = lane + 32 * i;
+                    wr0[i] = kb < KB ? b0[kb] : 0.0f;
+                    wr1[i] = kb < KB ? b1[kb] : 0.0f;
+                }
             }
         };
         auto publish_scales = [&](uint32_t ti) -> bool {
@@ -318,11 +366,19 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 // bytes of both (its MMA reads both CTAs' stages); each CTA loads its A rows and its half of B
                 const uint32_t bytes = PAIR ? 2u * (kABytes + SC::kBStage)
                                             : kABytes + (t.width == kBN ? kBBytes : kBBytes / 2);
-                for (int kb = 0; kb < KB; ++kb, ++it) {
+                for (int kb = 0; kb < t.nkb; ++kb, ++it) {
                     const int s = it % kStagesC;
                     const uint32_t ph = (it / kStagesC) & 1;
                     if (!mbar_wait(&sm.empty[s], ph ^ 1, wait_ns)) { fail(); ok = 0; break; }
-                    if constexpr (PAIR) {
+                    if constexpr (KG) {
+                        // operand blocks of forward row tile kb0 + kb: A rows (kb0 + kb) * M_rows + am0,
+                        // B rows (kb0 + kb) * N + n0, each 128 bytes of K
+                        const int m = t.kb0 + kb;
+                        mbar_arrive_expect_tx(&sm.full[s], bytes);
+                        tma_load_2d(sm.a[s], &tmA, &sm.full[s], 0, m * M_rows + t.am0);
+                        tma_load_2d(sm.b[s], &tmB, &sm.full[s], 0, m * N + t.n0);
+                        if (t.width == kBN) tma_load_2d(sm.b[s] + kBBytes / 2, &tmB, &sm.full[s], 0, m * N + t.n0 + 128);
+                    } else if constexpr (PAIR) {
                         const uint32_t fb = mapa_shared(smem_u32(&sm.full[s]), 0);
                         if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], bytes);
                         tma_load_2d_pair(sm.a[s], &tmA, fb, kb * kBK, t.m0);
@@ -338,7 +394,7 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const int j = it % kSaSlots;
                     if (!mbar_wait(&sm.sempty[j], ((it / kSaSlots) & 1) ^ 1, wait_ns)) { fail(); ok = 0; break; }
                     mbar_arrive_expect_tx(&sm.sfull[j], kBM * sizeof(float));
-                    bulk_load(sm.sa[j], As + static_cast<int64_t>(kb) * M_rows + t.m0, kBM * sizeof(float),
+                    bulk_load(sm.sa[j], As + static_cast<int64_t>(t.kb0 + kb) * M_rows + t.am0, kBM * sizeof(float),
                               &sm.sfull[j]);
                 }
             }
@@ -356,7 +412,7 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             for (int tile = tile0; tile < total && !sm.abort_flag; tile += tstep) {
                 const TileC t = decode(tile);
                 const uint32_t idesc = PAIR ? f8_idesc(2 * kBM, kBN) : f8_idesc(kBM, t.width);
-                for (int kb = 0; kb < KB; ++kb, ++it, ++kbt) {
+                for (int kb = 0; kb < t.nkb; ++kb, ++it, ++kbt) {
                     const int s = it % kStagesC;
                     const uint32_t ph = (it / kStagesC) & 1;
                     const int buf = kbt & 1;
@@ -408,7 +464,7 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
             float* acc = reinterpret_cast<float*>(acc2);
             bool ok = true;
-            for (int kb = 0; kb < KB; ++kb, ++kbt) {
+            for (int kb = 0; kb < t.nkb; ++kb, ++kbt) {
                 const int buf = kbt & 1;
                 const uint32_t bph = (kbt >> 1) & 1;
                 // scales: sa from the ring (the producer copied it several K blocks ago), the weight
@@ -1045,12 +1101,12 @@ static cudaError_t check_reg_split(Kern k) {
 
 // Contiguous kernel in one of its two forms: one CTA per tile, or (PAIR) clusters of two CTAs sharing
 // 256 x 256 tiles, as many clusters as fit on the device at once (queried once per device).
-template <int EPI, bool PAIR>
+template <int EPI, bool PAIR, bool KG = false>
 static cudaError_t launch_contig(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapD,
                                  const float* As, const int32_t* offsets, int M_rows, const float* Bs, int E, int N,
                                  int K, void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms,
-                                 cudaStream_t s) {
-    auto kern = gg_contig_kernel<EPI, PAIR>;
+                                 cudaStream_t s, int kg_rows = 0) {
+    auto kern = gg_contig_kernel<EPI, PAIR, KG>;
     const size_t smem = sizeof(SmemC<EPI, PAIR>) + 1024;
     cudaError_t err = set_smem(kern, smem);
     if (err == cudaSuccess) err = check_reg_split(kern);
@@ -1084,7 +1140,24 @@ static cudaError_t launch_contig(const CUtensorMap& mapA, const CUtensorMap& map
         cfg.attrs = nullptr;
         cfg.numAttrs = 0;
     }
-    return cudaLaunchKernelEx(&cfg, kern, mapA, mapB, mapD, As, offsets, M_rows, Bs, E, N, K, D, Ds, status, wait_ns);
+    return cudaLaunchKernelEx(&cfg, kern, mapA, mapB, mapD, As, offsets, M_rows, Bs, E, N, K, D, Ds, status, wait_ns,
+                              kg_rows);
+}
+
+// K-grouped grouped GEMM (the backward pass's weight gradients): D [E * M, N] bf16, expert e's rows
+// e * M .. : sum over the expert's 128-row tiles m of the forward contiguous layout (offsets [E + 1],
+// rows_fwd rows) of A_m [M, 128] x B_m [N, 128]^T, with A = [tiles * M, 128] codes, As = [tiles][M]
+// (one scale per row per tile), B = [tiles * N, 128] codes, Bs = [tiles][N / 128].
+cudaError_t launch_grouped_gemm_kgroup(int E, int M, int N, const uint8_t* A, const float* As, const int32_t* offsets,
+                                       int rows_fwd, const uint8_t* B, const float* Bs, void* D, int* status,
+                                       uint64_t wait_ns, int num_sms, cudaStream_t s) {
+    const uint64_t tiles = static_cast<uint64_t>(rows_fwd) / kBM;
+    CUtensorMap mapA, mapB, mapD;
+    if (!make_map(&mapA, A, kBK, tiles * M, kBM)) return cudaErrorInvalidValue;
+    if (!make_map(&mapB, B, kBK, tiles * N, 128)) return cudaErrorInvalidValue;
+    if (!make_out_map(&mapD, D, N, static_cast<uint64_t>(E) * M, 2)) return cudaErrorInvalidValue;
+    return launch_contig<0, false, true>(mapA, mapB, mapD, As, offsets, M, Bs, E, N, kBK, D, nullptr, status, wait_ns,
+                                         num_sms, s, rows_fwd);
 }
 
 // Which form of the contiguous kernel runs (moe_set_contig_kernel): 0 chooses by shape, 1 forces single

@@ -382,6 +382,23 @@ cudaError_t launch_ep_count(const int32_t* topk_idx, int T, int k, int E, int32_
     return cudaGetLastError();
 }
 
+// Every slot of every expert, dropped ones included, in token order: counts [E], offsets [E + 1] (unpadded
+// prefix) and list [T * k] (list[offsets[e] + r] = the slot t * k + j of expert e's r-th token); slot_tmp
+// [T * k] receives each slot's position. Scratch as launch_ep_count's.
+cudaError_t launch_slot_lists(const int32_t* topk_idx, int T, int k, int E, int32_t* counts, int32_t* offsets,
+                              int32_t* list, int32_t* slot_tmp, void* scratch, int* status, cudaStream_t s) {
+    const int nchunks = (T + kChunk - 1) / kChunk;
+    int32_t* cnt = static_cast<int32_t*>(scratch);
+    int32_t* base = cnt + static_cast<size_t>(nchunks) * E;
+    int32_t* unused_kept = base + static_cast<size_t>(nchunks) * E;
+    permute_count_kernel<<<(nchunks + 7) / 8, 256, 8 * E * sizeof(uint32_t), s>>>(topk_idx, T, k, E, nchunks, cnt);
+    permute_scan_kernel<<<E, 256, 0, s>>>(cnt, nchunks, -1, 0, base, counts, unused_kept, status);
+    const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1);
+    permute_map_kernel<<<nchunks, 256, smem, s>>>(topk_idx, T, 0, k, E, nchunks, 1, 1, 0, 0, base, counts, nullptr,
+                                                  nullptr, offsets, list, slot_tmp);
+    return cudaGetLastError();
+}
+
 size_t ep_scratch_bytes(int T, int E) { return permute_scratch_bytes(T, E) + sizeof(int32_t) * static_cast<size_t>(E); }
 
 // Bytes of one send / receive row: H codes, H/128 fp32 scales, padded to 16 bytes.

@@ -231,6 +231,14 @@ def interleave_w13_w4(W1q: torch.Tensor, S1: torch.Tensor, W3q: torch.Tensor, S3
     return w.reshape(E, 2 * I, Hp).contiguous(), s.reshape(E, KB, 2 * I).contiguous()
 
 
+def transpose_weights(W13: torch.Tensor, S13: torch.Tensor, W2: torch.Tensor, S2: torch.Tensor):
+    """The backward pass's transposed operands (pure layout): W13 [E, 2I, H] -> [E, H, 2I] with its block
+    scales [E, 2I/128, H/128] -> [E, H/128, 2I/128], and W2 [E, H, I] -> [E, I, H], [E, H/128, I/128] ->
+    [E, I/128, H/128]. A 128x128 block keeps its scale."""
+    t = lambda a: a.transpose(1, 2).contiguous()
+    return t(W13), t(S13), t(W2), t(S2)
+
+
 def capacity_rows_bound(cfg: MoeConfig, pad: int = BLOCK) -> int:
     """Upper bound on the rows of the permuted activation buffer: every kept
     slot plus at most pad-1 padding rows per expert (contiguous layout), or

@@ -76,7 +76,7 @@ typedef struct {
                            empty; moe_ep_count still zeroes its counts) */
     int H;              /* hidden size, multiple of 128 */
     int E;              /* experts, 1..MOE_MAX_EXPERTS */
-    int I;              /* expert intermediate size, multiple of 128 */
+    int I;              /* expert intermediate size, multiple of 128, at most 16384 */
     int k;              /* experts per token (1..min(E, MOE_MAX_TOPK)); hash routing needs k = 1 */
     int routing;        /* moe_routing_t */
     int cap_num;        /* capacity factor alpha = cap_num / cap_den; 0 / 0 = dropless */
@@ -264,6 +264,48 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
 moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
                                  uint8_t* Aq, float* As, int32_t* counts, int32_t* kept, int32_t* offsets,
                                  int32_t* row_src, int32_t* slot_row, void* stream);
+
+/*
+ * The layer's backward pass. Source: TP-MoE page, section 4.1, step 5 (the
+ * gradients run back along the dispatch path and the gate network is updated
+ * too). Given dy = dL/dy [T, H] bf16 of one moe_forward call, computes
+ *   dx   [T, H] bf16     = sum over kept slots of (g W13)[row] + sum over all
+ *                          slots of dl_j W_g[e_j]
+ *   dWg  [E, H] fp32, db [E] fp32: sum over the slots of each expert, in token
+ *                          order (dropped slots included), of dl x and of dl
+ *   dW13 [E, 2I, H] bf16 (rows in W13's W1/W3 128-row block alternation) and
+ *   dW2  [E, H, I] bf16: per expert, sums over its kept rows of g^T x and
+ *                          dO^T h
+ * with dw_j = <dy_t, o_j> (0 for a dropped slot), dl_j = w_j (dw_j -
+ * sum_i w_i dw_i), dO = w dy (fp32) on each kept row, dh = dO W2, a | b = x
+ * W13^T (recomputed), g = (dh b s (1 + a (1 - s)), dh a s), s = sigmoid(a).
+ * The forward's quantisation steps pass the gradient straight through; the
+ * selection and the capacity drop are held fixed. Every GEMM is FP8 with fp32
+ * scales and fp32 promotion: dO, g and x in 1x128 groups along the
+ * contraction (the weight gradients group along the expert's rows), h and x
+ * in 128x128 blocks as the second weight-gradient operand; dh, a, b, g and
+ * the GEMM outputs are bf16.
+ *   x, Wg, W13, S13         the forward's inputs
+ *   W13T [E, H, 2I], S13T [E, H/128, 2I/128], W2T [E, I, H], S2T [E, I/128,
+ *                          H/128]: W13 and W2 transposed with their block
+ *                          scales (a layout step done once, like the weights'
+ *                          quantisation)
+ *   topk_idx, topk_w, slot_row: the forward's outputs
+ *   fwd_ws                  the workspace of that moe_forward call, unchanged
+ *                          since (it holds the quantised x and h rows, the
+ *                          expert outputs and the row maps)
+ *   ws                      scratch, moe_backward_workspace_size(cfg) bytes,
+ *                          256-byte aligned
+ * Contiguous layout, E4M3 weights and softmax routing only
+ * (MOE_ERR_UNSUPPORTED_SHAPE otherwise), I at most 8192, and at most 16384
+ * rows per expert (T, or the capacity when smaller).
+ */
+size_t moe_backward_workspace_size(const moe_config_t* cfg);
+moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const float* Wg, const uint8_t* W13, const float* S13,
+                          const uint8_t* W13T, const float* S13T, const uint8_t* W2T, const float* S2T,
+                          const int32_t* topk_idx, const float* topk_w, const int32_t* slot_row, const void* fwd_ws,
+                          const void* dy, void* dx, float* dWg, float* db, void* dW13, void* dW2, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /*
  * Auxiliary-loss-free load balancing. Source: MegaMoE page, section 2.2: each
