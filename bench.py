@@ -528,7 +528,12 @@ def run_ours(args):
     balance = {"us_per_call": 1e3 * b0.elapsed_time(b1) / 200, "calls": 200, "timing": "CUDA graph replay",
                "bytes_per_call": 28 * cfg.E, "bound": "launch latency (one block, 28 B per expert)"}
 
-    backward = time_backward(layer, cfg, max(3, min(args.steps, 20))) if args.backward else None
+    backward = None
+    if args.backward:
+        try:
+            backward = time_backward(layer, cfg, max(3, min(args.steps, 20)))
+        except Exception as exc:     # the forward line stands on its own; report the failure in its key
+            backward = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
     peaks, peak_src = load_peaks()
     hbm = float(peaks["hbm_gbs"])

@@ -91,7 +91,7 @@ def lib() -> ctypes.CDLL:
         L.moe_ep_return.argtypes = [I, I, P, P, P, P]
         L.moe_backward_workspace_size.argtypes = [CP]
         L.moe_backward_workspace_size.restype = SZ
-        L.moe_backward.argtypes = [CP] + [P] * 18 + [SZ, P]
+        L.moe_backward.argtypes = [CP] + [P] * 19 + [SZ, P]
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in EXPORTS:

@@ -639,10 +639,14 @@ constexpr int kWBlk = kBM * kBK;              // 16 KB: 128 weight rows x 128 K 
 // threads: warp 0 TMA, warp 1 MMA, then the promotion warps: four for SwiGLU (a thread holds a weight
 // row's 32 gate and 32 up columns), eight for the bf16 output (two warps per lane quadrant, 16 token
 // columns each, so two warps share each scheduler's promotion work)
-// With 4-bit weights (W4) four more warps, one per tensor-memory lane quadrant, expand each stage's packed
-// levels to E4M3 codes and write them into tensor memory, where the MMA reads its A operand.
+// With 4-bit weights (W4) more warps, one per tensor-memory lane quadrant and K-block parity, expand each
+// stage's packed levels to E4M3 codes and write them into tensor memory, where the MMA reads its A operand:
+// eight for the bf16 output (two sets of four take alternate K blocks, so one set's load, expansion and
+// store latency overlaps the other's), four for SwiGLU (whose promotion threads need the registers).
 template <int EPI, bool W4 = false>
-__host__ __device__ constexpr int masked_threads() { return (EPI == 1 ? 192 : 320) + (W4 ? 128 : 0); }
+__host__ __device__ constexpr int conv_warps() { return W4 ? (EPI == 1 ? 4 : 8) : 0; }
+template <int EPI, bool W4 = false>
+__host__ __device__ constexpr int masked_threads() { return (EPI == 1 ? 192 : 320) + 32 * conv_warps<EPI, W4>(); }
 
 __device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
@@ -718,7 +722,8 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     S& sm = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kPW = EPI == 1 ? 4 : 8;                      // promotion warps (2 .. 2 + kPW - 1)
-    constexpr int kConvWarp0 = 2 + kPW;                        // W4: converter warps, four of them
+    constexpr int kConvWarp0 = 2 + kPW;                        // W4: converter warps (conv_warps of them)
+    constexpr int kConvSets = conv_warps<EPI, W4>() / 4;       // sets of four, taking alternate K blocks
     const int KB = K / kBK;
     const int NB = N / kBM;                          // 128-row weight blocks per expert
     const int NBt = EPI == 1 ? NB / 2 : NB;          // weight tiles per expert
@@ -876,12 +881,14 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         // rows) go to registers, which frees the stage's levels; the 128 codes go to the row's 32 columns
         // of an A slot (64 for the gate and up blocks), whose completion the MMA waits on.
         const int q = warp & 3;
+        const int set = (warp - kConvWarp0) >> 2;          // this warp expands the K blocks it % kConvSets == set
         const int r = q * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         uint32_t it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb, ++it) {
+                if (kConvSets > 1 && static_cast<int>(it % kConvSets) != set) continue;
                 if (sm.abort_flag) { ok = false; break; }
                 const int s = it % S::kStages;
                 const uint32_t ph = (it / S::kStages) & 1;

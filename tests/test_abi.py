@@ -36,6 +36,25 @@ def test_every_declared_symbol_is_exported(L):
     assert set(names) == set(api.EXPORTS)
 
 
+def declared_arity():
+    """name -> number of parameters of each prototype in the header (MOE_EP_ROW_BYTES-style macros aside)."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(moe_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header(L):
+    # every ctypes prototype of the binding takes exactly the header's parameters
+    arity = declared_arity()
+    assert set(arity) == set(api.EXPORTS)
+    for name, n in arity.items():
+        assert len(getattr(L, name).argtypes) == n, name
+
+
 def test_status_strings(L):
     for code in range(8):
         assert api.status_string(code)
