@@ -330,10 +330,12 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             int ok = 1;
             if (lane == 0) ok = !sm.abort_flag && mbar_wait(&sm.wempty[ws], ((ti >> 1) & 1) ^ 1, wait_ns);
             if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+            // K-grouped tiles have their own K block count (at most kMaxKB; read_scales zeroed the rest)
+            const int lim = KG ? kMaxKB : KB;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int kb = lane + 32 * i;
-                if (kb < KB) {
+                if (kb < lim) {
                     sm.wsc[ws][0][kb] = wr0[i];
                     sm.wsc[ws][1][kb] = wr1[i];
                 }

@@ -25,12 +25,16 @@ def _inputs(cfg, seed=0):
 
 
 CFG = MoeConfig("bwd", T=96, H=256, E=4, I=256, k=2, bias="zipf", cap_num=1, cap_den=1, seed=3)
+# experts of up to three 128-row tiles (several K blocks in the weight-gradient sums) and a ragged 384-wide H
+CFG_TILES = MoeConfig("bwd_tiles", T=600, H=384, E=8, I=256, k=4, bias="uniform", cap_num=1, cap_den=1, seed=4)
+_CFGS = {"small": CFG, "tiles": CFG_TILES}
 
 
-@pytest.fixture(scope="module")
-def bwd():
-    inp, d, dy = _inputs(CFG)
-    return CFG, inp, d, dy, oracle.backward(CFG, d, dy)
+@pytest.fixture(scope="module", params=list(_CFGS))
+def bwd(request):
+    cfg = _CFGS[request.param]
+    inp, d, dy = _inputs(cfg)
+    return cfg, inp, d, dy, oracle.backward(cfg, d, dy)
 
 
 def test_router_gradients_equal_autograd(bwd):
@@ -124,11 +128,19 @@ def test_whole_backward_within_fp8_error_of_unquantised_autograd(bwd):
         return np.linalg.norm(got - want) / np.linalg.norm(want)
 
     bf = lambda a: oracle.bf16_bits_to_f32(a)
-    assert rel(bf(r["dx"]), x.grad.numpy()) < 0.06
-    assert rel(r["dWg"], Wg.grad.numpy()) < 0.06
-    assert rel(r["db"], b.grad.numpy()) < 0.06
+    if cfg is CFG_TILES:
+        assert int(np.max(f["kept"])) > 256                   # some expert spans three row tiles
+    # E4M3 keeps 3 mantissa bits (a rounding error of up to 1/16 of each value): the FP8 forward's y sits
+    # about 4.5 % from the unquantised layer, and every backward product adds one or two more quantised
+    # operands. db sums signed per-token terms that largely cancel, so its error is that of the terms.
+    # 0.1 holds all of this; a dropped term, a swapped operand or a wrong sign gives errors near 1.
+    tol = 0.1
+    assert rel(bf(f["y"]), y.detach().numpy()) < 0.06
+    assert rel(bf(r["dx"]), x.grad.numpy()) < tol
+    assert rel(r["dWg"], Wg.grad.numpy()) < tol
+    assert rel(r["db"], b.grad.numpy()) < tol
     for e in range(E):
         dW13 = bf(r["dW13"][e]).reshape(I // 128, 2, 128, H)
-        assert rel(dW13[:, 0].reshape(I, H), W1[e].grad.numpy()) < 0.06, e
-        assert rel(dW13[:, 1].reshape(I, H), W3[e].grad.numpy()) < 0.06, e
-        assert rel(bf(r["dW2"][e]), W2[e].grad.numpy()) < 0.06, e
+        assert rel(dW13[:, 0].reshape(I, H), W1[e].grad.numpy()) < tol, e
+        assert rel(dW13[:, 1].reshape(I, H), W3[e].grad.numpy()) < tol, e
+        assert rel(bf(r["dW2"][e]), W2[e].grad.numpy()) < tol, e
