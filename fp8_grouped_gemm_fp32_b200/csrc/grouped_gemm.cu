@@ -890,7 +890,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb, ++it) {
-                if (kConvSets > 1 && static_cast<int>(it % kConvSets) != set) continue;
+                if (kConvSets > 1 && static_cast<int>(it % (kConvSets > 1 ? kConvSets : 1)) != set) continue;
                 if (sm.abort_flag) { ok = false; break; }
                 const int s = it % S::kStages;
                 const uint32_t ph = (it / S::kStages) & 1;
