@@ -224,7 +224,9 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStagesC; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 1);
+            // a stage is free once this CTA's eight promotion warps have seen its K block's accumulator
+            // complete (the MMA commits once per K block, to the accumulator buffer only)
+            mbar_init(&sm.empty[s], 8);
         }
         for (int j = 0; j < kSaSlots; ++j) {
             mbar_init(&sm.sfull[j], 1);
@@ -429,14 +431,12 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         for (int kk = 0; kk < kBK / 32; ++kk)
                             umma_f8_pair(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc,
                                          kk > 0);
-                        umma_commit_pair(&sm.empty[s], 0x3);     // both CTAs' stage s is free again
                         umma_commit_pair(&sm.tfull[buf], 0x3);   // both CTAs' accumulator buffer is ready
                     } else {
 #pragma unroll
                         for (int kk = 0; kk < kBK / 32; ++kk)
                             umma_f8(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc,
                                     kk > 0);
-                        umma_commit(&sm.empty[s]);
                         umma_commit(&sm.tfull[buf]);
                     }
                 }
@@ -481,6 +481,9 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const float f0 = sa * w0;
                 const float f1 = sa * w1;
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
+                // the K block's MMAs are done, so its operand stage (this CTA's; in a pair the leader's MMA
+                // read both CTAs' stages, and the commit reached both) can be refilled
+                if (lane == 0) mbar_arrive(&sm.empty[kbt % kStagesC]);
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * kBN + half * 64;
                 // The buffer is handed back to the MMA warp as soon as the last of its columns is in
@@ -678,7 +681,9 @@ struct SmemM {
     static constexpr int kBufs = 4;                            // MMA runs up to 3 K blocks ahead of promotion
     static constexpr int kSaSlots = 16;                        // scale ring deeper than the stage ring
     static constexpr int kACols = kW / kBM / 4;                // W4: tensor-memory columns of one A slot (32 or 64)
-    static constexpr int kA = W4 ? (EPI == 1 ? 4 : 8) : 1;     // W4: A slots after the accumulators
+    // W4: A slots after the accumulators, as many as the accumulator buffers: the MMA of K block j uses
+    // slot and buffer j % 4, so the buffer's completion also frees the slot
+    static constexpr int kA = W4 ? kBufs : 1;
     static constexpr uint32_t kTmemCols = W4 ? 512u : static_cast<uint32_t>(kBufs * kCols);
     static_assert(!W4 || kBufs * kCols + kA * kACols <= 512, "tensor memory holds the accumulators and A slots");
     alignas(1024) uint8_t x[kStages][kXBytes];                  // 128-byte swizzled tiles: 1024-byte aligned
@@ -692,7 +697,6 @@ struct SmemM {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t afull[kA];                                         // W4: A slot written by the converter warps
-    uint64_t aempty[kA];                                        // W4: A slot read by the MMA
     uint64_t sfull[kSaSlots];
     uint64_t sempty[kSaSlots];
     uint64_t tfull[kBufs];
@@ -757,12 +761,12 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     if (threadIdx.x == 32) {
         for (int s = 0; s < S::kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            // W4: a stage is free once the MMA has read its token tile and the four converter warps its levels
-            mbar_init(&sm.empty[s], W4 ? 5 : 1);
+            // a stage is free once the promotion warps have seen its K block's accumulator complete (the MMA
+            // has read its token tile) and, W4, the four converter warps have read its levels
+            mbar_init(&sm.empty[s], W4 ? 4 + kPW : kPW);
         }
         for (int a = 0; a < S::kA; ++a) {
             mbar_init(&sm.afull[a], 4);
-            mbar_init(&sm.aempty[a], 1);
         }
         for (int j = 0; j < S::kSaSlots; ++j) {
             mbar_init(&sm.sfull[j], 1);
@@ -861,7 +865,6 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                             umma_f8_ta(d, a0 + kk * 8, xd, idesc, kk > 0);
                             if (EPI == 1) umma_f8_ta(d + kBT, a0 + 32 + kk * 8, xd, idesc, kk > 0);
                         }
-                        umma_commit(&sm.aempty[a]);
                     } else {
                         const uint32_t w0 = smem_u32(sm.w[s]);
 #pragma unroll
@@ -871,8 +874,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                             if (EPI == 1) umma_f8(d + kBT, sw128_kmajor_desc(w0 + kWBlk + kk * 32), xd, idesc, kk > 0);
                         }
                     }
-                    umma_commit(&sm.empty[s]);
-                    umma_commit(&sm.tfull[buf]);
+                    umma_commit(&sm.tfull[buf]);     // the one commit of the K block
                 }
             }
         }
@@ -905,7 +907,8 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                                                                    ((c ^ ((r >> 1) & 3)) << 4));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.empty[s]);
-                if (!mbar_wait(&sm.aempty[a], ((it / S::kA) & 1) ^ 1, wait_ns)) { fail(); ok = false; break; }
+                // slot a was last read by the MMA of K block it - kA, whose accumulator buffer is a
+                if (!mbar_wait(&sm.tfull[a], ((it / S::kA) & 1) ^ 1, wait_ns)) { fail(); ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int b = 0; b < (EPI == 1 ? 2 : 1); ++b) {
@@ -988,6 +991,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                                    : 0.0f;
                 }
                 if (!mbar_wait(&sm.tfull[buf], bph, wait_ns)) { fail(); ok = false; break; }
+                if (lane == 0) mbar_arrive(&sm.empty[kbt % S::kStages]);     // the MMA has read the stage
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * S::kCols;
                 if constexpr (EPI == 0) {
