@@ -33,8 +33,8 @@ WEIGHTS_FP8, WEIGHTS_W4 = 0, 1
 EXPORTS = ("moe_rows_capacity", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_gemm_fp8",
            "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string",
            "moe_permute_noalloc", "moe_balance_bias", "moe_grouped_gemm_w4", "moe_set_contig_kernel",
-           "moe_ep_plan", "moe_ep_workspace_size", "moe_ep_count", "moe_ep_dispatch", "moe_ep_receive",
-           "moe_ep_return", "moe_backward_workspace_size", "moe_backward")
+           "moe_ep_plan", "moe_ep_plan_chunked", "moe_ep_workspace_size", "moe_ep_count", "moe_ep_dispatch",
+           "moe_ep_receive", "moe_ep_receive_chunk", "moe_ep_return", "moe_backward_workspace_size", "moe_backward")
 
 
 class MoeError(RuntimeError):
@@ -83,11 +83,13 @@ def lib() -> ctypes.CDLL:
         L.moe_selftest_wait_timeout.argtypes = [I, P]
         L.moe_set_contig_kernel.argtypes = [I]
         L.moe_ep_plan.argtypes = [I, I, I, ctypes.c_int64, I, I, I, P, P]
+        L.moe_ep_plan_chunked.argtypes = [I, I, I, ctypes.c_int64, I, I, I, P, I, P]
         L.moe_ep_workspace_size.argtypes = [CP]
         L.moe_ep_workspace_size.restype = SZ
         L.moe_ep_count.argtypes = [CP, P, P, P, SZ, P]
         L.moe_ep_dispatch.argtypes = [CP, P, P, P, P, P, P, SZ, P]
         L.moe_ep_receive.argtypes = [I, P, I, P, P, P, I, P, P, P]
+        L.moe_ep_receive_chunk.argtypes = [I, P, I, P, P, P, I, P, P, P]
         L.moe_ep_return.argtypes = [I, I, P, P, P, P]
         L.moe_backward_workspace_size.argtypes = [CP]
         L.moe_backward_workspace_size.restype = SZ
@@ -221,6 +223,11 @@ def moe_ep_dispatch(cfg, x, topk_idx, plan_dev, send, slot_row, ws, stream=None)
 def moe_ep_receive(H, plan_dev, rows_recv, recv, Aq, As, M_rows, offsets, group_row, stream=None):
     _check(lib().moe_ep_receive(H, _p(plan_dev), rows_recv, _p(recv) if rows_recv else None, _p(Aq), _p(As), M_rows,
                                 _p(offsets), _p(group_row), _stream(stream)), "moe_ep_receive")
+
+
+def moe_ep_receive_chunk(H, plan_dev, chunk, recv, Aq, As, M_rows, offsets, group_row, stream=None):
+    _check(lib().moe_ep_receive_chunk(H, _p(plan_dev), chunk, _p(recv), _p(Aq), _p(As), M_rows, _p(offsets),
+                                      _p(group_row), _stream(stream)), "moe_ep_receive_chunk")
 
 
 def moe_ep_return(H, rows_recv, O, group_row, ret, stream=None):

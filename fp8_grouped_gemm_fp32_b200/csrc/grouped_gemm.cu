@@ -669,15 +669,18 @@ __device__ __forceinline__ void w4x8_to_e4m3x8(uint32_t w, uint32_t& lo, uint32_
     hi = prmt_b32(0x44403800u, 0x4e4c4a48u, (w >> 16) & 0x7777u) | ((w << 4) & 0x80808080u);
 }
 
-template <int EPI, bool W4 = false>
+// WIDE (bf16 output only): a tile takes two consecutive 128-row weight blocks, so that each K block's fixed
+// cost (barriers, the commit, the promotion round trip) is spread over twice the weight bytes.
+template <int EPI, bool W4 = false, bool WIDE = false>
 struct SmemM {
-    static constexpr int kW = EPI == 1 ? 2 * kWBlk : kWBlk;    // weight bytes per stage: 256 rows (a|b) or 128
+    static constexpr bool kTwo = EPI == 1 || WIDE;              // two 128-row weight blocks per tile
+    static constexpr int kW = kTwo ? 2 * kWBlk : kWBlk;        // weight bytes per stage: 256 rows (a|b, or two) or 128
     // W4: a deep ring of packed stages (8 or 16 KB of levels + the 4 KB token tile each); the expanded
     // codes live in tensor memory (kA slots) instead of shared memory
-    static constexpr int kStages = W4 ? (EPI == 1 ? 8 : 16) : (EPI == 1 ? 4 : 10);
+    static constexpr int kStages = W4 ? (kTwo ? 8 : 16) : (EPI == 1 ? 4 : WIDE ? 5 : 10);
     static constexpr int kWS = W4 ? 16 : kW;                   // expanded codes in shared memory (FP8 only)
     static constexpr int kWP = W4 ? kW / 2 : 16;               // packed 4-bit levels per stage (W4 only)
-    static constexpr int kCols = EPI == 1 ? 2 * kBT : kBT;     // tensor-memory columns per accumulator buffer
+    static constexpr int kCols = kTwo ? 2 * kBT : kBT;         // tensor-memory columns per accumulator buffer
     static constexpr int kBufs = 4;                            // MMA runs up to 3 K blocks ahead of promotion
     static constexpr int kSaSlots = 16;                        // scale ring deeper than the stage ring
     static constexpr int kACols = kW / kBM / 4;                // W4: tensor-memory columns of one A slot (32 or 64)
@@ -714,16 +717,19 @@ static_assert(sizeof(SmemC<0, false>) + 1024 <= kSmemLimit && sizeof(SmemC<1, fa
               sizeof(SmemC<0, true>) + 1024 <= kSmemLimit && sizeof(SmemC<1, true>) + 1024 <= kSmemLimit,
               "contiguous kernel shared memory");
 static_assert(sizeof(SmemM<0, false>) + 1024 <= kSmemLimit && sizeof(SmemM<1, false>) + 1024 <= kSmemLimit &&
-              sizeof(SmemM<0, true>) + 1024 <= kSmemLimit && sizeof(SmemM<1, true>) + 1024 <= kSmemLimit,
+              sizeof(SmemM<0, true>) + 1024 <= kSmemLimit && sizeof(SmemM<1, true>) + 1024 <= kSmemLimit &&
+              sizeof(SmemM<0, false, true>) + 1024 <= kSmemLimit && sizeof(SmemM<0, true, true>) + 1024 <= kSmemLimit,
               "masked kernel shared memory");
 
-template <int EPI, bool W4>
+template <int EPI, bool W4, bool WIDE = false>
 __global__ void __launch_bounds__(masked_threads<EPI, W4>(), 1)
 gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ As, const int32_t* __restrict__ masked_m, int Mmax,
                  const float* __restrict__ Bs, int E, int N, int K, void* __restrict__ D, float* __restrict__ Ds,
                  int* status, uint64_t wait_ns) {
-    using S = SmemM<EPI, W4>;
+    static_assert(!WIDE || EPI == 0, "two output blocks per tile: bf16 epilogue only");
+    using S = SmemM<EPI, W4, WIDE>;
+    constexpr bool kTwo = S::kTwo;
     extern __shared__ uint8_t smem_raw[];
     S& sm = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -732,7 +738,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     constexpr int kConvSets = conv_warps<EPI, W4>() / 4;       // sets of four, taking alternate K blocks
     const int KB = K / kBK;
     const int NB = N / kBM;                          // 128-row weight blocks per expert
-    const int NBt = EPI == 1 ? NB / 2 : NB;          // weight tiles per expert
+    const int NBt = kTwo ? NB / 2 : NB;              // weight tiles per expert
     constexpr uint32_t kTmemCols = S::kTmemCols;
     constexpr uint32_t kA0 = S::kBufs * S::kCols;              // W4: first column of the A slots
 
@@ -811,7 +817,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             for (int tile = blockIdx.x; tile < total && !sm.abort_flag; tile += gridDim.x) {
                 int e, nb, tt, m_e;
                 decode(tile, e, nb, tt, m_e);
-                const int wrow = e * N + nb * (EPI == 1 ? 2 * kBM : kBM);
+                const int wrow = e * N + nb * (kTwo ? 2 * kBM : kBM);
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % S::kStages;
                     const uint32_t ph = (it / S::kStages) & 1;
@@ -819,11 +825,11 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     if constexpr (W4) {
                         mbar_arrive_expect_tx(&sm.full[s], S::kWP + kXBytes);
                         tma_load_2d(sm.wp[s], &tmW, &sm.full[s], kb * (kBK / 2), wrow);
-                        if (EPI == 1) tma_load_2d(sm.wp[s] + kWBlk / 2, &tmW, &sm.full[s], kb * (kBK / 2), wrow + kBM);
+                        if (kTwo) tma_load_2d(sm.wp[s] + kWBlk / 2, &tmW, &sm.full[s], kb * (kBK / 2), wrow + kBM);
                     } else {
                         mbar_arrive_expect_tx(&sm.full[s], S::kW + kXBytes);
                         tma_load_2d(sm.w[s], &tmW, &sm.full[s], kb * kBK, wrow);
-                        if (EPI == 1) tma_load_2d(sm.w[s] + kWBlk, &tmW, &sm.full[s], kb * kBK, wrow + kBM);
+                        if (kTwo) tma_load_2d(sm.w[s] + kWBlk, &tmW, &sm.full[s], kb * kBK, wrow + kBM);
                     }
                     tma_load_2d(sm.x[s], &tmX, &sm.full[s], kb * kBK, e * Mmax + tt * kBT);
                     // the token tile's 32 activation scales of this K block, into the scale ring
@@ -863,7 +869,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                         for (int kk = 0; kk < kBK / 32; ++kk) {
                             const uint64_t xd = sw128_kmajor_desc(x0 + kk * 32);
                             umma_f8_ta(d, a0 + kk * 8, xd, idesc, kk > 0);
-                            if (EPI == 1) umma_f8_ta(d + kBT, a0 + 32 + kk * 8, xd, idesc, kk > 0);
+                            if (kTwo) umma_f8_ta(d + kBT, a0 + 32 + kk * 8, xd, idesc, kk > 0);
                         }
                     } else {
                         const uint32_t w0 = smem_u32(sm.w[s]);
@@ -871,7 +877,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                         for (int kk = 0; kk < kBK / 32; ++kk) {
                             const uint64_t xd = sw128_kmajor_desc(x0 + kk * 32);
                             umma_f8(d, sw128_kmajor_desc(w0 + kk * 32), xd, idesc, kk > 0);
-                            if (EPI == 1) umma_f8(d + kBT, sw128_kmajor_desc(w0 + kWBlk + kk * 32), xd, idesc, kk > 0);
+                            if (kTwo) umma_f8(d + kBT, sw128_kmajor_desc(w0 + kWBlk + kk * 32), xd, idesc, kk > 0);
                         }
                     }
                     umma_commit(&sm.tfull[buf]);     // the one commit of the K block
@@ -898,9 +904,9 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 const uint32_t ph = (it / S::kStages) & 1;
                 const int a = it % S::kA;
                 if (!mbar_wait(&sm.full[s], ph, wait_ns)) { fail(); ok = false; break; }
-                uint4 pk[EPI == 1 ? 2 : 1][4];
+                uint4 pk[kTwo ? 2 : 1][4];
 #pragma unroll
-                for (int b = 0; b < (EPI == 1 ? 2 : 1); ++b)
+                for (int b = 0; b < (kTwo ? 2 : 1); ++b)
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
                         pk[b][c] = *reinterpret_cast<const uint4*>(sm.wp[s] + b * (kWBlk / 2) + r * (kBK / 2) +
@@ -911,7 +917,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 if (!mbar_wait(&sm.tfull[a], ((it / S::kA) & 1) ^ 1, wait_ns)) { fail(); ok = false; break; }
                 tc_fence_after();
 #pragma unroll
-                for (int b = 0; b < (EPI == 1 ? 2 : 1); ++b) {
+                for (int b = 0; b < (kTwo ? 2 : 1); ++b) {
                     uint32_t codes[32];
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
@@ -943,12 +949,12 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             if (tile >= total) return;
             int e, nb, tt, m_e;
             decode(tile, e, nb, tt, m_e);
-            const float* pa = Bs + (static_cast<int64_t>(e) * NB + (EPI == 1 ? 2 * nb : nb)) * KB;
+            const float* pa = Bs + (static_cast<int64_t>(e) * NB + (kTwo ? 2 * nb : nb)) * KB;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int kb = lane + 32 * i;
                 wa[i] = kb < KB ? pa[kb] : 0.0f;
-                wb[i] = EPI == 1 && kb < KB ? pa[KB + kb] : 0.0f;
+                wb[i] = kTwo && kb < KB ? pa[KB + kb] : 0.0f;
             }
         };
         if constexpr (!W4) load_w(blockIdx.x);
@@ -956,9 +962,11 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             if (sm.abort_flag) break;
             int e, nb, tt, m_e;
             decode(tile, e, nb, tt, m_e);
-            float acc[EPI == 1 ? 2 * kBT : kC];
+            // EPI 1: 32 gate then 32 up token columns; EPI 0: kC token columns of each weight block
+            constexpr int kAcc = EPI == 1 ? 2 * kBT : (WIDE ? 2 * kC : kC);
+            float acc[kAcc];
 #pragma unroll
-            for (int i = 0; i < (EPI == 1 ? 2 * kBT : kC); ++i) acc[i] = 0.0f;
+            for (int i = 0; i < kAcc; ++i) acc[i] = 0.0f;
             const float wta[4] = {wa[0], wa[1], wa[2], wa[3]};
             const float wtb[4] = {wb[0], wb[1], wb[2], wb[3]};
             if constexpr (!W4) load_w(tile + gridDim.x);
@@ -978,7 +986,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 float swa, swb;
                 if constexpr (W4) {            // this thread's weight row (and its up row) scale for the K block
                     swa = sm.wrs[j][r];
-                    swb = EPI == 1 ? sm.wrs[j][kBM + r] : 0.0f;
+                    swb = kTwo ? sm.wrs[j][kBM + r] : 0.0f;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.sempty[j]);
@@ -986,7 +994,7 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     const int wi = kb >> 5;
                     swa = __shfl_sync(0xffffffffu, wi == 0 ? wta[0] : wi == 1 ? wta[1] : wi == 2 ? wta[2] : wta[3],
                                       kb & 31);
-                    swb = EPI == 1 ? __shfl_sync(0xffffffffu, wi == 0 ? wtb[0] : wi == 1 ? wtb[1]
+                    swb = kTwo ? __shfl_sync(0xffffffffu, wi == 0 ? wtb[0] : wi == 1 ? wtb[1]
                                                               : wi == 2 ? wtb[2] : wtb[3], kb & 31)
                                    : 0.0f;
                 }
@@ -995,11 +1003,16 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * S::kCols;
                 if constexpr (EPI == 0) {
-                    float v[16];
+                    float v[16], v2[16];
                     tmem_ld16(taddr + cof, v);
+                    if constexpr (WIDE) tmem_ld16(taddr + kBT + cof, v2);
                     tmem_ld_wait();
 #pragma unroll
                     for (int c = 0; c < kC; ++c) acc[c] = fmaf(v[c], sa[c] * swa, acc[c]);
+                    if constexpr (WIDE) {
+#pragma unroll
+                        for (int c = 0; c < kC; ++c) acc[kC + c] = fmaf(v2[c], sa[c] * swb, acc[kC + c]);
+                    }
                 } else {
                     float v[32];
                     tmem_ld32(taddr, v);
@@ -1022,10 +1035,14 @@ gg_masked_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const int nv = min(kBT, m_e - tt * kBT);       // valid tokens in this tile
             const int64_t row0 = static_cast<int64_t>(e) * Mmax + tt * kBT;
             if constexpr (EPI == 0) {
-                uint16_t* out = static_cast<uint16_t*>(D) + (row0 + cof) * N + nb * kBM + r;
+                uint16_t* out = static_cast<uint16_t*>(D) + (row0 + cof) * N + nb * (WIDE ? 2 * kBM : kBM) + r;
 #pragma unroll
                 for (int c = 0; c < kC; ++c)
-                    if (cof + c < nv) out[static_cast<int64_t>(c) * N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[c]));
+                    if (cof + c < nv) {
+                        out[static_cast<int64_t>(c) * N] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[c]));
+                        if constexpr (WIDE)
+                            out[static_cast<int64_t>(c) * N + kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[kC + c]));
+                    }
             } else {
                 const int I = N / 2;
                 const int p = ep & 1;
@@ -1211,7 +1228,13 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
     } else {
         if (!make_map(&mapA, A, K, static_cast<uint64_t>(E) * M_rows, kBT)) return cudaErrorInvalidValue;
         if (!make_map(&mapB, B, K, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
-        if (epilogue == 0) {
+        if (epilogue == 0 && N % (2 * kBM) == 0) {
+            const size_t smem = sizeof(SmemM<0, false, true>) + 1024;
+            cudaError_t err = set_smem(gg_masked_kernel<0, false, true>, smem);
+            if (err != cudaSuccess) return err;
+            gg_masked_kernel<0, false, true><<<num_sms, masked_threads<0>(), smem, s>>>(
+                mapA, mapB, As, group_info, M_rows, Bs, E, N, K, D, Ds, status, wait_ns);
+        } else if (epilogue == 0) {
             const size_t smem = sizeof(SmemM<0>) + 1024;
             cudaError_t err = set_smem(gg_masked_kernel<0, false>, smem);
             if (err != cudaSuccess) return err;
@@ -1250,7 +1273,13 @@ cudaError_t launch_grouped_gemm_w4(int E, int N, int K, const uint8_t* A, const 
     CUtensorMap mapA, mapB;
     if (!make_map(&mapA, A, K, static_cast<uint64_t>(E) * M_rows, kBT)) return cudaErrorInvalidValue;
     if (!make_packed_map(&mapB, B, K / 2, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
-    if (epilogue == 0) {
+    if (epilogue == 0 && N % (2 * kBM) == 0) {
+        const size_t smem = sizeof(SmemM<0, true, true>) + 1024;
+        cudaError_t err = set_smem(gg_masked_kernel<0, true, true>, smem);
+        if (err != cudaSuccess) return err;
+        gg_masked_kernel<0, true, true><<<num_sms, masked_threads<0, true>(), smem, s>>>(
+            mapA, mapB, As, masked_m, M_rows, Bs, E, N, K, D, Ds, status, wait_ns);
+    } else if (epilogue == 0) {
         const size_t smem = sizeof(SmemM<0, true>) + 1024;
         cudaError_t err = set_smem(gg_masked_kernel<0, true>, smem);
         if (err != cudaSuccess) return err;

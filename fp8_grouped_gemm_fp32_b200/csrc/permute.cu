@@ -190,11 +190,13 @@ __device__ __forceinline__ GroupCodes quantise_group(uint4 raw, float amax) {
 // blockIdx.x < nchunks: the slot maps of one 32-token chunk (slot_row, row_src);
 // blockIdx.x >= nchunks (contiguous layout only): the padding rows of one expert, one slice of
 // pad_slices of its 128-groups (codes 0, scale 1, row_src -1). Block 0 also writes offsets.
+// row_base (nullable): each expert's first row, in place of the scan of kept (an expert-parallel
+// plan's send rows, which run in chunk order).
 __global__ void __launch_bounds__(256) permute_map_kernel(
     const int32_t* __restrict__ topk_idx, int T, int H, int k, int E, int nchunks, int pad, int pad_slices,
     int masked_max_m, int ld_rows, const int32_t* __restrict__ base, const int32_t* __restrict__ kept,
     uint8_t* __restrict__ Aq, float* __restrict__ As, int32_t* __restrict__ offsets, int32_t* __restrict__ row_src,
-    int32_t* __restrict__ slot_row) {
+    int32_t* __restrict__ slot_row, const int32_t* __restrict__ row_base) {
     extern __shared__ int32_t sm[];
     int32_t* off_s = sm;                    // [E + 1]
     int32_t* kept_s = off_s + (E + 1);      // [E]
@@ -203,6 +205,10 @@ __global__ void __launch_bounds__(256) permute_map_kernel(
     const int G = H / kGroup;
 
     group_offsets(kept, E, masked_max_m, pad, off_s, kept_s);
+    if (row_base) {
+        for (int e = tid; e < E; e += blockDim.x) off_s[e] = row_base[e];
+        __syncthreads();
+    }
     if (blockIdx.x == 0 && offsets)
         for (int e = tid; e <= E; e += blockDim.x) offsets[e] = off_s[e];
 
@@ -353,7 +359,7 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, int T, in
     const int gx = nchunks + (masked_max_m > 0 ? 0 : E * pad_slices);
     const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1);
     permute_map_kernel<<<gx, 256, smem, s>>>(topk_idx, T, H, k, E, nchunks, kGroup, pad_slices, masked_max_m, ld_rows,
-                                             base, kept, Aq, As, offsets, row_src, slot_row);
+                                             base, kept, Aq, As, offsets, row_src, slot_row, nullptr);
     // one warp per (token, 8-group slice); enough blocks to keep every SM full, striding beyond that
     const int64_t warps = static_cast<int64_t>(T) * ((G + 7) / 8);
     int per_sm = 0;
@@ -395,7 +401,7 @@ cudaError_t launch_slot_lists(const int32_t* topk_idx, int T, int k, int E, int3
     permute_scan_kernel<<<E, 256, 0, s>>>(cnt, nchunks, -1, 0, base, counts, unused_kept, status);
     const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1);
     permute_map_kernel<<<nchunks, 256, smem, s>>>(topk_idx, T, 0, k, E, nchunks, 1, 1, 0, 0, base, counts, nullptr,
-                                                  nullptr, offsets, list, slot_tmp);
+                                                  nullptr, offsets, list, slot_tmp, nullptr);
     return cudaGetLastError();
 }
 
@@ -408,13 +414,13 @@ int64_t ep_row_bytes(int H) { return (static_cast<int64_t>(H) + 4 * (H / kGroup)
 // ranks exactly as the capacity does in moe_permute; rows are unpadded (pad 1), in expert order, which
 // is destination-rank order since each rank's experts are contiguous.
 cudaError_t launch_ep_dispatch(const uint16_t* x, const int32_t* topk_idx, int T, int H, int k, int E,
-                               const int32_t* kept_mine, uint8_t* send, int32_t* slot_row, void* scratch,
-                               int num_sms, cudaStream_t s) {
+                               const int32_t* kept_mine, const int32_t* send_off, uint8_t* send, int32_t* slot_row,
+                               void* scratch, int num_sms, cudaStream_t s) {
     const int nchunks = (T + kChunk - 1) / kChunk;
     int32_t* base = static_cast<int32_t*>(scratch) + static_cast<size_t>(nchunks) * E;
     const size_t smem = sizeof(int32_t) * (3 * static_cast<size_t>(E) + 1);
     permute_map_kernel<<<nchunks, 256, smem, s>>>(topk_idx, T, H, k, E, nchunks, 1, 1, 0, 0, base, kept_mine,
-                                                  nullptr, nullptr, nullptr, nullptr, slot_row);
+                                                  nullptr, nullptr, nullptr, nullptr, slot_row, send_off);
     const int G = H / kGroup;
     const int64_t warps = static_cast<int64_t>(T) * ((G + 7) / 8);
     int per_sm = 0;

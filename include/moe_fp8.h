@@ -398,8 +398,22 @@ moe_status_t moe_selftest_wait_timeout(int limit_us, void* stream);
  *
  * A send/receive row is H bytes of E4M3 codes followed by H/128 fp32 scales,
  * padded to a multiple of 16 bytes (row stride MOE_EP_ROW_BYTES(H)).
+ *
+ * Chunked overlap (MegaMoE page, section 2.3: with the work cut into C chunks
+ * of compute time T_comp and exchange time T_comm each, the exchange of one
+ * chunk runs while another is computed, and a step takes T_comp + T_comm +
+ * (C - 1) max(T_comp, T_comm) instead of C (T_comp + T_comm)): a
+ * plan made with C chunks (moe_ep_plan_chunked) splits every rank's local
+ * experts into C consecutive groups and orders the send and receive rows by
+ * chunk first, so that chunk c is one contiguous slice of each buffer, with its
+ * own per-rank row counts. The caller then runs, per chunk, the all-to-all of
+ * its slice, moe_ep_receive_chunk, the two grouped GEMMs on the chunk's experts
+ * (pointer offsets into the grouped layout, offsets from moe_ep_receive_chunk)
+ * and moe_ep_return on its rows, with the collectives on a stream of their own;
+ * results equal those of C = 1 bit for bit.
  */
 #define MOE_EP_MAX_RANKS 64
+#define MOE_EP_MAX_CHUNKS 8
 #define MOE_EP_ROW_BYTES(H) (((size_t)(H) + 4u * ((size_t)(H) / 128u) + 15u) / 16u * 16u)
 
 /* The exchange plan of one rank (host memory; the device steps read a device
@@ -413,10 +427,19 @@ typedef struct {
     int32_t kept_mine[MOE_MAX_EXPERTS];      /* per expert e: this rank's slots of e kept */
     int32_t send_rows[MOE_EP_MAX_RANKS];     /* rows for each destination rank */
     int32_t recv_rows[MOE_EP_MAX_RANKS];     /* rows from each source rank */
-    int32_t recv_start[MOE_MAX_EXPERTS + 1]; /* block b = s * E_local + e_loc: first receive row */
+    /* blocks (source s, local expert l) in receive order, which is (chunk, s, l, token): with one chunk
+     * block b = s * E_local + l */
+    int32_t recv_start[MOE_MAX_EXPERTS + 1]; /* block b: first receive row; [G * E_local] = rows_recv */
     int32_t group_start[MOE_MAX_EXPERTS];    /* block b: its first row in the grouped layout */
     int32_t offsets[MOE_MAX_EXPERTS + 1];    /* grouped layout of the local experts, multiples of 128 */
     int32_t kept[MOE_MAX_EXPERTS];           /* rows of each local expert (all sources) */
+    int32_t chunks;                                     /* C, 1 .. MOE_EP_MAX_CHUNKS */
+    int32_t chunk_first[MOE_EP_MAX_CHUNKS + 1];         /* chunk c = local experts [chunk_first[c], [c+1]) */
+    int32_t send_off[MOE_MAX_EXPERTS];                  /* per expert e: its first send row */
+    int32_t send_chunk[MOE_EP_MAX_CHUNKS + 1];          /* first send row of each chunk */
+    int32_t recv_chunk[MOE_EP_MAX_CHUNKS + 1];          /* first receive row of each chunk */
+    int32_t send_rows_c[MOE_EP_MAX_CHUNKS][MOE_EP_MAX_RANKS];   /* chunk c: rows for each destination */
+    int32_t recv_rows_c[MOE_EP_MAX_CHUNKS][MOE_EP_MAX_RANKS];   /* chunk c: rows from each source */
 } moe_ep_plan_t;
 
 /* Host-only, no GPU needed. counts_all [G][E] int32 (host): counts_all[s][e] =
@@ -427,9 +450,15 @@ typedef struct {
  * order, so rank s keeps clamp(C - sum_{s' < s} counts_all[s'][e], 0,
  * counts_all[s][e]). Errors: G outside 1..MOE_EP_MAX_RANKS, E not a multiple
  * of G or above MOE_MAX_EXPERTS, rank outside [0, G), negative counts,
- * MOE_ERR_UNSUPPORTED_SHAPE when a row count would pass 2^31 / 128. */
+ * MOE_ERR_UNSUPPORTED_SHAPE when a row count would pass 2^31 / 128. Send rows
+ * are ordered by chunk, destination rank, expert, token; received rows by
+ * chunk, source rank, local expert, token. moe_ep_plan is the one-chunk plan. */
 moe_status_t moe_ep_plan(int G, int rank, int E, int64_t T_total, int k, int cap_num, int cap_den,
                          const int32_t* counts_all, moe_ep_plan_t* plan);
+/* chunks: 1 .. min(MOE_EP_MAX_CHUNKS, E / G) (MOE_ERR_INVALID_ARG otherwise); chunk c holds local experts
+ * [c E_local / C, (c + 1) E_local / C). */
+moe_status_t moe_ep_plan_chunked(int G, int rank, int E, int64_t T_total, int k, int cap_num, int cap_den,
+                                 const int32_t* counts_all, int chunks, moe_ep_plan_t* plan);
 
 /* Per-expert counts of this rank's slots: counts [E] int32 out. cfg as for
  * moe_route on this rank's batch (cfg->T its tokens; capacity fields unused
@@ -447,17 +476,31 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const void* x, const int32
                              const moe_ep_plan_t* plan_dev, uint8_t* send, int32_t* slot_row, void* ws,
                              size_t ws_bytes, void* stream);
 
-/* Received rows (recv: plan.rows_recv rows x MOE_EP_ROW_BYTES(H), ordered by
- * source rank, then local expert, then token) into the grouped layout of the
- * local experts: Aq [M_rows, H] u8 and As [H/128][M_rows] fp32 (moe_permute's
- * contiguous layout; padding rows code 0, scale 1), offsets [E_local + 1] out
- * (the plan's), group_row [plan.rows_recv] int32 out: the grouped row of each
- * received row. M_rows >= plan.rows_group, a multiple of 4. */
+/* Received rows (recv: plan.rows_recv rows x MOE_EP_ROW_BYTES(H), in the
+ * plan's receive order) into the grouped layout of the local experts: Aq
+ * [M_rows, H] u8 and As [H/128][M_rows] fp32 (moe_permute's contiguous layout;
+ * padding rows code 0, scale 1), offsets [E_local + 1] out (the plan's),
+ * group_row [plan.rows_recv] int32 out: the grouped row of each received row.
+ * M_rows >= plan.rows_group, a multiple of 4. A plan whose sizes disagree with
+ * the call's is reported (MOE_ERR_CAPACITY in the device status) and nothing
+ * is written. */
 moe_status_t moe_ep_receive(int H, const moe_ep_plan_t* plan_dev, int rows_recv, const uint8_t* recv, uint8_t* Aq,
                             float* As, int M_rows, int32_t* offsets, int32_t* group_row, void* stream);
+/* The same for chunk `chunk` of the plan only: its receive rows (recv is the
+ * whole receive buffer; the chunk's rows are [plan.recv_chunk[chunk],
+ * plan.recv_chunk[chunk + 1])) and the padding rows of its experts; offsets
+ * [E_c + 1] out: the chunk's experts' offsets less that of its first expert, for
+ * a grouped GEMM over the chunk's rows (A = Aq + plan.offsets[first] * H, As +
+ * plan.offsets[first], M_rows unchanged as the scales' row stride); group_row
+ * entries of the chunk's rows. chunk outside [0, plan.chunks) is reported like a
+ * plan that disagrees. */
+moe_status_t moe_ep_receive_chunk(int H, const moe_ep_plan_t* plan_dev, int chunk, const uint8_t* recv, uint8_t* Aq,
+                                  float* As, int M_rows, int32_t* offsets, int32_t* group_row, void* stream);
 
 /* ret [rows_recv, H] bf16 out: row i = O [group_row[i]] (the local experts'
- * output rows, moe_grouped_gemm_fp8's bf16 epilogue) in receive order. */
+ * output rows, moe_grouped_gemm_fp8's bf16 epilogue) in receive order.
+ * group_row needs 4-byte alignment only, so that a chunk's rows can be passed
+ * as group_row + plan.recv_chunk[c], ret + plan.recv_chunk[c] * H. */
 moe_status_t moe_ep_return(int H, int rows_recv, const void* O, const int32_t* group_row, void* ret, void* stream);
 
 const char* moe_status_string(moe_status_t status);

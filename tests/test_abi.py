@@ -137,3 +137,25 @@ def test_product_and_oracle_share_no_code():
     osrc = open(os.path.join(ROOT, "oracle", "__init__.py")).read()
     assert not re.search(r"^\s*(import|from)\s+fp8_grouped_gemm_fp32_b200\b", osrc, re.M)
     assert "moe_fp8.h" not in open(os.path.join(ROOT, "oracle", "moe_oracle.c")).read()
+
+
+def test_ep_plan_struct_layout_matches_the_header(tmp_path):
+    """The binding's moe_ep_plan_t (ctypes) has the C compiler's size and field offsets: the planner writes
+    the whole struct into it and the kernels read a byte copy of it."""
+    import ctypes
+    import shutil
+    import subprocess
+    from fp8_grouped_gemm_fp32_b200 import ep
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = [f[0] for f in ep.EpPlan._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include "moe_fp8.h"\nint main(void) {\n'
+                   '  printf("%zu\\n", sizeof(moe_ep_plan_t));\n' +
+                   "".join(f'  printf("%zu\\n", offsetof(moe_ep_plan_t, {f}));\n' for f in fields) + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call([cc, "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = [int(v) for v in subprocess.check_output([str(exe)]).split()]
+    assert got[0] == ctypes.sizeof(ep.EpPlan)
+    assert got[1:] == [getattr(ep.EpPlan, f).offset for f in fields]

@@ -54,22 +54,31 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("chunks", [1, 2, 3])
 @pytest.mark.parametrize("cfg,G", CASES)
-def test_plan_matches_one_process_dispatch(cfg, G):
+def test_plan_matches_one_process_dispatch(cfg, G, chunks):
     inp, idx, _ = _routing(cfg)
     E, k, El = cfg.E, cfg.k, cfg.E // G
+    if chunks > El:
+        pytest.skip("more chunks than local experts")
     cap = oracle.capacity(cfg.T, k, E, cfg.cap_num, cfg.cap_den)
     rows_cap = -(-(cfg.T * k + E * 127) // 128) * 128
     ref = oracle.dispatch(idx, E, cap, 0, 128, 0, rows_cap)
     sizes = _split(cfg.T, G, cfg.seed)
     bounds = np.concatenate([[0], np.cumsum(sizes)])
     counts_all = np.stack([np.bincount(idx[bounds[s]:bounds[s + 1]].ravel(), minlength=E) for s in range(G)])
-    plans = [ep.plan(G, r, E, cfg.T, k, cfg.cap_num, cfg.cap_den, counts_all) for r in range(G)]
+    plans = [ep.plan(G, r, E, cfg.T, k, cfg.cap_num, cfg.cap_den, counts_all, chunks) for r in range(G)]
     for s in range(G):
         p = plans[s]
-        assert p.rows_send == sum(p.send_rows[:G])
+        assert p.chunks == chunks and p.chunk_first[0] == 0 and p.chunk_first[chunks] == El
+        assert p.rows_send == sum(p.send_rows[:G]) == p.send_chunk[chunks]
         for d in range(G):
             assert p.send_rows[d] == plans[d].recv_rows[s]     # what s sends to d is what d expects from s
+            for c in range(chunks):                             # ... chunk by chunk
+                assert p.send_rows_c[c][d] == plans[d].recv_rows_c[c][s]
+        for c in range(chunks):
+            assert p.send_chunk[c + 1] - p.send_chunk[c] == sum(p.chunk_send(c))
+            assert p.recv_chunk[c + 1] - p.recv_chunk[c] == sum(p.chunk_recv(c))
     for d in range(G):
         p = plans[d]
         assert p.rows_recv == p.recv_start[G * El] == sum(p.recv_rows[:G])
@@ -83,7 +92,6 @@ def test_plan_matches_one_process_dispatch(cfg, G):
         loc = idx[bounds[s]:bounds[s + 1]]
         lr = _local_ranks(loc, E)
         p = plans[s]
-        send_base = np.concatenate([[0], np.cumsum(p.kept_mine[:E])])
         seen_send = set()
         for t in range(loc.shape[0]):
             for j in range(k):
@@ -93,20 +101,33 @@ def test_plan_matches_one_process_dispatch(cfg, G):
                 assert kept == (ref["slot_row"][g_slot] >= 0), (s, t, j)
                 if not kept:
                     continue
-                srow = send_base[e] + lr[t, j]
+                srow = p.send_off[e] + lr[t, j]
                 assert srow not in seen_send and srow < p.rows_send
                 seen_send.add(srow)
                 d, l = divmod(e, El)
+                c = int(np.searchsorted(np.array(p.chunk_first[:chunks + 1]), l, side="right")) - 1
+                # the send row lies in its chunk's slice, in the part for destination d
+                lo = p.send_chunk[c] + sum(p.send_rows_c[c][:d])
+                assert lo <= srow < lo + p.send_rows_c[c][d]
                 q = plans[d]
-                grow = q.group_start[s * El + l] + lr[t, j]
+                # receive block of (source s, local expert l): blocks run (chunk, source, expert)
+                cf = q.chunk_first
+                b = G * cf[c] + s * (cf[c + 1] - cf[c]) + (l - cf[c])
+                grow = q.group_start[b] + lr[t, j]
                 assert grow - q.offsets[l] == ref["slot_row"][g_slot] - ref["offsets"][e]
-                rrow = q.recv_start[s * El + l] + lr[t, j]
-                assert rrow < q.recv_start[s * El + l + 1]
+                rrow = q.recv_start[b] + lr[t, j]
+                assert q.recv_chunk[c] <= rrow < q.recv_start[b + 1] <= q.recv_chunk[c + 1]
+                # ... at the same place in d's chunk slice as srow in s's part of it
+                assert rrow - q.recv_chunk[c] - sum(q.recv_rows_c[c][:s]) == srow - lo
 
 
 def test_plan_rejects_bad_arguments():
     from fp8_grouped_gemm_fp32_b200 import api
     c = np.zeros((2, 8), np.int32)
+    with pytest.raises(api.MoeError):
+        ep.plan(2, 0, 8, 10, 2, 0, 0, c, chunks=5)     # more chunks than the 4 local experts
+    with pytest.raises(api.MoeError):
+        ep.plan(2, 0, 8, 10, 2, 0, 0, c, chunks=0)
     with pytest.raises(api.MoeError):
         ep.plan(2, 2, 8, 10, 2, 0, 0, c)              # rank outside [0, G)
     with pytest.raises(api.MoeError):
@@ -121,7 +142,7 @@ CFG2 = MoeConfig("ep_gloo", T=160, H=256, E=8, I=256, k=2, bias="zipf", cap_num=
 SIZES2 = [70, 90]
 
 
-def _rank_main(rank, port, out):
+def _rank_main(rank, port, out, chunks):
     import torch.distributed as dist
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -137,13 +158,13 @@ def _rank_main(rank, port, out):
         idx, w, _ = oracle.route(c_loc, x, to_np(inp.Wg), to_np(inp.bias), None)
         tr = ep.DistTransport()
         counts_all = tr.all_gather_counts(torch.from_numpy(np.bincount(idx.ravel(), minlength=E).astype(np.int32)))
-        p = ep.plan(G, rank, E, cfg.T, k, cfg.cap_num, cfg.cap_den, counts_all)
+        p = ep.plan(G, rank, E, cfg.T, k, cfg.cap_num, cfg.cap_den, counts_all, chunks)
         # send rows as the dispatch kernel lays them out: codes, scales, padding to 16 bytes
         xq, xs = oracle.quant_rows(oracle.bf16_bits_to_f32(x))
         rb = ep.row_bytes(H)
         send = np.zeros((p.rows_send, rb), np.uint8)
         lr = _local_ranks(idx, E)
-        base = np.concatenate([[0], np.cumsum(p.kept_mine[:E])])
+        base = np.array(p.send_off[:E])
         slot_row = np.full(idx.size, -1, np.int32)
         for t in range(idx.shape[0]):
             for j in range(k):
@@ -153,7 +174,9 @@ def _rank_main(rank, port, out):
                     send[r, :H] = xq[t]
                     send[r, H:H + 4 * (H // 128)] = xs[t].view(np.uint8)
                     slot_row[t * k + j] = r
-        recv = tr.exchange(torch.from_numpy(send), list(p.send_rows[:G]), list(p.recv_rows[:G])).numpy()
+        # one all-to-all per chunk, each on its slice of the send and receive rows
+        recv = np.concatenate([tr.exchange(torch.from_numpy(send[p.send_chunk[c]:p.send_chunk[c + 1]]), p.chunk_send(c),
+                                           p.chunk_recv(c)).numpy() for c in range(chunks)])
         # the owner's grouped layout and its experts (the oracle's grouped GEMMs on the local weights)
         M = max(p.rows_group, 128)
         Aq = np.zeros((M, H), np.uint8)
@@ -171,8 +194,9 @@ def _rank_main(rank, port, out):
         Hq, Hs = oracle.grouped_gemm(0, El, 2 * cfg.I, H, Aq, As, off, M, W13.numpy(), S13.numpy(), 1)
         O, _ = oracle.grouped_gemm(0, El, H, cfg.I, Hq, Hs, off, M, to_np(inp.W2q[sl]), to_np(inp.S2[sl]), 0)
         ret = O[group_row] if p.rows_recv else np.zeros((0, H), np.uint16)
-        back = tr.exchange(torch.from_numpy(ret.view(np.int16)), list(p.recv_rows[:G]), list(p.send_rows[:G]))
-        back = back.numpy().view(np.uint16)
+        back = np.concatenate([tr.exchange(torch.from_numpy(ret[p.recv_chunk[c]:p.recv_chunk[c + 1]].view(np.int16)),
+                                           p.chunk_recv(c), p.chunk_send(c)).numpy() for c in range(chunks)])
+        back = back.view(np.uint16).reshape(-1, H)
         y = oracle.combine(slot_row, w, back if back.shape[0] else np.zeros((1, H), np.uint16), c_loc.T, k)
         np.save(os.path.join(out, f"y{rank}.npy"), y)
         np.save(os.path.join(out, f"slot_row{rank}.npy"), slot_row)
@@ -180,13 +204,14 @@ def _rank_main(rank, port, out):
         dist.destroy_process_group()
 
 
-def test_two_ranks_over_gloo_equal_one_process(tmp_path):
+@pytest.mark.parametrize("chunks", [1, 3])
+def test_two_ranks_over_gloo_equal_one_process(tmp_path, chunks):
     import socket
     import torch.multiprocessing as mp
     with socket.socket() as s_:
         s_.bind(("127.0.0.1", 0))
         port = s_.getsockname()[1]
-    mp.spawn(_rank_main, args=(port, str(tmp_path)), nprocs=2, join=True)
+    mp.spawn(_rank_main, args=(port, str(tmp_path), chunks), nprocs=2, join=True)
     cfg = CFG2
     inp = make_inputs(cfg)
     ref = oracle.forward(cfg, oracle.moe_inputs_to_numpy(inp))

@@ -5,7 +5,9 @@ ranks' buffers between their kernels; no kernel waits on another rank's), and a 
 the torch.distributed transport (ep.forward_dist). Against the oracle on the ranks' batches concatenated in
 rank order: dropped slots bit-exact, the send rows' codes and scales bit-exact with the oracle's 1x128
 quantisation, y within max_rel 2e-2 / mean_rel 2e-3; and against moe_forward on the same concatenated batch
-(one GPU, same kernel form): y bit for bit, since every row meets the same arithmetic."""
+(one GPU, same kernel form): y bit for bit, since every row meets the same arithmetic. Plans of several
+chunks (each chunk's rows exchanged, its experts run and their outputs returned in turn; in the NCCL case
+the collectives on a stream of their own) give the same y bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -36,15 +38,16 @@ def _ranks(cfg, inp, G, sizes):
     return ranks, xs
 
 
-@pytest.mark.parametrize("G,sizes", [(1, [600]), (2, [250, 350]), (4, [100, 0, 300, 200])])
-def test_ep_local_ranks_equal_one_gpu(G, sizes):
+@pytest.mark.parametrize("G,sizes,chunks", [(1, [600], 1), (2, [250, 350], 1), (4, [100, 0, 300, 200], 1),
+                                            (1, [600], 5), (2, [250, 350], 3), (4, [100, 0, 300, 200], 4)])
+def test_ep_local_ranks_equal_one_gpu(G, sizes, chunks):
     ensure_lib()
     cfg = CFG
     inp = gpu_inputs(cfg)
     api.moe_set_contig_kernel(api.CONTIG_SINGLE)
     try:
         ranks, xs = _ranks(cfg, inp, G, sizes)
-        ys = ep.forward_local(ranks, xs)
+        ys = ep.forward_local(ranks, xs, chunks=chunks)
         torch.cuda.synchronize()
         assert api.moe_get_device_status() == api.MOE_OK
         one = gpu_forward(cfg, inp)
@@ -74,7 +77,8 @@ def test_ep_local_ranks_equal_one_gpu(G, sizes):
         t0 += r.cfg.T
 
 
-def test_ep_forward_dist_one_rank_nccl():
+@pytest.mark.parametrize("chunks", [1, 4])
+def test_ep_forward_dist_one_rank_nccl(chunks):
     # the torch.distributed transport on a one-rank NCCL group: all-gather and both all-to-alls really run
     import torch.distributed as dist
     ensure_lib()
@@ -85,7 +89,7 @@ def test_ep_forward_dist_one_rank_nccl():
     try:
         api.moe_set_contig_kernel(api.CONTIG_SINGLE)
         ranks, xs = _ranks(cfg, inp, 1, [cfg.T])
-        y = ep.forward_dist(ranks[0], xs[0], ep.DistTransport(), cfg.T)
+        y = ep.forward_dist(ranks[0], xs[0], ep.DistTransport(), cfg.T, chunks=chunks)
         torch.cuda.synchronize()
         one = gpu_forward(cfg, inp)
     finally:

@@ -262,10 +262,12 @@ GEMM_CASES = [
     (1, 1, 2, 256, 16384, [32, 7], 32),
     # far more tiles than the 148 persistent CTAs (contiguous: 28 M tiles x 16 N tiles = 448; masked: up to
     # 16 experts x 16 weight tiles x up to 2 token tiles), so every CTA runs several tiles and the stage,
-    # scale and accumulator rings wrap across tile boundaries
+    # scale and accumulator rings wrap across tile boundaries; the masked bf16 output in both tile widths
+    # (two 128-row weight blocks per tile where N allows, one for N = 1920)
     (0, 0, 8, 4096, 256, [600, 517, 0, 640, 129, 380, 700, 255], None),
     (0, 1, 8, 4096, 256, [600, 517, 0, 640, 129, 380, 700, 255], None),
-    (1, 0, 16, 2048, 256, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64),
+    (1, 0, 16, 4096, 256, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64),
+    (1, 0, 16, 1920, 256, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64),
     (1, 1, 16, 4096, 256, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64),
 ]
 
@@ -275,16 +277,20 @@ MANY_TILES = 296          # two tiles per persistent CTA on a 148-SM part
 def _tile_count(layout, epi, E, N, groups, M_rows):
     if layout == 0:
         return sum(-(-g // 128) for g in groups) * -(-N // 256)
-    return sum(-(-g // 32) for g in groups) * (N // 256 if epi == 1 else N // 128)
+    # masked: a weight tile is 256 rows (gate and up, or two output blocks when N allows) or 128
+    return sum(-(-g // 32) for g in groups) * (N // 256 if epi == 1 or N % 256 == 0 else N // 128)
 
 
 def test_gemm_cases_include_multi_tile_launches():
     # the coverage the cases above claim: both layouts and both epilogues have a launch with more tiles
-    # than two per CTA
+    # than two per CTA, the masked bf16 output in both tile widths
     for layout in (0, 1):
         for epi in (0, 1):
             assert any(c[0] == layout and c[1] == epi and _tile_count(layout, epi, c[2], c[3], c[5], c[6])
                        > MANY_TILES for c in GEMM_CASES), (layout, epi)
+    for wide in (True, False):
+        assert any(c[0] == 1 and c[1] == 0 and (c[3] % 256 == 0) == wide and
+                   _tile_count(1, 0, c[2], c[3], c[5], c[6]) > MANY_TILES for c in GEMM_CASES), wide
 
 
 class contig_form:
@@ -340,7 +346,8 @@ W4_CASES = [
     # more tiles than two per CTA in both epilogues (16 experts x 16 weight tiles x up to 2 token
     # tiles): the converter warps' stage counter, their barrier phases and the per-tile reload of the row
     # scales carry across tiles
-    (16, 2048, 1024, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64, 0, 6),
+    (16, 4096, 1024, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64, 0, 6),
+    (16, 1920, 1024, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64, 0, 8),
     (16, 4096, 1024, [64, 3, 0, 33, 64, 17, 40, 1, 64, 0, 63, 32, 9, 64, 50, 2], 64, 1, 7),
 ]
 
@@ -348,6 +355,9 @@ W4_CASES = [
 def test_w4_cases_include_multi_tile_launches():
     for epi in (0, 1):
         assert any(c[5] == epi and _tile_count(1, epi, c[0], c[1], c[3], c[4]) > MANY_TILES for c in W4_CASES)
+    for wide in (True, False):
+        assert any(c[5] == 0 and (c[1] % 256 == 0) == wide and _tile_count(1, 0, c[0], c[1], c[3], c[4]) > MANY_TILES
+                   for c in W4_CASES), wide
 
 
 @pytest.mark.parametrize("case", W4_CASES)
