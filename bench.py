@@ -541,6 +541,9 @@ def run_ours(args):
     # the burst figure: FP8 = 2 x the measured bf16 cuBLAS burst rate (the nominal B200 FP8:BF16 ratio).
     fp8_burst = FP8_PER_BF16 * float(peaks["bf16_tflops"])
     fp8_sus = FP8_PER_BF16 * float(peaks["bf16_tflops_sustained"])
+    if backward and "gemm_tflops_lower_bound" in backward:
+        # the backward's FP8 GEMM work against the burst FP8 rate (its elementwise steps count as time only)
+        backward["frac_fp8_burst_lower_bound"] = backward["gemm_tflops_lower_bound"] / fp8_burst
     fp8_lib = measure_fp8_peak(dev)
     dom = max(per, key=per.get)
     w = work[dom]

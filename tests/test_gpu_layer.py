@@ -31,6 +31,13 @@ SMALL = {
     "one_expert": (MoeConfig("one_expert", T=200, H=256, E=1, I=256, k=1, bias="zero", seed=14), None),
     "w4_masked": (MoeConfig("w4_masked", T=80, H=384, E=16, I=256, k=4, bias="uniform", layout="masked",
                             masked_max_m=64, seed=15, weights="w4"), None),
+    # the most experts and the largest k the boundary takes, through both GEMMs: 512 groups of a few rows
+    # (contiguous: 512 padded 128-row groups; masked: 512 blocks of 32 rows, E4M3 and 4-bit weights)
+    "limits_contig": (MoeConfig("limits_contig", T=64, H=256, E=512, I=128, k=32, bias="uniform", seed=16), None),
+    "limits_masked": (MoeConfig("limits_masked", T=64, H=256, E=512, I=128, k=32, bias="uniform", layout="masked",
+                                masked_max_m=32, seed=17), None),
+    "limits_w4": (MoeConfig("limits_w4", T=64, H=256, E=512, I=128, k=32, bias="uniform", layout="masked",
+                            masked_max_m=32, seed=18, weights="w4"), None),
 }
 
 
