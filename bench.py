@@ -273,30 +273,42 @@ def time_backward(layer, cfg, steps):
     dx, dWg, db = z(cfg.T, cfg.H, dt=torch.bfloat16), z(cfg.E, cfg.H, dt=torch.float32), z(cfg.E, dt=torch.float32)
     dW13, dW2 = z(cfg.E, 2 * cfg.I, cfg.H, dt=torch.bfloat16), z(cfg.E, cfg.H, cfg.I, dt=torch.bfloat16)
     bws = z(api.moe_backward_workspace_size(layer.c), dt=torch.uint8)
-    layer.forward()
+    # the training forward keeps the gate and up values, so the backward reads them instead of recomputing
+    tws = z(api.moe_workspace_size(layer.c, 2), dt=torch.uint8)
+
+    def fwd_train():
+        api.moe_forward_train(layer.c, i.x, i.Wg, i.bias, i.token_ids, layer.W13, layer.S13, i.W2q, i.S2, layer.y,
+                              layer.topk_idx, layer.topk_w, layer.counts, layer.slot_row, tws)
 
     def call():
         api.moe_backward(layer.c, i.x, i.Wg, layer.W13, layer.S13, W13T, S13T, W2T, S2T, layer.topk_idx, layer.topk_w,
-                         layer.slot_row, layer.ws, dy, dx, dWg, db, dW13, dW2, bws)
-    for _ in range(2):
-        call()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        call()
-    e1.record()
-    torch.cuda.synchronize()
+                         layer.slot_row, tws, dy, dx, dWg, db, dW13, dW2, bws, fwd_train=True)
+
+    def timed(fn, n):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    fwd_ms = timed(fwd_train, steps)           # leaves the last training forward's state in tws
+    ms = timed(call, steps)
     assert api.moe_get_device_status() == api.MOE_OK
-    ms = e0.elapsed_time(e1) / steps
     Rk = int(layer.kept.sum().item()) if hasattr(layer.kept, "sum") else 0
-    # FP8 tensor work: dh (H x I), a|b recomputed (2I x H), dx rows (H x 2I), dW2 (H x I), dW13 (2I x H),
-    # each 2 FLOP per multiply-add over the kept rows
-    flops = 2.0 * Rk * cfg.H * cfg.I * (1 + 2 + 2 + 1 + 2)
-    del bws, dW13, dW2
+    # FP8 tensor work: dh (H x I), dx rows (H x 2I), dW2 (H x I), dW13 (2I x H), each 2 FLOP per
+    # multiply-add over the kept rows (a | b comes from the training forward)
+    flops = 2.0 * Rk * cfg.H * cfg.I * (1 + 2 + 1 + 2)
+    del bws, dW13, dW2, tws
     return {"ms": ms, "tokens_per_s": cfg.T / (ms / 1e3), "calls": steps, "gemm_tflops_lower_bound": flops / (ms / 1e3) / 1e12,
-            "what": "moe_backward: dx, dW_g, db, dW13, dW2 of one step (five FP8 grouped GEMMs, two of them "
-                    "K-grouped weight gradients), after one forward"}
+            "forward_train_ms": fwd_ms,
+            "what": "moe_backward: dx, dW_g, db, dW13, dW2 of one step (four FP8 grouped GEMMs, two of them "
+                    "K-grouped weight gradients) after moe_forward_train, which keeps the gate and up values "
+                    "(forward_train_ms: that forward's own time)"}
 
 
 def run_e2e(layer, cfg, steps, world):

@@ -31,7 +31,7 @@ EPI_BF16, EPI_SWIGLU_FP8 = 0, 1
 CONTIG_AUTO, CONTIG_SINGLE, CONTIG_PAIR = 0, 1, 2
 WEIGHTS_FP8, WEIGHTS_W4 = 0, 1
 EXPORTS = ("moe_rows_capacity", "moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_gemm_fp8",
-           "moe_combine", "moe_forward", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string",
+           "moe_combine", "moe_forward", "moe_forward_train", "moe_get_device_status", "moe_selftest_wait_timeout", "moe_status_string",
            "moe_permute_noalloc", "moe_balance_bias", "moe_grouped_gemm_w4", "moe_set_contig_kernel",
            "moe_ep_plan", "moe_ep_plan_chunked", "moe_ep_workspace_size", "moe_ep_count", "moe_ep_dispatch",
            "moe_ep_receive", "moe_ep_receive_chunk", "moe_ep_return", "moe_backward_workspace_size", "moe_backward")
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_gemm_w4.argtypes = [I, I, I, I, P, P, P, I, P, P, I, P, P, P]
         L.moe_combine.argtypes = [CP, P, P, P, P, P]
         L.moe_forward.argtypes = [CP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_forward_train.argtypes = [CP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.moe_balance_bias.argtypes = [I, P, P, P, ctypes.c_float, I, P]
         L.moe_get_device_status.argtypes = [P]
         L.moe_selftest_wait_timeout.argtypes = [I, P]
@@ -93,7 +94,7 @@ def lib() -> ctypes.CDLL:
         L.moe_ep_return.argtypes = [I, I, P, P, P, P]
         L.moe_backward_workspace_size.argtypes = [CP]
         L.moe_backward_workspace_size.restype = SZ
-        L.moe_backward.argtypes = [CP] + [P] * 19 + [SZ, P]
+        L.moe_backward.argtypes = [CP] + [P] * 12 + [I] + [P] * 7 + [SZ, P]
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in EXPORTS:
@@ -135,7 +136,8 @@ def moe_rows_capacity(cfg: Config) -> int:
     return int(lib().moe_rows_capacity(ctypes.byref(cfg)))
 
 
-def moe_workspace_size(cfg: Config, for_forward: bool = False) -> int:
+def moe_workspace_size(cfg: Config, for_forward: int = 0) -> int:
+    """Scratch bytes: 0 route / permute, 1 moe_forward, 2 moe_forward_train."""
     return int(lib().moe_workspace_size(ctypes.byref(cfg), int(for_forward)))
 
 
@@ -179,6 +181,15 @@ def moe_forward(cfg, x, Wg, bias, token_ids, W13, S13, W2, S2, y, topk_idx, topk
     _check(lib().moe_forward(ctypes.byref(cfg), _p(x), _p(Wg), _p(bias), _p(token_ids), _p(W13), _p(S13), _p(W2),
                              _p(S2), _p(y), _p(topk_idx), _p(topk_w), _p(counts), _p(slot_row), _p(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+
+
+def moe_forward_train(cfg, x, Wg, bias, token_ids, W13, S13, W2, S2, y, topk_idx, topk_w, counts, slot_row, ws,
+                      stream=None):
+    """moe_forward that also keeps the gate and up values in ws (moe_workspace_size(cfg, 2) bytes) for
+    moe_backward(..., fwd_train=True)."""
+    _check(lib().moe_forward_train(ctypes.byref(cfg), _p(x), _p(Wg), _p(bias), _p(token_ids), _p(W13), _p(S13),
+                                   _p(W2), _p(S2), _p(y), _p(topk_idx), _p(topk_w), _p(counts), _p(slot_row), _p(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)), "moe_forward_train")
 
 
 def moe_balance_bias(E, counts, load, bias, gamma, update, stream=None):
@@ -240,7 +251,9 @@ def moe_backward_workspace_size(cfg: Config) -> int:
 
 
 def moe_backward(cfg, x, Wg, W13, S13, W13T, S13T, W2T, S2T, topk_idx, topk_w, slot_row, fwd_ws, dy, dx, dWg, db,
-                 dW13, dW2, ws, stream=None):
+                 dW13, dW2, ws, stream=None, fwd_train: bool = False):
+    """fwd_train: fwd_ws comes from moe_forward_train (the gate and up values are read, not recomputed)."""
     _check(lib().moe_backward(ctypes.byref(cfg), _p(x), _p(Wg), _p(W13), _p(S13), _p(W13T), _p(S13T), _p(W2T),
-                              _p(S2T), _p(topk_idx), _p(topk_w), _p(slot_row), _p(fwd_ws), _p(dy), _p(dx), _p(dWg),
-                              _p(db), _p(dW13), _p(dW2), _p(ws), _nbytes(ws), _stream(stream)), "moe_backward")
+                              _p(S2T), _p(topk_idx), _p(topk_w), _p(slot_row), _p(fwd_ws), int(bool(fwd_train)),
+                              _p(dy), _p(dx), _p(dWg), _p(db), _p(dW13), _p(dW2), _p(ws), _nbytes(ws),
+                              _stream(stream)), "moe_backward")

@@ -24,7 +24,8 @@ cudaError_t launch_permute(const uint16_t* x, const int32_t* topk_idx, int T, in
                            int num_sms, cudaStream_t s);
 cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                                 const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs, int epilogue,
-                                void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s);
+                                void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s,
+                                uint16_t* save_ab = nullptr);
 cudaError_t launch_grouped_gemm_w4(int E, int N, int K, const uint8_t* A, const float* As, const int32_t* masked_m,
                                    int M_rows, const uint8_t* B, const float* Bs, int epilogue, void* D, float* Ds,
                                    int* status, uint64_t wait_ns, int num_sms, cudaStream_t s);
@@ -154,10 +155,11 @@ struct FwdWs {
     int32_t* offsets;
     int32_t* row_src;
     void* step;   // route / permute scratch
+    uint16_t* ab; // training workspace only: the up GEMM's gate and up values, bf16 [rows, 2I]
     size_t total;
 };
 
-FwdWs carve(const moe_config_t* c, void* base) {
+FwdWs carve(const moe_config_t* c, void* base, bool train = false) {
     FwdWs w;
     const size_t rows = rows_of(c);
     uint8_t* p = static_cast<uint8_t*>(base);
@@ -176,6 +178,7 @@ FwdWs carve(const moe_config_t* c, void* base) {
     w.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (c->E + 1)));
     w.row_src = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * rows));
     w.step = take(std::max(route_scratch(c), align_up(moe::permute_scratch_bytes(c->T, c->E))));
+    w.ab = train ? reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * rows * 2 * c->I)) : nullptr;
     w.total = off;
     return w;
 }
@@ -263,7 +266,7 @@ size_t moe_rows_capacity(const moe_config_t* cfg) {
 
 size_t moe_workspace_size(const moe_config_t* cfg, int for_forward) {
     if (check_cfg(cfg) != MOE_OK) return 0;
-    if (for_forward) return carve(cfg, nullptr).total;
+    if (for_forward) return carve(cfg, nullptr, for_forward == 2).total;
     return std::max(route_scratch(cfg), align_up(permute_scratch_bytes(cfg->T, cfg->E)));
 }
 
@@ -368,12 +371,15 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* O, const int32_t* 
                                       static_cast<uint16_t*>(y), static_cast<cudaStream_t>(stream)));
 }
 
-moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg, const float* bias,
-                         const int32_t* token_ids, const uint8_t* W13, const float* S13, const uint8_t* W2,
-                         const float* S2, void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
-                         int32_t* slot_row, void* ws, size_t ws_bytes, void* stream) {
+static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const float* Wg, const float* bias,
+                                 const int32_t* token_ids, const uint8_t* W13, const float* S13, const uint8_t* W2,
+                                 const float* S2, void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                 int32_t* slot_row, void* ws, size_t ws_bytes, void* stream, bool train) {
     moe_status_t st = check_cfg(cfg);
     if (st != MOE_OK) return st;
+    if (train && (cfg->layout != MOE_LAYOUT_CONTIGUOUS || cfg->weights != MOE_WEIGHTS_FP8 ||
+                  cfg->routing != MOE_ROUTE_SOFTMAX_TOPK))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
     DeviceInfo* dev;
     if ((st = device_info(&dev)) != MOE_OK) return st;
     if (!ptr_ok(x) || !ptr_ok(W13) || !ptr_ok(S13) || !ptr_ok(W2) || !ptr_ok(S2) || !ptr_ok(y) || !ptr_ok(topk_idx) ||
@@ -383,7 +389,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
         return MOE_ERR_INVALID_ARG;
     if (cfg->routing == MOE_ROUTE_HASH && !ptr_ok(token_ids)) return MOE_ERR_INVALID_ARG;
     if (cfg->weights == MOE_WEIGHTS_W4 && cfg->layout != MOE_LAYOUT_MASKED) return MOE_ERR_UNSUPPORTED_SHAPE;
-    const FwdWs w = carve(cfg, ws);
+    const FwdWs w = carve(cfg, ws, train);
     if (ws_bytes < w.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (cfg->T == 0) return MOE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -410,7 +416,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
                                    nullptr, dev->status, kWaitNs, dev->num_sms, s);
     } else {
         e = launch_grouped_gemm(cfg->layout, cfg->E, 2 * cfg->I, cfg->H, w.Aq, w.As, group, M_rows, W13, S13,
-                                MOE_EPI_SWIGLU_FP8, w.Hq, w.Hs, dev->status, kWaitNs, dev->num_sms, s);
+                                MOE_EPI_SWIGLU_FP8, w.Hq, w.Hs, dev->status, kWaitNs, dev->num_sms, s, w.ab);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         e = launch_grouped_gemm(cfg->layout, cfg->E, cfg->H, cfg->I, w.Hq, w.Hs, group, M_rows, W2, S2, MOE_EPI_BF16,
                                 w.O, nullptr, dev->status, kWaitNs, dev->num_sms, s);
@@ -418,6 +424,22 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_combine(w.O, slot_row, topk_w, cfg->T, cfg->k, cfg->H, static_cast<uint16_t*>(y), s);
     return cuda_status(e);
+}
+
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg, const float* bias,
+                         const int32_t* token_ids, const uint8_t* W13, const float* S13, const uint8_t* W2,
+                         const float* S2, void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                         int32_t* slot_row, void* ws, size_t ws_bytes, void* stream) {
+    return forward_impl(cfg, x, Wg, bias, token_ids, W13, S13, W2, S2, y, topk_idx, topk_w, counts, slot_row, ws,
+                        ws_bytes, stream, false);
+}
+
+moe_status_t moe_forward_train(const moe_config_t* cfg, const void* x, const float* Wg, const float* bias,
+                               const int32_t* token_ids, const uint8_t* W13, const float* S13, const uint8_t* W2,
+                               const float* S2, void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                               int32_t* slot_row, void* ws, size_t ws_bytes, void* stream) {
+    return forward_impl(cfg, x, Wg, bias, token_ids, W13, S13, W2, S2, y, topk_idx, topk_w, counts, slot_row, ws,
+                        ws_bytes, stream, true);
 }
 
 size_t moe_backward_workspace_size(const moe_config_t* cfg) {
@@ -428,8 +450,8 @@ size_t moe_backward_workspace_size(const moe_config_t* cfg) {
 moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const float* Wg, const uint8_t* W13, const float* S13,
                           const uint8_t* W13T, const float* S13T, const uint8_t* W2T, const float* S2T,
                           const int32_t* topk_idx, const float* topk_w, const int32_t* slot_row, const void* fwd_ws,
-                          const void* dy, void* dx, float* dWg, float* db, void* dW13, void* dW2, void* ws,
-                          size_t ws_bytes, void* stream) {
+                          int fwd_train, const void* dy, void* dx, float* dWg, float* db, void* dW13, void* dW2,
+                          void* ws, size_t ws_bytes, void* stream) {
     moe_status_t st = check_cfg(cfg);
     if (st != MOE_OK) return st;
     if (cfg->layout != MOE_LAYOUT_CONTIGUOUS || cfg->weights != MOE_WEIGHTS_FP8 ||
@@ -448,7 +470,8 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const float* W
         return MOE_ERR_INVALID_ARG;
     const BwdWs b = carve_bwd(cfg, ws);
     if (ws_bytes < b.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
-    const FwdWs f = carve(cfg, const_cast<void*>(fwd_ws));
+    if (fwd_train != 0 && fwd_train != 1) return MOE_ERR_INVALID_ARG;
+    const FwdWs f = carve(cfg, const_cast<void*>(fwd_ws), fwd_train != 0);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int T = cfg->T, k = cfg->k, H = cfg->H, I = cfg->I, E = cfg->E;
     const int rows = static_cast<int>(rows_of(cfg));
@@ -460,10 +483,15 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const float* W
     if (!ok(launch_grouped_gemm(MOE_LAYOUT_CONTIGUOUS, E, I, H, b.dOq, b.dOs, f.offsets, rows, W2T, S2T, MOE_EPI_BF16,
                                 b.dh, nullptr, dev->status, kWaitNs, dev->num_sms, s)))
         return MOE_ERR_CUDA;
-    if (!ok(launch_grouped_gemm(MOE_LAYOUT_CONTIGUOUS, E, 2 * I, H, f.Aq, f.As, f.offsets, rows, W13, S13, MOE_EPI_BF16,
-                                b.ab, nullptr, dev->status, kWaitNs, dev->num_sms, s)))
-        return MOE_ERR_CUDA;
-    if (!ok(launch_bwd_swiglu(b.ab, b.dh, f.row_src, rows, I, b.g, b.gq, b.gs, s))) return MOE_ERR_CUDA;
+    // a | b: saved by moe_forward_train, else recomputed (the same kernel arithmetic, so the same values)
+    const uint16_t* ab = f.ab;
+    if (!fwd_train) {
+        if (!ok(launch_grouped_gemm(MOE_LAYOUT_CONTIGUOUS, E, 2 * I, H, f.Aq, f.As, f.offsets, rows, W13, S13,
+                                    MOE_EPI_BF16, b.ab, nullptr, dev->status, kWaitNs, dev->num_sms, s)))
+            return MOE_ERR_CUDA;
+        ab = b.ab;
+    }
+    if (!ok(launch_bwd_swiglu(ab, b.dh, f.row_src, rows, I, b.g, b.gq, b.gs, s))) return MOE_ERR_CUDA;
     if (!ok(launch_grouped_gemm(MOE_LAYOUT_CONTIGUOUS, E, H, 2 * I, b.gq, b.gs, f.offsets, rows, W13T, S13T,
                                 MOE_EPI_BF16, b.dxr, nullptr, dev->status, kWaitNs, dev->num_sms, s)))
         return MOE_ERR_CUDA;

@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kThreadsC, 1)
 gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmD, const float* __restrict__ As, const int32_t* __restrict__ offsets, int M_rows,
                  const float* __restrict__ Bs, int E, int N, int K, void* __restrict__ D, float* __restrict__ Ds,
-                 int* status, uint64_t wait_ns, int kg_rows) {
+                 int* status, uint64_t wait_ns, int kg_rows, uint16_t* __restrict__ save_ab) {
     static_assert(!KG || (EPI == 0 && !PAIR), "K-grouped tiles run on single CTAs with the bf16 epilogue");
     extern __shared__ uint8_t smem_raw[];
     using SC = SmemC<EPI, PAIR>;
@@ -575,6 +575,24 @@ gg_contig_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     bulk_commit();
                 }
             } else {
+                if (save_ab) {
+                    // training: the gate and up values themselves, rounded to bf16, kept for the backward
+                    // pass ([M_rows, N] in W13's interleaved column order, as a bf16-output GEMM writes them)
+                    uint16_t* dst = save_ab + grow * N + t.n0 + half * 64;
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb)
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) {
+                            uint32_t u[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const __nv_bfloat162 b2 =
+                                    __floats2bfloat162_rn(acc[hb * 64 + p * 8 + 2 * i], acc[hb * 64 + p * 8 + 2 * i + 1]);
+                                u[i] = *reinterpret_cast<const uint32_t*>(&b2);
+                            }
+                            *reinterpret_cast<uint4*>(dst + hb * kBM + p * 8) = make_uint4(u[0], u[1], u[2], u[3]);
+                        }
+                }
                 // SwiGLU on (a = acc[0..63], b = acc[64..127]) for h columns n0/2 + half*64 + [0, 64)
                 float amax = 0.0f;
 #pragma unroll
@@ -1135,7 +1153,7 @@ template <int EPI, bool PAIR, bool KG = false>
 static cudaError_t launch_contig(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapD,
                                  const float* As, const int32_t* offsets, int M_rows, const float* Bs, int E, int N,
                                  int K, void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms,
-                                 cudaStream_t s, int kg_rows = 0) {
+                                 cudaStream_t s, int kg_rows = 0, uint16_t* save_ab = nullptr) {
     auto kern = gg_contig_kernel<EPI, PAIR, KG>;
     const size_t smem = sizeof(SmemC<EPI, PAIR>) + 1024;
     cudaError_t err = set_smem(kern, smem);
@@ -1171,7 +1189,7 @@ static cudaError_t launch_contig(const CUtensorMap& mapA, const CUtensorMap& map
         cfg.numAttrs = 0;
     }
     return cudaLaunchKernelEx(&cfg, kern, mapA, mapB, mapD, As, offsets, M_rows, Bs, E, N, K, D, Ds, status, wait_ns,
-                              kg_rows);
+                              kg_rows, save_ab);
 }
 
 // K-grouped grouped GEMM (the backward pass's weight gradients): D [E * M, N] bf16, expert e's rows
@@ -1205,9 +1223,12 @@ static bool use_pairs(int E, int N, int M_rows) {
     return __atomic_load_n(&g_contig_mode, __ATOMIC_RELAXED) == 2;
 }
 
+// save_ab (contiguous layout, SwiGLU epilogue only; nullable): also write the gate and up values, bf16
+// [M_rows, N], for the backward pass.
 cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* A, const float* As,
                                 const int32_t* group_info, int M_rows, const uint8_t* B, const float* Bs, int epilogue,
-                                void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s) {
+                                void* D, float* Ds, int* status, uint64_t wait_ns, int num_sms, cudaStream_t s,
+                                uint16_t* save_ab) {
     CUtensorMap mapA, mapB, mapD;
     if (layout == 0) {
         if (!make_map(&mapA, A, K, static_cast<uint64_t>(M_rows), kBM)) return cudaErrorInvalidValue;
@@ -1222,10 +1243,11 @@ cudaError_t launch_grouped_gemm(int layout, int E, int N, int K, const uint8_t* 
         }
         if (!make_out_map(&mapD, D, N / 2, static_cast<uint64_t>(M_rows), 1)) return cudaErrorInvalidValue;
         return pair ? launch_contig<1, true>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K, D, Ds, status,
-                                             wait_ns, num_sms, s)
+                                             wait_ns, num_sms, s, 0, save_ab)
                     : launch_contig<1, false>(mapA, mapB, mapD, As, group_info, M_rows, Bs, E, N, K, D, Ds, status,
-                                              wait_ns, num_sms, s);
+                                              wait_ns, num_sms, s, 0, save_ab);
     } else {
+        if (save_ab) return cudaErrorInvalidValue;
         if (!make_map(&mapA, A, K, static_cast<uint64_t>(E) * M_rows, kBT)) return cudaErrorInvalidValue;
         if (!make_map(&mapB, B, K, static_cast<uint64_t>(E) * N, 128)) return cudaErrorInvalidValue;
         if (epilogue == 0 && N % (2 * kBM) == 0) {

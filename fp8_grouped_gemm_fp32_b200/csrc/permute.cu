@@ -189,7 +189,8 @@ __device__ __forceinline__ GroupCodes quantise_group(uint4 raw, float amax) {
 
 // blockIdx.x < nchunks: the slot maps of one 32-token chunk (slot_row, row_src);
 // blockIdx.x >= nchunks (contiguous layout only): the padding rows of one expert, one slice of
-// pad_slices of its 128-groups (codes 0, scale 1, row_src -1). Block 0 also writes offsets.
+// pad_slices of its 128-groups (codes 0, scale 1, row_src -1), and (the last expert's first slice)
+// row_src -1 for the rows past the last group. Block 0 also writes offsets.
 // row_base (nullable): each expert's first row, in place of the scan of kept (an expert-parallel
 // plan's send rows, which run in chunk order).
 __global__ void __launch_bounds__(256) permute_map_kernel(
@@ -229,6 +230,10 @@ __global__ void __launch_bounds__(256) permute_map_kernel(
         }
         if (sl == 0)
             for (int r = r0 + tid; r < r1; r += blockDim.x) row_src[r] = -1;
+        // the rows past the last group, up to ld_rows, belong to no group: marked as padding too, so that a
+        // step that walks every row (the backward pass) reads no stale source slot there
+        if (sl == 0 && e == E - 1 && row_src)
+            for (int r = off_s[E] + tid; r < ld_rows; r += blockDim.x) row_src[r] = -1;
         return;
     }
 

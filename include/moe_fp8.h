@@ -91,8 +91,10 @@ typedef struct {
  * padding rows per expert); masked: E * masked_max_m. 0 on a bad config. */
 size_t moe_rows_capacity(const moe_config_t* cfg);
 
-/* Scratch bytes moe_route and moe_permute need (ws_bytes >= this) and, with
- * for_forward != 0, the bytes moe_forward needs. 0 on a bad config. */
+/* Scratch bytes moe_route and moe_permute need (ws_bytes >= this); with
+ * for_forward = 1 the bytes moe_forward needs, with for_forward = 2 those of
+ * moe_forward_train (the same plus the saved gate and up values, 4 I bytes per
+ * row). 0 on a bad config. */
 size_t moe_workspace_size(const moe_config_t* cfg, int for_forward);
 
 /*
@@ -242,6 +244,17 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const float* Wg
                          const uint8_t* W2, const float* S2, void* y, int32_t* topk_idx, float* topk_w,
                          int32_t* counts, int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_forward for training: the same step and outputs, and the up GEMM also
+ * keeps each row's gate and up values (a | b, bf16, W13's column order) in the
+ * workspace, for moe_backward with fwd_train = 1 (which then needs no second
+ * x W13^T GEMM). ws: moe_workspace_size(cfg, 2) bytes. Contiguous layout, E4M3
+ * weights and softmax routing only (MOE_ERR_UNSUPPORTED_SHAPE otherwise), as
+ * for moe_backward. */
+moe_status_t moe_forward_train(const moe_config_t* cfg, const void* x, const float* Wg, const float* bias,
+                               const int32_t* token_ids, const uint8_t* W13, const float* S13,
+                               const uint8_t* W2, const float* S2, void* y, int32_t* topk_idx, float* topk_w,
+                               int32_t* counts, int32_t* slot_row, void* ws, size_t ws_bytes, void* stream);
+
 /*
  * Permutation without a workspace, for callers that may not allocate device
  * memory (code running during CUDA graph capture, servers that fix their
@@ -278,7 +291,8 @@ moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const void* x, const i
  *                          dO^T h
  * with dw_j = <dy_t, o_j> (0 for a dropped slot), dl_j = w_j (dw_j -
  * sum_i w_i dw_i), dO = w dy (fp32) on each kept row, dh = dO W2, a | b = x
- * W13^T (recomputed), g = (dh b s (1 + a (1 - s)), dh a s), s = sigmoid(a).
+ * W13^T (saved by moe_forward_train, else recomputed with the same kernel, so
+ * the same values), g = (dh b s (1 + a (1 - s)), dh a s), s = sigmoid(a).
  * The forward's quantisation steps pass the gradient straight through; the
  * selection and the capacity drop are held fixed. Every GEMM is FP8 with fp32
  * scales and fp32 promotion: dO, g and x in 1x128 groups along the
@@ -291,9 +305,11 @@ moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const void* x, const i
  *                          scales (a layout step done once, like the weights'
  *                          quantisation)
  *   topk_idx, topk_w, slot_row: the forward's outputs
- *   fwd_ws                  the workspace of that moe_forward call, unchanged
- *                          since (it holds the quantised x and h rows, the
- *                          expert outputs and the row maps)
+ *   fwd_ws                  the workspace of that moe_forward (fwd_train = 0)
+ *                          or moe_forward_train (fwd_train = 1) call,
+ *                          unchanged since (it holds the quantised x and h
+ *                          rows, the expert outputs and the row maps, and with
+ *                          fwd_train = 1 the gate and up values)
  *   ws                      scratch, moe_backward_workspace_size(cfg) bytes,
  *                          256-byte aligned
  * Contiguous layout, E4M3 weights and softmax routing only
@@ -304,8 +320,8 @@ size_t moe_backward_workspace_size(const moe_config_t* cfg);
 moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const float* Wg, const uint8_t* W13, const float* S13,
                           const uint8_t* W13T, const float* S13T, const uint8_t* W2T, const float* S2T,
                           const int32_t* topk_idx, const float* topk_w, const int32_t* slot_row, const void* fwd_ws,
-                          const void* dy, void* dx, float* dWg, float* db, void* dW13, void* dW2, void* ws,
-                          size_t ws_bytes, void* stream);
+                          int fwd_train, const void* dy, void* dx, float* dWg, float* db, void* dW13, void* dW2,
+                          void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Auxiliary-loss-free load balancing. Source: MegaMoE page, section 2.2: each

@@ -2,7 +2,8 @@
 dx and the weight gradients dW13, dW2 (bf16) within max_rel 2e-2 / mean_rel 2e-3, the gate's dW_g and db
 (fp32) within 1e-3 of the largest entry. The cases drop slots at capacity (their gate gradients still
 count), leave an expert empty or nearly so, and give experts several 128-row tiles, so the weight-gradient
-GEMM runs several K blocks per expert."""
+GEMM runs several K blocks per expert. The backward after moe_forward_train (the gate and up values saved
+by the forward) equals the one after moe_forward (recomputed) bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -37,24 +38,33 @@ def test_backward_matches_oracle(name):
     T, k, H, E, I = cfg.T, cfg.k, cfg.H, cfg.E, cfg.I
     W13, S13 = interleave_w13(inp.W1q, inp.S1, inp.W3q, inp.S3)
     W13T, S13T, W2T, S2T = transpose_weights(W13, S13, inp.W2q, inp.S2)
-    y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
-    w = torch.empty(T, k, dtype=torch.float32, device=dev)
-    counts = torch.empty(E, dtype=torch.int32, device=dev)
-    slot_row = torch.empty(T * k, dtype=torch.int32, device=dev)
-    fws = torch.empty(api.moe_workspace_size(c, True), dtype=torch.uint8, device=dev)
-    api.moe_forward(c, inp.x, inp.Wg, inp.bias, inp.token_ids, W13, S13, inp.W2q, inp.S2, y, idx, w, counts, slot_row,
-                    fws)
-    dx = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-    dWg = torch.empty(E, H, dtype=torch.float32, device=dev)
-    db = torch.empty(E, dtype=torch.float32, device=dev)
-    dW13 = torch.empty(E, 2 * I, H, dtype=torch.bfloat16, device=dev)
-    dW2 = torch.empty(E, H, I, dtype=torch.bfloat16, device=dev)
-    bws = torch.empty(api.moe_backward_workspace_size(c), dtype=torch.uint8, device=dev)
-    api.moe_backward(c, inp.x, inp.Wg, W13, S13, W13T, S13T, W2T, S2T, idx, w, slot_row, fws, dy, dx, dWg, db, dW13,
-                     dW2, bws)
+
+    def run(train):
+        y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        counts = torch.empty(E, dtype=torch.int32, device=dev)
+        slot_row = torch.empty(T * k, dtype=torch.int32, device=dev)
+        # workspaces hold stale bytes, as reused memory does: nothing may depend on their contents
+        fws = torch.full((api.moe_workspace_size(c, 2 if train else 1),), 0x5a, dtype=torch.uint8, device=dev)
+        fwd = api.moe_forward_train if train else api.moe_forward
+        fwd(c, inp.x, inp.Wg, inp.bias, inp.token_ids, W13, S13, inp.W2q, inp.S2, y, idx, w, counts, slot_row, fws)
+        out = dict(slot_row=slot_row, dx=torch.empty(T, H, dtype=torch.bfloat16, device=dev),
+                   dWg=torch.empty(E, H, dtype=torch.float32, device=dev), db=torch.empty(E, dtype=torch.float32, device=dev),
+                   dW13=torch.empty(E, 2 * I, H, dtype=torch.bfloat16, device=dev),
+                   dW2=torch.empty(E, H, I, dtype=torch.bfloat16, device=dev))
+        bws = torch.full((api.moe_backward_workspace_size(c),), 0x5a, dtype=torch.uint8, device=dev)
+        api.moe_backward(c, inp.x, inp.Wg, W13, S13, W13T, S13T, W2T, S2T, idx, w, slot_row, fws, dy, out["dx"],
+                         out["dWg"], out["db"], out["dW13"], out["dW2"], bws, fwd_train=train)
+        return out
+
+    out = run(False)
+    trained = run(True)
     torch.cuda.synchronize()
     assert api.moe_get_device_status() == api.MOE_OK
+    for key in out:
+        assert torch.equal(out[key], trained[key]), key
+    dx, dWg, db, dW13, dW2, slot_row = (out[key] for key in ("dx", "dWg", "db", "dW13", "dW2", "slot_row"))
     ref = oracle.backward(cfg, oracle.moe_inputs_to_numpy(inp), to_np(dy))
     f = ref["forward"]
     assert np.array_equal(to_np(slot_row), f["slot_row"])

@@ -146,6 +146,7 @@ def test_permute_bit_exact(name, T):
     else:
         used = ref["offsets"][-1]
         assert np.array_equal(got["row_src"][:used], ref["row_src"][:used])
+        assert np.all(got["row_src"][used:] == -1)                         # rows past the last group: padding
         assert np.array_equal(got["Aq"][:used], ref["Aq"][:used])          # padding rows are 0 too
         assert np.array_equal(got["As"][:, :used], ref["As"][:, :used])    # padding scales are 1
     if cfg.cap_num:
