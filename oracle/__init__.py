@@ -559,3 +559,114 @@ def backward(cfg, inp: dict, dy_bits: np.ndarray, nthreads=None):
         dW13[e] = f64_to_bf16_bits(acc13)
     return dict(dx=dx, dWg=dWg.astype(np.float32), db=db.astype(np.float32), dW13=dW13, dW2=dW2, dw=dw, dl=dl,
                 dOq=dOq, dOs=dOs, dh=dh, ab=ab, g=g, gq=gq, gs=gs, dx_rows=dxr, forward=f)
+
+
+
+def _w13_of(inp, e, I, H):
+    """Expert e's up operand as the backward uses it: W13 [2I, H] (W1 and W3 128-row blocks alternating)
+    and S13 [2I/128, H/128]."""
+    W13 = np.stack((np.asarray(inp["W1q"][e]).reshape(I // GROUP, GROUP, H),
+                    np.asarray(inp["W3q"][e]).reshape(I // GROUP, GROUP, H)), axis=1).reshape(2 * I, H)
+    S13 = np.stack((np.asarray(inp["S1"][e]), np.asarray(inp["S3"][e])), axis=1).reshape(2 * I // GROUP, H // GROUP)
+    return np.ascontiguousarray(W13), np.ascontiguousarray(S13)
+
+
+def backward_sampled(cfg, inp: dict, dy_bits: np.ndarray, tokens, experts, nthreads=None):
+    """`backward` restricted to what some outputs need, for checks at sizes the whole oracle cannot reach:
+    dx of `tokens` and dW13[e], dW2[e] of `experts`. Routing, capacity and the permutation still run over
+    all T (ranks are global); every other step runs on the rows involved only, through the same routines
+    in the same order (each row's GEMMs are independent of the others', an expert's weight gradients sum
+    over its own tiles), so the results equal `backward`'s at those entries. Returns dx {token: bf16 row},
+    dW13 {e: [2I, H] bf16}, dW2 {e: [H, I] bf16}."""
+    x32 = bf16_bits_to_f32(inp["x"])
+    dy = bf16_bits_to_f32(dy_bits)
+    T, H = inp["x"].shape
+    E = cfg.E
+    I = np.asarray(inp["W1q"][0]).shape[0]
+    idx, w, _ = route(cfg, inp["x"], inp["Wg"], inp["bias"], inp["token_ids"], nthreads)
+    k = idx.shape[1]
+    rows_cap = -(-(T * k + E * (GROUP - 1)) // GROUP) * GROUP
+    cap = capacity(T, k, E, cfg.cap_num, cfg.cap_den)
+    d = dispatch(idx, E, cap, 0, GROUP, 0, rows_cap)
+    slot_row, offsets, kept, row_src = d["slot_row"], d["offsets"], d["kept"], d["row_src"]
+    xq, xs = quant_rows(x32)
+    Wg = np.asarray(inp["Wg"], np.float64)
+
+    def rows_chain(e, rows):
+        """Expert e on some of its rows (grouped-layout indices): the forward's h and o, then dO, dh, a | b,
+        g and the dx rows, as `backward` computes them row by row."""
+        rows = np.asarray(rows, np.int64)
+        n = rows.size
+        slots = row_src[rows]
+        toks = slots // k
+        hq, hs, o = expert_rows(xq[toks], xs[toks], inp["W1q"][e], inp["S1"][e], inp["W3q"][e], inp["S3"][e],
+                                inp["W2q"][e], inp["S2"][e], nthreads)
+        dO = np.float32(w[toks, slots % k])[:, None] * dy[toks]
+        dOq, dOs = quant_rows(dO.astype(np.float32))
+        gi = np.array([0, n], np.int32)
+        W13, S13 = _w13_of(inp, e, I, H)
+        W2 = np.asarray(inp["W2q"][e])
+        S2 = np.asarray(inp["S2"][e])
+        W2T, S2T = np.ascontiguousarray(W2.T)[None], np.ascontiguousarray(S2.T)[None]
+        W13T, S13T = np.ascontiguousarray(W13.T)[None], np.ascontiguousarray(S13.T)[None]
+        dh, _ = grouped_gemm(0, 1, I, H, dOq, np.ascontiguousarray(dOs.T), gi, n, W2T, S2T, 0, nthreads)
+        ab, _ = grouped_gemm(0, 1, 2 * I, H, xq[toks], np.ascontiguousarray(xs[toks].T), gi, n, W13[None],
+                             S13[None], 0, nthreads)
+        abf = bf16_bits_to_f32(ab).reshape(n, I // GROUP, 2, GROUP)
+        dhf = bf16_bits_to_f32(dh).reshape(n, I // GROUP, GROUP)
+        da, dbb = swiglu_backward(abf[:, :, 0], abf[:, :, 1], dhf)
+        gf = bf16_bits_to_f32(f64_to_bf16_bits(np.stack((da, dbb), axis=2).reshape(n, 2 * I)))
+        gq, gs = quant_rows(gf)
+        dxr, _ = grouped_gemm(0, 1, H, 2 * I, gq, np.ascontiguousarray(gs.T), gi, n, W13T, S13T, 0, nthreads)
+        hf = (e4m3_decode_array(hq).astype(np.float32) * np.repeat(hs, GROUP, axis=1)).astype(np.float32)
+        xf = (e4m3_decode_array(xq[toks]).astype(np.float32) * np.repeat(xs[toks], GROUP, axis=1)).astype(np.float32)
+        return dict(o=o, dO=dO.astype(np.float32), h=hf, g=gf, x=xf, dxr=dxr)
+
+    dx = {}
+    for t in np.asarray(tokens, np.int64):
+        t = int(t)
+        dw = np.zeros((1, k), np.float64)
+        dxr_rows = {}
+        for j in range(k):
+            r = int(slot_row[t * k + j])
+            if r < 0:
+                continue
+            c = rows_chain(int(idx[t, j]), [r])
+            dw[0, j] = np.dot(dy[t].astype(np.float64), bf16_bits_to_f32(c["o"][0]).astype(np.float64))
+            dxr_rows[j] = bf16_bits_to_f32(c["dxr"][0]).astype(np.float64)
+        dl = router_backward(w[t:t + 1], dw.astype(np.float32)).astype(np.float32)
+        acc = np.zeros(H, np.float64)
+        for j in range(k):
+            acc += float(dl[0, j]) * Wg[int(idx[t, j])]
+        for j in range(k):
+            if j in dxr_rows:
+                acc += dxr_rows[j]
+        dx[t] = f64_to_bf16_bits(acc)
+    dW13, dW2 = {}, {}
+    for e in experts:
+        e = int(e)
+        a0, n = int(offsets[e]), int(kept[e])
+        pad = int(offsets[e + 1]) - a0
+        if n == 0:
+            dW13[e] = np.zeros((2 * I, H), np.uint16)
+            dW2[e] = np.zeros((H, I), np.uint16)
+            continue
+        c = rows_chain(e, np.arange(a0, a0 + n))
+        off1, kept1 = np.array([0, pad], np.int32), np.array([n], np.int32)
+
+        def padded(v):
+            out = np.zeros((pad, v.shape[1]), np.float32)
+            out[:n] = v
+            return out
+        A2 = _deq_tiles(*tile_transpose_quant(padded(c["dO"]), off1, kept1, "row"))
+        B2 = _deq_tiles(*tile_transpose_quant(padded(c["h"]), off1, kept1, "block"))
+        A13 = _deq_tiles(*tile_transpose_quant(padded(c["g"]), off1, kept1, "row"))
+        B13 = _deq_tiles(*tile_transpose_quant(padded(c["x"]), off1, kept1, "block"))
+        acc2 = np.zeros((H, I), np.float64)
+        acc13 = np.zeros((2 * I, H), np.float64)
+        for m in range(pad // GROUP):
+            acc2 += A2[m].astype(np.float64) @ B2[m].astype(np.float64).T
+            acc13 += A13[m].astype(np.float64) @ B13[m].astype(np.float64).T
+        dW2[e] = f64_to_bf16_bits(acc2)
+        dW13[e] = f64_to_bf16_bits(acc13)
+    return dict(dx=dx, dW13=dW13, dW2=dW2, slot_row=slot_row, offsets=offsets, kept=kept)

@@ -144,3 +144,21 @@ def test_whole_backward_within_fp8_error_of_unquantised_autograd(bwd):
         assert rel(dW13[:, 0].reshape(I, H), W1[e].grad.numpy()) < tol, e
         assert rel(dW13[:, 1].reshape(I, H), W3[e].grad.numpy()) < tol, e
         assert rel(bf(r["dW2"][e]), W2[e].grad.numpy()) < tol, e
+
+
+def test_sampled_backward_equals_the_whole_one():
+    # the restricted form the full-size GPU check uses: dx of some tokens and the weight gradients of some
+    # experts, each equal bit for bit to the whole backward's (same routines, same order, on fewer rows)
+    cfg = CFG_TILES
+    inp, d, dy = _inputs(cfg)
+    full = oracle.backward(cfg, d, dy)
+    f = full["forward"]
+    dropped_tok = int(np.nonzero((f["slot_row"] < 0).reshape(cfg.T, cfg.k).any(axis=1))[0][0])
+    tokens = [0, 7, dropped_tok, cfg.T - 1]                        # one of them has a slot dropped
+    experts = [int(np.argmax(f["kept"])), 3]
+    s = oracle.backward_sampled(cfg, d, dy, tokens, experts)
+    for t in tokens:
+        assert np.array_equal(s["dx"][t], full["dx"][t]), t
+    for e in experts:
+        assert np.array_equal(s["dW13"][e], full["dW13"][e]), e
+        assert np.array_equal(s["dW2"][e], full["dW2"][e]), e
