@@ -297,7 +297,9 @@ def time_backward(layer, cfg, steps):
         return e0.elapsed_time(e1) / n
 
     fwd_ms = timed(fwd_train, steps)           # leaves the last training forward's state in tws
+    torch.cuda.nvtx.range_push("backward")     # lets a profiler select this leg's launches (ncu --nvtx)
     ms = timed(call, steps)
+    torch.cuda.nvtx.range_pop()
     assert api.moe_get_device_status() == api.MOE_OK
     Rk = int(layer.kept.sum().item()) if hasattr(layer.kept, "sum") else 0
     # FP8 tensor work: dh (H x I), dx rows (H x 2I), dW2 (H x I), dW13 (2I x H), each 2 FLOP per

@@ -10,8 +10,8 @@ import torch
 
 import oracle
 from fp8_grouped_gemm_fp32_b200 import api
-from fp8_grouped_gemm_fp32_b200.inputs import MoeConfig, interleave_w13, make_inputs, transpose_weights
-from gpu_helpers import assert_close_bf16, ensure_lib, to_np
+from fp8_grouped_gemm_fp32_b200.inputs import CONFIGS, MoeConfig, interleave_w13, make_inputs, transpose_weights
+from gpu_helpers import assert_close_bf16, ensure_lib, gpu_inputs, oracle_inputs, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -76,3 +76,48 @@ def test_backward_matches_oracle(name):
     assert_close_bf16(to_np(dW2).reshape(E, -1), ref["dW2"].reshape(E, -1), "dW2")
     if name == "tiles":
         assert int(np.max(f["kept"])) > 256                           # some expert spans three row tiles
+
+
+def test_backward_full_size_sampled():
+    # the prefill workload at full size, as the benchmark runs it (moe_forward_train, then moe_backward
+    # reading the kept gate and up values): one token's dx row and one expert's whole weight gradients against
+    # the oracle's backward restricted to those outputs (a few minutes of CPU: each of the token's eight
+    # slots runs the oracle's GEMMs with a whole expert's weights)
+    ensure_lib()
+    cfg = CONFIGS["prefill"]
+    inp = gpu_inputs(cfg, on_device=True)
+    c = api.Config.from_moe(cfg)
+    dev = "cuda"
+    T, k, H, E, I = cfg.T, cfg.k, cfg.H, cfg.E, cfg.I
+    g = torch.Generator(device=dev).manual_seed(17)
+    dy = (torch.randn(T, H, generator=g, device=dev) * 0.1).to(torch.bfloat16)
+    W13, S13 = interleave_w13(inp.W1q, inp.S1, inp.W3q, inp.S3)
+    W13T, S13T, W2T, S2T = transpose_weights(W13, S13, inp.W2q, inp.S2)
+    z = lambda *shape, dt: torch.empty(*shape, dtype=dt, device=dev)
+    y, idx, w = z(T, H, dt=torch.bfloat16), z(T, k, dt=torch.int32), z(T, k, dt=torch.float32)
+    counts, slot_row = z(E, dt=torch.int32), z(T * k, dt=torch.int32)
+    fws = z(api.moe_workspace_size(c, 2), dt=torch.uint8)
+    api.moe_forward_train(c, inp.x, inp.Wg, inp.bias, inp.token_ids, W13, S13, inp.W2q, inp.S2, y, idx, w, counts,
+                          slot_row, fws)
+    dx, dWg, db = z(T, H, dt=torch.bfloat16), z(E, H, dt=torch.float32), z(E, dt=torch.float32)
+    dW13, dW2 = z(E, 2 * I, H, dt=torch.bfloat16), z(E, H, I, dt=torch.bfloat16)
+    bws = z(api.moe_backward_workspace_size(c), dt=torch.uint8)
+    api.moe_backward(c, inp.x, inp.Wg, W13, S13, W13T, S13T, W2T, S2T, idx, w, slot_row, fws, dy, dx, dWg, db, dW13,
+                     dW2, bws, fwd_train=True)
+    torch.cuda.synchronize()
+    assert api.moe_get_device_status() == api.MOE_OK
+    del W13T, S13T, W2T, S2T, bws
+    oin = oracle_inputs(inp)
+    # the sampled outputs are chosen from the oracle's own routing: the expert with the most rows, and the
+    # first token routed to it
+    idx_o, _, _ = oracle.route(cfg, oin["x"], oin["Wg"], oin["bias"], oin["token_ids"])
+    counts_o = np.bincount(idx_o.reshape(-1), minlength=E)
+    assert np.array_equal(to_np(counts), counts_o)
+    e = int(np.argmax(counts_o))
+    assert -(-int(counts_o[e]) // 128) >= 3                            # three or more 128-row tiles
+    t = int(np.nonzero((idx_o == e).any(axis=1))[0][0])
+    ref = oracle.backward_sampled(cfg, oin, to_np(dy), [t], [e])
+    assert np.array_equal(to_np(slot_row), ref["slot_row"])
+    assert_close_bf16(to_np(dx[t]), ref["dx"][t], f"dx[{t}]")
+    assert_close_bf16(to_np(dW13[e]), ref["dW13"][e], f"dW13[{e}]")
+    assert_close_bf16(to_np(dW2[e]), ref["dW2"][e], f"dW2[{e}]")
