@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/moe_fp8.h"
+#include "backward.cuh"
 #include "common.cuh"
 
 namespace moe {
@@ -39,15 +40,6 @@ cudaError_t launch_grouped_gemm_kgroup(int E, int M, int N, const uint8_t* A, co
 cudaError_t launch_slot_lists(const int32_t* topk_idx, int T, int k, int E, int32_t* counts, int32_t* offsets,
                               int32_t* list, int32_t* slot_tmp, void* scratch, int* status, cudaStream_t s);
 size_t ep_scratch_bytes(int T, int E);
-struct TqArgs {
-    const uint16_t* dy;
-    const float* topk_w;
-    const uint8_t* codes;
-    const float* scales;
-    const uint16_t* bf;
-    const int32_t* row_src;
-    int rows, k, C;
-};
 cudaError_t launch_bwd_dl(const uint16_t* dy, const uint16_t* O, const int32_t* slot_row, const float* topk_w, int T,
                           int k, int H, float* dl, cudaStream_t s);
 cudaError_t launch_bwd_dout(const uint16_t* dy, const float* topk_w, const int32_t* row_src, int rows, int k, int H,

@@ -14,6 +14,7 @@
 //           db[e] = sum of dl, all in token order (dropped slots included: their logits still moved w).
 // The quantisation steps of the forward pass pass the gradient through; selection and capacity are held.
 #include "../../include/moe_fp8.h"
+#include "backward.cuh"
 #include "common.cuh"
 
 #include <type_traits>
@@ -214,19 +215,6 @@ __global__ void __launch_bounds__(256) bwd_swiglu_kernel(const uint16_t* __restr
         }
     }
 }
-
-// Sources of the transposed quantisation: the value of row r, column c of an activation-like matrix.
-enum TqSource { kTqDout = 0, kTqFp8 = 1, kTqBf16 = 2 };
-
-struct TqArgs {
-    const uint16_t* dy;       // kTqDout: w * dy of the row's slot
-    const float* topk_w;
-    const uint8_t* codes;     // kTqFp8: codes [rows, C] with scales [C/128][rows]
-    const float* scales;
-    const uint16_t* bf;       // kTqBf16: [rows, C]
-    const int32_t* row_src;   // the forward layout's rows: slot, or -1 for padding (value 0)
-    int rows, k, C;
-};
 
 // For forward row tile m (blockIdx.x) and column block cb (blockIdx.y): the transposed 128 x 128 block
 // quantised. ROWS: one scale per transposed row (column c over the tile's 128 rows), out scales [tiles][C];
