@@ -257,7 +257,11 @@ size_t moe_rows_capacity(const moe_config_t* cfg) {
 }
 
 size_t moe_workspace_size(const moe_config_t* cfg, int for_forward) {
-    if (check_cfg(cfg) != MOE_OK) return 0;
+    if (check_cfg(cfg) != MOE_OK || for_forward < 0 || for_forward > 2) return 0;
+    // the training forward takes what the backward takes: contiguous layout, E4M3 weights, softmax routing
+    if (for_forward == 2 && (cfg->layout != MOE_LAYOUT_CONTIGUOUS || cfg->weights != MOE_WEIGHTS_FP8 ||
+                             cfg->routing != MOE_ROUTE_SOFTMAX_TOPK))
+        return 0;
     if (for_forward) return carve(cfg, nullptr, for_forward == 2).total;
     return std::max(route_scratch(cfg), align_up(permute_scratch_bytes(cfg->T, cfg->E)));
 }

@@ -94,7 +94,9 @@ size_t moe_rows_capacity(const moe_config_t* cfg);
 /* Scratch bytes moe_route and moe_permute need (ws_bytes >= this); with
  * for_forward = 1 the bytes moe_forward needs, with for_forward = 2 those of
  * moe_forward_train (the same plus the saved gate and up values, 4 I bytes per
- * row). 0 on a bad config. */
+ * row). 0 on a bad config, on for_forward outside 0..2, and with for_forward = 2
+ * on a configuration moe_forward_train does not take (masked layout, 4-bit
+ * weights or hash routing). */
 size_t moe_workspace_size(const moe_config_t* cfg, int for_forward);
 
 /*

@@ -159,3 +159,41 @@ def test_ep_plan_struct_layout_matches_the_header(tmp_path):
     got = [int(v) for v in subprocess.check_output([str(exe)]).split()]
     assert got[0] == ctypes.sizeof(ep.EpPlan)
     assert got[1:] == [getattr(ep.EpPlan, f).offset for f in fields]
+
+
+def test_training_workspace_only_for_what_the_training_forward_takes(L):
+    prefill = api.Config.from_moe(CONFIGS["prefill"])
+    rows = api.moe_rows_capacity(prefill)
+    # the training forward keeps the gate and up values: 2 I bf16 values, 4 I bytes, per row
+    assert api.moe_workspace_size(prefill, 2) >= api.moe_workspace_size(prefill, 1) + 4 * 2048 * rows
+    for name in ("decode", "decode_hash", "decode_w4"):                # masked, hash, 4-bit: no backward
+        assert api.moe_workspace_size(api.Config.from_moe(CONFIGS[name]), 2) == 0, name
+        assert api.moe_workspace_size(api.Config.from_moe(CONFIGS[name]), 1) > 0, name
+    assert L.moe_workspace_size(ctypes.byref(prefill), 3) == 0
+    assert L.moe_workspace_size(ctypes.byref(prefill), -1) == 0
+
+
+@pytest.mark.parametrize("name", ["decode", "decode_hash", "decode_w4"])
+def test_training_calls_reject_what_the_backward_does_not_take(L, name):
+    # returned before the device is queried: no GPU needed, no pointer read
+    c = api.Config.from_moe(CONFIGS[name])
+    p = None
+    st = L.moe_forward_train(ctypes.byref(c), *([p] * 14), 0, None)
+    assert st == api.MOE_ERR_UNSUPPORTED_SHAPE
+    st = L.moe_backward(ctypes.byref(c), *([p] * 12), 1, *([p] * 7), 0, None)
+    assert st == api.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+def test_backward_rejects_experts_beyond_its_k_limit(L):
+    # an expert's rows are the K of its weight-gradient GEMMs, at most 16384; without a capacity every
+    # token may reach one expert
+    c = api.Config.from_moe(CONFIGS["prefill"])
+    c.T = 16512
+    assert api.moe_workspace_size(c, 2) > 0                             # a valid forward configuration
+    st = L.moe_backward(ctypes.byref(c), *([None] * 12), 1, *([None] * 7), 0, None)
+    assert st == api.MOE_ERR_UNSUPPORTED_SHAPE
+    # a capacity bounds every expert's rows (ceil(T k / E) = 516 here), so the shape passes; the call then
+    # stops at the device query (no GPU: a CUDA error, or a device other than sm_100) or at the null pointers
+    c.cap_num, c.cap_den = 1, 1
+    st = L.moe_backward(ctypes.byref(c), *([None] * 12), 1, *([None] * 7), 0, None)
+    assert st in (api.MOE_ERR_CUDA, api.MOE_ERR_UNSUPPORTED_DEVICE, api.MOE_ERR_INVALID_ARG)
