@@ -438,8 +438,19 @@ moe_status_t moe_forward_train(const moe_config_t* cfg, const void* x, const flo
                         ws_bytes, stream, true);
 }
 
+// What moe_backward takes beyond a valid configuration: contiguous layout, E4M3 weights, softmax routing, and
+// K of the weight-gradient GEMMs (an expert's rows; 2I for g W13) within the 128 K blocks they stage.
+static moe_status_t check_backward_shape(const moe_config_t* cfg) {
+    if (cfg->layout != MOE_LAYOUT_CONTIGUOUS || cfg->weights != MOE_WEIGHTS_FP8 ||
+        cfg->routing != MOE_ROUTE_SOFTMAX_TOPK)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    const int64_t most = cfg->cap_num ? std::min<int64_t>(cfg->T, capacity_of(cfg)) : cfg->T;
+    if (most > 16384 || 2 * cfg->I > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
 size_t moe_backward_workspace_size(const moe_config_t* cfg) {
-    if (check_cfg(cfg) != MOE_OK) return 0;
+    if (check_cfg(cfg) != MOE_OK || check_backward_shape(cfg) != MOE_OK) return 0;
     return carve_bwd(cfg, nullptr).total;
 }
 
@@ -450,12 +461,7 @@ moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const float* W
                           void* ws, size_t ws_bytes, void* stream) {
     moe_status_t st = check_cfg(cfg);
     if (st != MOE_OK) return st;
-    if (cfg->layout != MOE_LAYOUT_CONTIGUOUS || cfg->weights != MOE_WEIGHTS_FP8 ||
-        cfg->routing != MOE_ROUTE_SOFTMAX_TOPK)
-        return MOE_ERR_UNSUPPORTED_SHAPE;
-    // the weight-gradient GEMM stages at most 128 K blocks per expert: 16384 rows
-    const int64_t most = cfg->cap_num ? std::min<int64_t>(cfg->T, capacity_of(cfg)) : cfg->T;
-    if (most > 16384 || 2 * cfg->I > 16384) return MOE_ERR_UNSUPPORTED_SHAPE;   // K of g W13 is 2I
+    if ((st = check_backward_shape(cfg)) != MOE_OK) return st;
     DeviceInfo* dev;
     if ((st = device_info(&dev)) != MOE_OK) return st;
     if (cfg->T == 0) return MOE_OK;

@@ -317,6 +317,8 @@ moe_status_t moe_permute_noalloc(const moe_config_t* cfg, const void* x, const i
  * Contiguous layout, E4M3 weights and softmax routing only
  * (MOE_ERR_UNSUPPORTED_SHAPE otherwise), I at most 8192, and at most 16384
  * rows per expert (T, or the capacity when smaller).
+ * moe_backward_workspace_size gives 0 on a bad configuration and on one that
+ * moe_backward rejects.
  */
 size_t moe_backward_workspace_size(const moe_config_t* cfg);
 moe_status_t moe_backward(const moe_config_t* cfg, const void* x, const float* Wg, const uint8_t* W13, const float* S13,

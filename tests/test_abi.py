@@ -180,6 +180,7 @@ def test_training_calls_reject_what_the_backward_does_not_take(L, name):
     p = None
     st = L.moe_forward_train(ctypes.byref(c), *([p] * 14), 0, None)
     assert st == api.MOE_ERR_UNSUPPORTED_SHAPE
+    assert api.moe_backward_workspace_size(c) == 0
     st = L.moe_backward(ctypes.byref(c), *([p] * 12), 1, *([p] * 7), 0, None)
     assert st == api.MOE_ERR_UNSUPPORTED_SHAPE
 
@@ -190,10 +191,12 @@ def test_backward_rejects_experts_beyond_its_k_limit(L):
     c = api.Config.from_moe(CONFIGS["prefill"])
     c.T = 16512
     assert api.moe_workspace_size(c, 2) > 0                             # a valid forward configuration
+    assert api.moe_backward_workspace_size(c) == 0
     st = L.moe_backward(ctypes.byref(c), *([None] * 12), 1, *([None] * 7), 0, None)
     assert st == api.MOE_ERR_UNSUPPORTED_SHAPE
     # a capacity bounds every expert's rows (ceil(T k / E) = 516 here), so the shape passes; the call then
     # stops at the device query (no GPU: a CUDA error, or a device other than sm_100) or at the null pointers
     c.cap_num, c.cap_den = 1, 1
+    assert api.moe_backward_workspace_size(c) > 0
     st = L.moe_backward(ctypes.byref(c), *([None] * 12), 1, *([None] * 7), 0, None)
     assert st in (api.MOE_ERR_CUDA, api.MOE_ERR_UNSUPPORTED_DEVICE, api.MOE_ERR_INVALID_ARG)
